@@ -1,0 +1,82 @@
+"""Oracle FP8 linear layer: forward, dX and dW, delayed or dynamic scaling.
+
+Test infrastructure only (see ``oracle/__init__.py``).
+
+What the pages fix (AstrAI compare view, ``astrai/extension/fp8.py``):
+
+* ``fp8_linear_forward``: delayed scaling snapshots ``sx, sw`` from the rings
+  before the quantize kernels fold the fresh amax and publish the next step;
+  the GEMM dequantizes with ``sx * sw`` and fuses the bias.  Dynamic scaling
+  measures the current amax of x and w first, with no ring.
+* ``_LinearFp8.backward``: g is quantized once in both orientations
+  (``quantize_dual``, folding into the g ring); x and w are re-quantized
+  *transposed* with the forward's steps (no ring, amax discarded);
+  ``grad_x = g8 @ w8T^T * (sg*sw)`` and ``grad_w = g8T @ x8T^T * (sg*sx)`` both in
+  the NT layout; ``grad_b = g.sum(0)``.  Dynamic backward re-measures g, w and x.
+* ``FP8Format.HYBRID``: E4M3 forward, E5M2 backward; the backward GEMM takes both
+  operands in one format, so x and w are re-quantized to E5M2 as well.
+
+Readings: ``grad_b`` is the fp64 column sum rounded once to bf16; the gradient
+outputs are returned unrounded (fp64) for the bound check.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .fp8_codec import bf16_bits_to_f64, round_to_bf16
+from .gemm import gemm_ref
+from .quantize import quantize, quantize_dual, quantize_transposed
+from .scaling import Ring, dynamic_scale
+
+
+def forward(x_bits, w_bits, bias_bits=None, fmt="e4m3", ring_x: Ring = None,
+            ring_w: Ring = None, margin: int = 0):
+    """Returns a dict with ``y`` (fp64, unrounded), ``s_abs``, ``sc``, ``x8``, ``w8``,
+    ``sx``, ``sw``, ``amax_x``, ``amax_w``.  Rings (if given) are folded in place;
+    the caller advances them afterwards, as the pages' host code does."""
+    xv = bf16_bits_to_f64(x_bits).astype(np.float32)
+    wv = bf16_bits_to_f64(w_bits).astype(np.float32)
+    dynamic = ring_x is None
+    if dynamic:
+        sx = dynamic_scale(xv, fmt, margin)
+        sw = dynamic_scale(wv, fmt, margin)
+    else:
+        sx = np.float32(ring_x.scale)
+        sw = np.float32(ring_w.scale)
+    x8, ax = quantize(xv, sx, fmt)
+    w8, aw = quantize(wv, sw, fmt)
+    if not dynamic:
+        ring_x.fold(ax, sx)
+        ring_w.fold(aw, sw)
+    y, s_abs, sc = gemm_ref(x8, w8, "NT", fmt, fmt, sx, sw, bias_bits)
+    return dict(y=y, s_abs=s_abs, sc=sc, x8=x8, w8=w8, sx=sx, sw=sw,
+                amax_x=ax, amax_w=aw)
+
+
+def backward(g_bits, x_bits, w_bits, fmt="e5m2", sx_fwd=None, sw_fwd=None,
+             ring_g: Ring = None, margin: int = 0):
+    """Returns a dict with ``dx``, ``dw`` (fp64, unrounded) and their ``s_abs``/``sc``,
+    ``grad_b`` (bf16 values), the quantized operands and the steps used."""
+    gv = bf16_bits_to_f64(g_bits).astype(np.float32)
+    xv = bf16_bits_to_f64(x_bits).astype(np.float32)
+    wv = bf16_bits_to_f64(w_bits).astype(np.float32)
+    dynamic = ring_g is None
+    if dynamic:
+        sg = dynamic_scale(gv, fmt, margin)
+        sw = dynamic_scale(wv, fmt, margin)
+        sx = dynamic_scale(xv, fmt, margin)
+    else:
+        sg = np.float32(ring_g.scale)
+        sx, sw = np.float32(sx_fwd), np.float32(sw_fwd)
+    g8, g8t, ag = quantize_dual(gv, sg, fmt)
+    if not dynamic:
+        ring_g.fold(ag, sg)
+    x8t, _ = quantize_transposed(xv, sx, fmt)
+    w8t, _ = quantize_transposed(wv, sw, fmt)
+    dx, dx_abs, dx_sc = gemm_ref(g8, w8t, "NT", fmt, fmt, sg, sw)
+    dw, dw_abs, dw_sc = gemm_ref(g8t, x8t, "NT", fmt, fmt, sg, sx)
+    grad_b = round_to_bf16(np.sum(gv.astype(np.float64), axis=0))
+    return dict(dx=dx, dx_abs=dx_abs, dx_sc=dx_sc, dw=dw, dw_abs=dw_abs, dw_sc=dw_sc,
+                grad_b=grad_b, g8=g8, g8t=g8t, x8t=x8t, w8t=w8t, sg=sg, sx=sx, sw=sw,
+                amax_g=ag)

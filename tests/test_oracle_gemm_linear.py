@@ -1,0 +1,206 @@
+"""Pins for the oracle's GEMM and linear compositions (no GPU).
+
+Sources: AstrAI compare view -- ``astrai/extension/ops/fp8.py`` (``mm_fp8``:
+``a @ b * scale (+ bias)``, 2-D / 3-D with batch broadcast),
+``csrc/kernels/fp8/gemm/epilogue.cuh`` (bias added to the fp32 accumulator before
+one bf16 rounding), ``csrc/kernels/fp8/common.h`` (layout tags) and
+``astrai/extension/fp8.py`` (``_LinearFp8``: NT routing of forward, dX, dW).
+The GEMM is pinned against an exact-rational brute-force triple loop, layout
+equivalences, one-hot and zero operands, and the batch broadcast rule.
+"""
+
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import fp8_codec as C
+from oracle import gemm as G
+from oracle import linear as L
+from oracle import quantize as Q
+from oracle import scaling as S
+
+
+def _rand_codes(rng, shape, fmt):
+    """Random finite fp8 codes (all magnitudes, both signs)."""
+    tab = C.decode_table(fmt)
+    finite = np.array([c for c in range(256) if np.isfinite(tab[c])], np.uint8)
+    return rng.choice(finite, size=shape)
+
+
+def _brute(a_codes, b_codes, fmt_a, fmt_b, sa, sb, bias_bits):
+    """Exact rational A[M,K] @ B[K,N] * RN32(sa*sb) + bias, triple loop."""
+    m, k = a_codes.shape
+    n = b_codes.shape[1]
+    sc = Fraction(float(np.float32(sa) * np.float32(sb)))
+    out = np.zeros((m, n), dtype=object)
+    for i in range(m):
+        for j in range(n):
+            acc = Fraction(0)
+            for p in range(k):
+                acc += Fraction(C.decode_code(int(a_codes[i, p]), fmt_a)) * \
+                    Fraction(C.decode_code(int(b_codes[p, j]), fmt_b))
+            v = acc * sc
+            if bias_bits is not None:
+                v += Fraction(float(C.bf16_bits_to_f64(bias_bits[j:j + 1])[0]))
+            out[i, j] = v
+    return out
+
+
+@pytest.mark.parametrize("fmt_a,fmt_b", [("e4m3", "e4m3"), ("e5m2", "e5m2"), ("e5m2", "e4m3")])
+def test_gemm_equals_exact_brute_force(fmt_a, fmt_b):
+    rng = np.random.default_rng(21)
+    for m, n, k in ((1, 1, 1), (3, 5, 7), (16, 16, 16), (9, 4, 13)):
+        a = _rand_codes(rng, (m, k), fmt_a)
+        b = _rand_codes(rng, (k, n), fmt_b)
+        bias = C.f64_to_bf16_bits(rng.standard_normal(n))
+        ref, s_abs, sc = G.gemm_ref(a, b, "NN", fmt_a, fmt_b, 0.75, 1.3, bias)
+        exact = _brute(a, b, fmt_a, fmt_b, 0.75, 1.3, bias)
+        for i in range(m):
+            for j in range(n):
+                # one fp64 rounding for the scale product and one for the bias
+                # add, each relative to the magnitudes involved
+                mag = Fraction(float(s_abs[i, j])) * Fraction(float(sc)) + \
+                    abs(Fraction(float(C.bf16_bits_to_f64(bias[j:j + 1])[0])))
+                tol = mag * Fraction(2) ** -51
+                if not fmt_a == fmt_b == "e4m3":
+                    # E5M2 partial sums may round in fp64
+                    tol += Fraction(2) ** -45 * Fraction(float(s_abs[i, j])) * Fraction(float(sc))
+                assert abs(Fraction(ref[i, j]) - exact[i, j]) <= tol
+
+
+def test_e4m3_accumulation_is_order_independent_at_k8192():
+    """E4M3 partial sums are multiples of 2^-18 below 2^31, so fp64 is exact."""
+    rng = np.random.default_rng(4)
+    k = 8192
+    a = _rand_codes(rng, (1, k), "e4m3")
+    b = _rand_codes(rng, (k, 1), "e4m3")
+    av = C.decode(a, "e4m3")[0]
+    bv = C.decode(b, "e4m3")[:, 0]
+    scaled = [int(x * 2 ** 9) * int(y * 2 ** 9) for x, y in zip(av, bv)]
+    exact = Fraction(sum(scaled), 2 ** 18)
+    ref, _, _ = G.gemm_ref(a, b, "NN", sa=1.0, sb=1.0)
+    assert Fraction(ref[0, 0]) == exact
+    assert Fraction(float(np.sum(av[::-1] * bv[::-1]))) == exact
+
+
+def test_layouts_are_equivalent():
+    rng = np.random.default_rng(8)
+    a = _rand_codes(rng, (24, 40), "e4m3")   # [M][K]
+    b = _rand_codes(rng, (40, 17), "e4m3")   # [K][N]
+    ref, _, _ = G.gemm_ref(a, b, "NN", sa=0.5, sb=2.0)
+    for layout, a_st, b_st in (("NT", a, b.T), ("TN", a.T, b), ("TT", a.T, b.T)):
+        got, _, _ = G.gemm_ref(np.ascontiguousarray(a_st), np.ascontiguousarray(b_st),
+                               layout, sa=0.5, sb=2.0)
+        assert np.array_equal(got, ref), layout
+
+
+def test_one_hot_rows_copy_columns_and_zero_gives_bias():
+    rng = np.random.default_rng(1)
+    k, n = 32, 20
+    b = _rand_codes(rng, (n, k), "e4m3")  # stored [N][K] (NT)
+    one = C.encode(np.array([1.0]), "e4m3")[0]
+    a = np.zeros((k, k), np.uint8)
+    a[np.arange(k), np.arange(k)] = one
+    bias = C.f64_to_bf16_bits(rng.standard_normal(n))
+    ref, _, sc = G.gemm_ref(a, b, "NT", sa=1.0, sb=1.0, bias=bias)
+    want = C.decode(b, "e4m3").T + C.bf16_bits_to_f64(bias)[None, :]
+    assert np.array_equal(ref, want)
+    zero = np.zeros((5, k), np.uint8)
+    ref0, s_abs0, _ = G.gemm_ref(zero, b, "NT", sa=3.0, sb=7.0, bias=bias)
+    assert np.array_equal(ref0, np.broadcast_to(C.bf16_bits_to_f64(bias), (5, n)))
+    assert np.all(s_abs0 == 0)
+
+
+def test_batch_broadcast_and_entry():
+    rng = np.random.default_rng(2)
+    a = _rand_codes(rng, (3, 8, 16), "e4m3")
+    b = _rand_codes(rng, (1, 12, 16), "e4m3")  # one B shared by every batch
+    ref, s_abs, sc = G.gemm_ref(a, b, "NT", sa=1.5, sb=0.5)
+    assert ref.shape == (3, 8, 12)
+    for i in range(3):
+        r_i, _, _ = G.gemm_ref(a[i], b[0], "NT", sa=1.5, sb=0.5)
+        assert np.array_equal(ref[i], r_i)
+        e, e_abs, _ = G.gemm_entry(a, b, "NT", "e4m3", "e4m3", 1.5, 0.5, None, None, i, 5, 7)
+        assert e == ref[i, 5, 7] and e_abs == s_abs[i, 5, 7]
+
+
+def test_fp8_bias_with_scale():
+    rng = np.random.default_rng(3)
+    a = _rand_codes(rng, (4, 8), "e4m3")
+    b = _rand_codes(rng, (6, 8), "e4m3")
+    b8 = _rand_codes(rng, (6,), "e4m3")
+    ref, _, sc = G.gemm_ref(a, b, "NT", sa=1.0, sb=1.0, bias=b8, bias_scale=0.125)
+    plain, _, _ = G.gemm_ref(a, b, "NT", sa=1.0, sb=1.0)
+    assert np.array_equal(ref - plain, np.broadcast_to(C.decode(b8, "e4m3") * 0.125, (4, 6)))
+
+
+def test_tolerance_formula():
+    ref = np.array([1.0, -2.0, 0.0])
+    s_abs = np.array([4.0, 4.0, 1024.0])
+    tol = G.gemm_tolerance(ref, s_abs, np.float32(0.5))
+    assert np.allclose(tol, [2 ** -8 + 2 ** -19, 2 ** -7 + 2 ** -19, 2 ** -11])
+
+
+def _bits(x):
+    return C.f64_to_bf16_bits(np.asarray(x, np.float64))
+
+
+def test_linear_forward_dynamic_close_to_fp64():
+    rng = np.random.default_rng(0)
+    x = _bits(rng.standard_normal((64, 128)))
+    w = _bits(rng.standard_normal((96, 128)) * 0.02)
+    b = _bits(rng.standard_normal(96) * 0.1)
+    out = L.forward(x, w, b, "e4m3")
+    exact = C.bf16_bits_to_f64(x) @ C.bf16_bits_to_f64(w).T + C.bf16_bits_to_f64(b)
+    err = np.abs(out["y"] - exact)
+    # each product carries <= 2 * 2^-4 relative quantization error
+    bound = 2 * 2.0 ** -4 * (np.abs(C.bf16_bits_to_f64(x)) @ np.abs(C.bf16_bits_to_f64(w)).T) + 1e-6
+    assert np.all(err <= bound)
+    assert out["sx"] == S.dynamic_scale(C.bf16_bits_to_f64(x).astype(np.float32), "e4m3")
+
+
+def test_linear_backward_routes_and_grad_bias():
+    rng = np.random.default_rng(5)
+    m, k, n = 48, 32, 40
+    g = _bits(rng.standard_normal((m, n)) * 1e-3)
+    x = _bits(rng.standard_normal((m, k)))
+    w = _bits(rng.standard_normal((n, k)) * 0.02)
+    out = L.backward(g, x, w, "e5m2")
+    gv, xv, wv = (C.bf16_bits_to_f64(t) for t in (g, x, w))
+    # the NT routing computes g @ w and g^T @ x on the quantized operands
+    g8 = C.decode(out["g8"], "e5m2") * float(out["sg"])
+    w8 = C.decode(out["w8t"], "e5m2").T * float(out["sw"])
+    x8 = C.decode(out["x8t"], "e5m2").T * float(out["sx"])
+    sc_dx = float(np.float32(out["sg"]) * np.float32(out["sw"]))
+    assert np.allclose(out["dx"], (C.decode(out["g8"], "e5m2") @ C.decode(out["w8t"], "e5m2").T) * sc_dx)
+    assert np.allclose(out["dx"], g8 @ w8, rtol=1e-6, atol=1e-12)
+    assert np.allclose(out["dw"], g8.T @ x8, rtol=1e-6, atol=1e-12)
+    # and against full precision within E5M2's 2^-3 relative step per operand
+    assert np.all(np.abs(out["dx"] - gv @ wv) <= 2 * 2.0 ** -3 * (np.abs(gv) @ np.abs(wv)) + 1e-9)
+    assert np.array_equal(out["grad_b"], C.round_to_bf16(gv.sum(0)))
+
+
+def test_delayed_linear_sequence_and_backward_reuses_forward_steps():
+    rng = np.random.default_rng(12)
+    m, k, n = 32, 64, 48
+    w = _bits(rng.standard_normal((n, k)) * 0.02)
+    rx, rw = S.Ring(16, "e4m3"), S.Ring(16, "e4m3")
+    rg = S.Ring(16, "e5m2")
+    amax_hist = []
+    for t in range(6):
+        x = _bits(rng.standard_normal((m, k)) * 2.0 ** rng.uniform(-4, 4))
+        g = _bits(rng.standard_normal((m, n)) * 1e-3)
+        if t == 0:
+            rx.seed(C.bf16_bits_to_f64(x).astype(np.float32))
+            rw.seed(C.bf16_bits_to_f64(w).astype(np.float32))
+            rg.seed(C.bf16_bits_to_f64(g).astype(np.float32))
+        sx_before = rx.scale
+        fwd = L.forward(x, w, None, "e4m3", rx, rw)
+        assert fwd["sx"] == sx_before and rx.scale_used == sx_before
+        amax_hist.append(fwd["amax_x"])
+        assert rx.scale == np.float32(np.float32(max(amax_hist)) / np.float32(448.0))
+        bwd = L.backward(g, x, w, "e5m2", fwd["sx"], fwd["sw"], rg)
+        assert bwd["sx"] == fwd["sx"] and bwd["sw"] == fwd["sw"]
+        for r in (rx, rw, rg):
+            r.advance()
