@@ -1,0 +1,514 @@
+// FP8 x FP8 -> bf16 GEMM with dequantization and fused bias, on the sm_100a tensor cores.
+//
+// Computes  out[b][i][j] = RN_bf16( acc[b][i][j] * RN32(sa * sb) + bias[j] ),
+//           acc = sum_k A[b][i][k] * B[b][k][j]   (fp32, tcgen05.mma kind::f8f6f4)
+// for the four operand layouts and batched / broadcast operands.  Definition: AstrAI compare
+// view 3e57cc8...main -- astrai/extension/ops/fp8.py (mm_fp8), csrc/kernels/fp8/common.h
+// (RowMajor / ColMajor operand tags, FP8Params batch strides), csrc/kernels/fp8/gemm/
+// epilogue.cuh (bias added to the fp32 accumulator before the single bf16 rounding) and the
+// extension commit log (bias_scale: fp8 bias dequantized after the operand scaling).
+//
+// B200 design (the pages' sm_89 mma.sync / cp.async / ldmatrix design is not used):
+//  * persistent grid, one CTA per SM, grouped-raster static tile schedule;
+//  * warp 0 = TMA producer: 3-D tensor maps (K-major or MN-major), 128-byte swizzle, into a
+//    ring of shared-memory stages guarded by full / empty mbarriers;
+//  * warp 1 = MMA issuer: one thread issues tcgen05.mma (M = 128, N = BN, K = 32) into a
+//    TMEM accumulator; tcgen05.commit releases each stage and, per tile, hands the
+//    accumulator to the epilogue.  Two accumulators (2 x BN TMEM columns) let the epilogue
+//    of tile i overlap the MMAs of tile i + 1;
+//  * warps 2-5 = epilogue: tcgen05.ld 32 columns at a time, fma with the combined scale and
+//    the bias, round to bf16, 128-bit stores;
+//  * every wait is bounded (globaltimer); on expiry the CTA records a status code, drains its
+//    in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+
+namespace fp8dsa {
+namespace {
+
+constexpr int kBM = 128;      // tile rows (TMEM lanes)
+constexpr int kBK = 128;      // K bytes per stage (one 128-byte swizzle row)
+constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
+constexpr int kThreads = 192; // 6 warps
+constexpr int kEpiThreads = 128;
+
+template <int BN>
+struct Cfg {
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kAStage = kBM * kBK;
+    static constexpr int kBStage = BN * kBK;
+    static constexpr int kTmemCols = 2 * BN;
+    static constexpr int kBarBytes = 256;
+    static constexpr int kBiasBytes = 4 * BN * 4;  // one bias copy per epilogue warp
+    static constexpr int kSmem = 1024 + kStages * (kAStage + kBStage) + kBarBytes + kBiasBytes;
+};
+
+struct GemmArgs {
+    int m, n, k;
+    int tiles_m, tiles_n, num_tiles, k_blocks;
+    int a_batched, b_batched;
+    int a_mn, b_mn;
+    uint32_t idesc;
+    uint16_t* out;
+    int64_t ldo, stride_o;
+    int vec_out;
+    const void* bias;
+    int bias_kind;  // 0 none, 1 bf16, 2 fp8 e4m3 * bias_scale, 3 fp8 e5m2 * bias_scale
+    const float* bias_scale;
+    const float* scale_a;
+    const float* scale_b;
+    WaitCtl wait;
+};
+
+// UMMA shared-memory matrix descriptor: 128-byte swizzle, sm_100 descriptor version.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& b, int& tm, int& tn) {
+    constexpr int kGroupM = 8;
+    const int per = g.tiles_m * g.tiles_n;
+    b = tile / per;
+    const int r = tile - b * per;
+    const int group = kGroupM * g.tiles_n;
+    const int gi = r / group;
+    const int first_m = gi * kGroupM;
+    const int gm = min(g.tiles_m - first_m, kGroupM);
+    const int within = r - gi * group;
+    tm = first_m + within % gm;
+    tn = within / gm;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                    const GemmArgs g) {
+    using C = Cfg<BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S * C::kAStage;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::kBStage);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* bias_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(acc_full + a, 1);
+            mbar_init(acc_empty + a, kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tma_a);
+        prefetch_tensormap(&tma_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_parity = 0;  // per-stage: ever issued, parity of the last issue
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
+                int b, tm, tn;
+                decode_tile(tile, g, b, tm, tn);
+                const int ba = g.a_batched ? b : 0;
+                const int bb = g.b_batched ? b : 0;
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(empty + stage, phase ^ 1u, g.wait, abort_flag, kStatusWaitProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full + stage, C::kAStage + C::kBStage);
+                    uint8_t* a_dst = sA + stage * C::kAStage;
+                    uint8_t* b_dst = sB + stage * C::kBStage;
+                    if (!g.a_mn)
+                        tma_load_3d(a_dst, &tma_a, full + stage, kb * kBK, tm * kBM, ba);
+                    else
+                        tma_load_3d(a_dst, &tma_a, full + stage, tm * kBM, kb * kBK, ba);
+                    if (!g.b_mn) {
+                        tma_load_3d(b_dst, &tma_b, full + stage, kb * kBK, tn * BN, bb);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_3d(b_dst + h * 128 * kBK, &tma_b, full + stage, tn * BN + h * 128, kb * kBK, bb);
+                    }
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let every copy already in flight land before the CTA can exit.
+                for (int s = 0; s < S; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait_bounded(full + s, (issued_parity >> s) & 1u, g.wait, nullptr, kStatusWaitDrain);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        bool ok = true;
+        constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
+        for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
+            if (!mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag, kStatusWaitMma)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                if (!mbar_wait_bounded(full + stage, phase, g.wait, abort_flag, kStatusWaitMma)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t a_base = smem_addr(sA + stage * C::kAStage);
+                    const uint32_t b_base = smem_addr(sB + stage * C::kBStage);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                        // K-major: step 32 bytes along the swizzled row; MN-major: step 32 rows.
+                        const uint64_t ad = g.a_mn ? smem_desc(a_base + kk * kUmmaK * 128, C::kAStage, 1024)
+                                                   : smem_desc(a_base + kk * kUmmaK, 16, 1024);
+                        const uint64_t bd = g.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
+                                                   : smem_desc(b_base + kk * kUmmaK, 16, 1024);
+                        umma_f8f6f4(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty + stage);
+                }
+                __syncwarp();
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(acc_full + acc);
+            __syncwarp();
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        // Every MMA this thread issued must complete before TMEM is released.
+        if (lane == 0) {
+            umma_commit(drain);
+            mbar_wait_bounded(drain, 0, g.wait, nullptr, kStatusWaitDrain);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // this warp may access TMEM lanes 32q .. 32q+31
+        const int row_in_tile = q * 32 + lane;
+        float* my_bias = bias_s + (warp - 2) * BN;
+        const float sc = __fmul_rn(__ldg(g.scale_a), __ldg(g.scale_b));
+        const float bsc = g.bias_kind >= 2 ? __ldg(g.bias_scale) : 0.0f;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x) {
+            int b, tm, tn;
+            decode_tile(tile, g, b, tm, tn);
+            const int col0 = tn * BN;
+            // this warp's copy of the tile's bias, as fp32
+            __syncwarp();
+            for (int c = lane; c < BN; c += 32) {
+                const int col = col0 + c;
+                float bv = 0.0f;
+                if (col < g.n) {
+                    if (g.bias_kind == 1)
+                        bv = bf16_bits_to_float(static_cast<const uint16_t*>(g.bias)[col]);
+                    else if (g.bias_kind == 2)
+                        bv = __fmul_rn(fp8_to_float<0>(static_cast<const uint8_t*>(g.bias)[col]), bsc);
+                    else if (g.bias_kind == 3)
+                        bv = __fmul_rn(fp8_to_float<1>(static_cast<const uint8_t*>(g.bias)[col]), bsc);
+                }
+                my_bias[c] = bv;
+            }
+            __syncwarp();
+            if (!mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue)) break;
+            tc_fence_after_sync();
+            const int64_t row = static_cast<int64_t>(tm) * kBM + row_in_tile;
+            uint16_t* orow = g.out + static_cast<int64_t>(b) * g.stride_o + row * g.ldo;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                tmem_load_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c), r);
+                tmem_wait_ld();
+                const int colg = col0 + c;
+                if (row < g.m && colg < g.n) {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float v0 = fmaf(__uint_as_float(r[2 * e]), sc, my_bias[c + 2 * e]);
+                        const float v1 = fmaf(__uint_as_float(r[2 * e + 1]), sc, my_bias[c + 2 * e + 1]);
+                        packed[e] = pack_bf16x2(v0, v1);
+                    }
+                    if (g.vec_out && colg + 32 <= g.n) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + colg);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    } else {
+                        for (int e = 0; e < 32 && colg + e < g.n; ++e)
+                            orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(acc_empty + acc);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// k == 0: the product is empty; out = bias (or 0), rounded to bf16.
+__global__ void bias_fill_kernel(uint16_t* out, int64_t m, int64_t n, int64_t ldo, int64_t stride_o, int64_t batch,
+                                 const void* bias, int bias_kind, const float* bias_scale) {
+    const int64_t total = batch * m * n;
+    const float bsc = bias_kind >= 2 ? __ldg(bias_scale) : 0.0f;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t j = i % n;
+        const int64_t r = (i / n) % m;
+        const int64_t b = i / (n * m);
+        float v = 0.0f;
+        if (bias_kind == 1)
+            v = bf16_bits_to_float(static_cast<const uint16_t*>(bias)[j]);
+        else if (bias_kind == 2)
+            v = __fmul_rn(fp8_to_float<0>(static_cast<const uint8_t*>(bias)[j]), bsc);
+        else if (bias_kind == 3)
+            v = __fmul_rn(fp8_to_float<1>(static_cast<const uint8_t*>(bias)[j]), bsc);
+        out[b * stride_o + r * ldo + j] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 3-D uint8 tensor map: dims {inner, outer, batch}, row stride `ld` bytes, batch stride
+// `bstride` bytes, box {128, box_outer, 1}, 128-byte swizzle, zero fill out of bounds.
+int make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t batch, int64_t ld,
+             int64_t bstride, int box_outer) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
+                                static_cast<cuuint64_t>(batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(bstride)};
+    const cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_outer), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+    return FP8DSA_OK;
+}
+
+template <int BN>
+int launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& g, int64_t batch, cudaStream_t stream) {
+    using C = Cfg<BN>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(attr_err));
+    g.tiles_n = (g.n + BN - 1) / BN;
+    g.idesc |= (static_cast<uint32_t>(BN >> 3) << 17);
+    const int64_t per = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
+    const int64_t tiles = per * batch;
+    if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
+    g.num_tiles = static_cast<int>(tiles);
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
+    fp8_gemm_kernel<BN><<<grid, kThreads, C::kSmem, stream>>>(ma, mb, g);
+    return FP8DSA_OK;
+}
+
+// Choose the tile width: fewer waves x narrower tiles wins; ties go to the wider tile
+// (half the operand traffic per flop).
+int choose_bn(int64_t m, int64_t n, int64_t batch) {
+    if (n <= 128) return 128;
+    const int64_t sms = sm_count();
+    const int64_t tm = (m + kBM - 1) / kBM;
+    const int64_t t256 = tm * ((n + 255) / 256) * batch;
+    const int64_t t128 = tm * ((n + 127) / 128) * batch;
+    const int64_t cost256 = ((t256 + sms - 1) / sms) * 256;
+    const int64_t cost128 = ((t128 + sms - 1) / sms) * 128;
+    return cost128 < cost256 ? 128 : 256;
+}
+
+}  // namespace
+
+int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn, int b_mn, int64_t m,
+                int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch, int64_t stride_a,
+                int64_t stride_b, int64_t stride_o, const float* scale_a, const float* scale_b, const void* bias,
+                int bias_kind, const float* bias_scale, void* out, cudaStream_t stream) {
+    if (m == 0 || n == 0 || batch == 0) return FP8DSA_OK;
+    const double flops = 2.0 * static_cast<double>(m) * n * k * batch;
+    if (k == 0) {
+        const int64_t total = batch * m * n;
+        const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 8));
+        launch_begin(kKindOther, stream);
+        bias_fill_kernel<<<blocks, 256, 0, stream>>>(static_cast<uint16_t*>(out), m, n, ldo, stride_o, batch, bias,
+                                                     bias_kind, bias_scale);
+        launch_end(kKindOther, stream, static_cast<double>(total) * 2);
+        return check_launch("bias fill kernel");
+    }
+    const bool a_bat = stride_a != 0 && batch > 1;
+    const bool b_bat = stride_b != 0 && batch > 1;
+    const int bn = choose_bn(m, n, batch);
+
+    CUtensorMap ma, mb;
+    int rc;
+    if (!a_mn)
+        rc = make_map(&ma, a, k, m, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * m, kBM);
+    else
+        rc = make_map(&ma, a, m, k, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * k, kBK);
+    if (rc) return rc;
+    if (!b_mn)
+        rc = make_map(&mb, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, bn);
+    else
+        rc = make_map(&mb, b, n, k, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * k, kBK);
+    if (rc) return rc;
+
+    GemmArgs g{};
+    g.m = static_cast<int>(m);
+    g.n = static_cast<int>(n);
+    g.k = static_cast<int>(k);
+    g.tiles_m = static_cast<int>((m + kBM - 1) / kBM);
+    g.k_blocks = static_cast<int>((k + kBK - 1) / kBK);
+    g.a_batched = a_bat;
+    g.b_batched = b_bat;
+    g.a_mn = a_mn;
+    g.b_mn = b_mn;
+    g.idesc = (1u << 4) | (static_cast<uint32_t>(fmt_a) << 7) | (static_cast<uint32_t>(fmt_b) << 10) |
+              (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+              (static_cast<uint32_t>(kBM >> 4) << 24);
+    g.out = static_cast<uint16_t*>(out);
+    g.ldo = ldo;
+    g.stride_o = stride_o;
+    g.vec_out = aligned16(out) && ldo % 8 == 0 && stride_o % 8 == 0;
+    g.bias = bias;
+    g.bias_kind = bias_kind;
+    g.bias_scale = bias_scale;
+    g.scale_a = scale_a;
+    g.scale_b = scale_b;
+    rc = wait_ctl(&g.wait);
+    if (rc) return rc;
+
+    launch_begin(kKindGemm, stream);
+    rc = bn == 256 ? launch_bn<256>(ma, mb, g, batch, stream) : launch_bn<128>(ma, mb, g, batch, stream);
+    if (rc) return rc;
+    launch_end(kKindGemm, stream, flops);
+    return check_launch("fp8 gemm kernel");
+}
+
+}  // namespace fp8dsa
+
+using namespace fp8dsa;
+
+extern "C" int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b, fp8_layout_t layout,
+                        int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch,
+                        int64_t stride_a, int64_t stride_b, int64_t stride_o, const float* scale_a,
+                        const float* scale_b, const void* bias, const float* bias_scale, void* out,
+                        cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt_a) || !valid_fmt(fmt_b)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
+    if (layout < FP8_LAYOUT_NT || layout > FP8_LAYOUT_TT) return fail(FP8DSA_ERR_INVALID_ARG, "bad layout");
+    if (m < 0 || n < 0 || k < 0 || batch < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (m > 0x7FFFFFFF || n > 0x7FFFFFFF || k > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "sizes must be < 2^31");
+    if (batch > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "batch must be < 2^31");
+    if (out == nullptr || scale_a == nullptr || scale_b == nullptr)
+        return fail(FP8DSA_ERR_INVALID_ARG, "out, scale_a and scale_b are required");
+    if (bias == nullptr && bias_scale != nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "bias_scale without bias");
+    if (ldo < n) return fail(FP8DSA_ERR_INVALID_ARG, "ldo must be >= n");
+    if (batch > 1 && stride_o < ldo * m && stride_o != 0 && m > 1)
+        return fail(FP8DSA_ERR_INVALID_ARG, "stride_o overlaps batches");
+    if (batch > 1 && stride_o == 0 && m > 0 && n > 0) return fail(FP8DSA_ERR_INVALID_ARG, "stride_o must be non-zero when batch > 1");
+    const int a_mn = (layout == FP8_LAYOUT_TN || layout == FP8_LAYOUT_TT) ? 1 : 0;
+    const int b_mn = (layout == FP8_LAYOUT_NN || layout == FP8_LAYOUT_TN) ? 1 : 0;
+    if (m > 0 && n > 0 && batch > 0 && k > 0) {
+        if (a == nullptr || b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "a and b are required");
+        if (lda < (a_mn ? m : k)) return fail(FP8DSA_ERR_INVALID_ARG, "lda too small for the layout");
+        if (ldb < (b_mn ? n : k)) return fail(FP8DSA_ERR_INVALID_ARG, "ldb too small for the layout");
+        if (lda % 16 != 0 || ldb % 16 != 0)
+            return fail(FP8DSA_ERR_UNSUPPORTED, "lda and ldb must be multiples of 16 (TMA row strides)");
+        if (!aligned16(a) || !aligned16(b)) return fail(FP8DSA_ERR_UNSUPPORTED, "a and b must be 16-byte aligned");
+        if (stride_a % 16 != 0 || stride_b % 16 != 0)
+            return fail(FP8DSA_ERR_UNSUPPORTED, "batch strides must be multiples of 16");
+        if (stride_a < 0 || stride_b < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative batch stride");
+    }
+    int rc = check_device();
+    if (rc) return rc;
+    int bias_kind = 0;
+    if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt_a == FP8_E4M3 ? 2 : 3);
+    return gemm_launch(a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
+                       scale_a, scale_b, bias, bias_kind, bias_scale, out, stream);
+}

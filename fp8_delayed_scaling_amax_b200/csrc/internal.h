@@ -1,0 +1,98 @@
+// Host-side internals shared by the library's translation units: error reporting, the
+// per-device status word, launch bookkeeping (timeout, optional per-kernel timing) and
+// small argument-check helpers.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+#include "../../include/fp8dsa.h"
+#include "device.cuh"
+
+namespace fp8dsa {
+
+// Record a message for fp8_last_error() and return `code`.
+int fail(int code, const std::string& msg);
+// Clear the thread-local error message.
+void clear_error();
+
+// Check the current device is compute capability 10.x (cached per device).
+int check_device();
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// WaitCtl for the current device (status word address + timeout).
+int wait_ctl(WaitCtl* ctl);
+
+// Kernel classes for the optional per-kernel timing.
+enum KernelKind : int { kKindQuantize = 0, kKindGemm = 1, kKindOther = 2 };
+
+// Bracket a launch with timing events when profiling is on.  `work` is the algorithmic
+// bytes (quantize, other) or flops (GEMM) the launch performs.
+void launch_begin(int kind, cudaStream_t stream);
+void launch_end(int kind, cudaStream_t stream, double work);
+
+// After a launch: map a launch failure to FP8DSA_ERR_CUDA.
+int check_launch(const char* what);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline int in_type_bytes(fp8_in_t t) { return t == FP8_IN_F32 ? 4 : 2; }
+
+inline bool valid_in_type(int t) { return t == FP8_IN_BF16 || t == FP8_IN_F16 || t == FP8_IN_F32; }
+inline bool valid_fmt(int f) { return f == FP8_E4M3 || f == FP8_E5M2; }
+inline float fmt_max(fp8_fmt_t f) { return f == FP8_E5M2 ? 57344.0f : 448.0f; }
+
+// ---------------------------------------------------------------------------------------
+// Internal launchers (each enqueues exactly the kernels named; arguments already checked).
+// ---------------------------------------------------------------------------------------
+
+// Amax of up to three tensors in one launch; for tensor t, its last block writes
+// scale_out[t] = max(RN32(amax / fp8_max) / pow2_margin, 1e-12) (if non-null),
+// amax_out[t] (if non-null), or folds into ring seed slots (if ring[t].state non-null,
+// hist[idx] = amax, scale = formula over the window).  scratch: 16 bytes per tensor,
+// zero on entry and left zero.
+struct AmaxJob {
+    const void* x = nullptr;
+    fp8_in_t in_type = FP8_IN_BF16;
+    int64_t numel = 0;
+    float fp8_max = 448.0f;
+    float pow2_margin = 1.0f;
+    float* scale_out = nullptr;
+    float* amax_out = nullptr;
+    fp8_ring_t ring{};  // ring.state == nullptr: no seeding
+};
+int launch_amax_jobs(const AmaxJob* jobs, int njobs, uint32_t* scratch, cudaStream_t stream);
+
+// Quantize launch description (row-major, transposed or dual).
+struct QuantJob {
+    const void* x = nullptr;
+    fp8_in_t in_type = FP8_IN_BF16;
+    int64_t rows = 0, cols = 0;
+    const float* scale = nullptr;
+    fp8_fmt_t fmt = FP8_E4M3;
+    uint8_t* out = nullptr;     // [rows][cols] or nullptr
+    uint8_t* out_t = nullptr;   // [cols][rows] or nullptr
+    float* amax_out = nullptr;  // final amax (may be nullptr)
+    const fp8_ring_t* ring = nullptr;
+    float* scale_used_out = nullptr;  // the step used, written once (may be nullptr)
+    float* colsum_partial = nullptr;  // [ceil(rows/128)][cols] fp32 column sums (tiled only)
+};
+int launch_quantize(const QuantJob& job, cudaStream_t stream);
+
+// grad_b[c] = RN_bf16(sum_t partial[t][c]) in a fixed order.
+int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,
+                           cudaStream_t stream);
+
+// The GEMM entry with arguments already validated (used by the linear compositions).
+int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn_major,
+                int b_mn_major, int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb,
+                int64_t ldo, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_o,
+                const float* scale_a, const float* scale_b, const void* bias, int bias_kind,
+                const float* bias_scale, void* out, cudaStream_t stream);
+
+}  // namespace fp8dsa

@@ -1,0 +1,328 @@
+// FP8 linear layer forward / backward, composed from the quantize and GEMM kernels.
+//
+// Definition: AstrAI compare view 3e57cc8...main, astrai/extension/fp8.py --
+// fp8_linear_forward (delayed: snapshot the ring steps, quantize x and w folding their rings,
+// NT GEMM with sx*sw and the fused bias; dynamic: measure the current amax first) and
+// _LinearFp8.backward (g quantized once in both orientations folding the g ring; x and w
+// re-quantized transposed with the forward's steps and no ring; grad_x = g8 . w8T^T and
+// grad_w = g8T . x8T^T, both NT; grad_b = column sum of g).
+//
+// Launches per call (delayed scaling):
+//   forward : quantize x (ring fold) + quantize w (ring fold) + GEMM                  = 3
+//   backward: dual quantize g (ring fold + per-tile column sums) + transposed quantize x
+//             + transposed quantize w + GEMM dX + GEMM dW + column-sum finalize       = 6
+// The snapshot of each step is written by the folding kernel itself (no clone launches), so
+// the GEMM dequantizes with exactly the step the bytes were quantized with.
+#include <cuda_runtime.h>
+
+#include <string>
+
+#include "internal.h"
+
+namespace fp8dsa {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kScratchBytes = 128;  // 3 x 16 B amax scratch + 4 internal fp32 steps
+
+struct FwdLayout {
+    size_t x8, w8, scratch, total;
+};
+
+FwdLayout fwd_layout(int64_t m, int64_t k, int64_t n) {
+    FwdLayout L;
+    size_t off = 0;
+    L.x8 = off;
+    off = align_up(off + static_cast<size_t>(m) * k, kAlign);
+    L.w8 = off;
+    off = align_up(off + static_cast<size_t>(n) * k, kAlign);
+    L.scratch = off;
+    off = align_up(off + kScratchBytes, kAlign);
+    L.total = off;
+    return L;
+}
+
+struct BwdLayout {
+    size_t g8, g8t, x8t, w8t, colsum, scratch, total;
+};
+
+BwdLayout bwd_layout(int64_t m, int64_t k, int64_t n) {
+    BwdLayout L;
+    size_t off = 0;
+    const size_t mn = static_cast<size_t>(m) * n;
+    L.g8 = off;
+    off = align_up(off + mn, kAlign);
+    L.g8t = off;
+    off = align_up(off + mn, kAlign);
+    L.x8t = off;
+    off = align_up(off + static_cast<size_t>(k) * m, kAlign);
+    L.w8t = off;
+    off = align_up(off + static_cast<size_t>(k) * n, kAlign);
+    L.colsum = off;
+    off = align_up(off + sizeof(float) * static_cast<size_t>((m + 127) / 128) * n, kAlign);
+    L.scratch = off;
+    off = align_up(off + kScratchBytes, kAlign);
+    L.total = off;
+    return L;
+}
+
+int check_ring_arg(const fp8_ring_t* r, const char* name) {
+    if (r == nullptr) return FP8DSA_OK;
+    if (r->state == nullptr || r->hist_len < 1 || r->hist_idx < 0 || r->hist_idx >= r->hist_len ||
+        !(r->fp8_max > 0.0f) || !(r->pow2_margin > 0.0f))
+        return fail(FP8DSA_ERR_INVALID_ARG, std::string(name) + ": invalid ring (state, hist_len, hist_idx, fp8_max, pow2_margin)");
+    if (!aligned16(r->state)) return fail(FP8DSA_ERR_UNSUPPORTED, std::string(name) + ": ring state must be 16-byte aligned");
+    return FP8DSA_OK;
+}
+
+}  // namespace
+}  // namespace fp8dsa
+
+using namespace fp8dsa;
+
+extern "C" {
+
+size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
+    if (m < 0 || k < 0 || n < 0) return 0;
+    return fwd_layout(m, k, n).total;
+}
+
+size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
+    if (m < 0 || k < 0 || n < 0) return 0;
+    return bwd_layout(m, k, n).total;
+}
+
+int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
+                       const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                       const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                       float* sw_used, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
+    if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (x == nullptr || w == nullptr || y == nullptr || workspace == nullptr)
+        return fail(FP8DSA_ERR_INVALID_ARG, "x, w, y and workspace are required");
+    if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
+    if (w_is_fp8 && w_step == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "w_is_fp8 needs w_step");
+    if (bias == nullptr && bias_scale != nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "bias_scale without bias");
+    const bool dynamic = x_ring == nullptr;
+    if (dynamic && w_ring != nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "w_ring given without x_ring");
+    if (!dynamic && !w_is_fp8 && w_ring == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "delayed scaling needs w_ring");
+    if (dynamic && !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "pow2_margin must be > 0");
+    int rc = check_ring_arg(x_ring, "x_ring");
+    if (rc) return rc;
+    rc = check_ring_arg(w_is_fp8 ? nullptr : w_ring, "w_ring");
+    if (rc) return rc;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    const FwdLayout L = fwd_layout(m, k, n);
+    if (workspace_bytes < L.total)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    if (w_is_fp8 && !aligned16(w)) return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 w must be 16-byte aligned");
+    rc = check_device();
+    if (rc) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* x8 = ws + L.x8;
+    uint8_t* w8 = w_is_fp8 ? static_cast<uint8_t*>(const_cast<void*>(w)) : ws + L.w8;
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
+    float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
+    float* sx = sx_used ? sx_used : internal;
+    float* sw = sw_used ? sw_used : internal + 1;
+
+    if (w_is_fp8) {
+        cudaError_t e = cudaMemcpyAsync(sw, w_step, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("copy w_step: ") + cudaGetErrorString(e));
+    }
+    if (dynamic) {
+        cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset scratch: ") + cudaGetErrorString(e));
+        AmaxJob jobs[2];
+        int nj = 0;
+        jobs[nj].x = x;
+        jobs[nj].numel = m * k;
+        jobs[nj].fp8_max = fmt_max(fmt);
+        jobs[nj].pow2_margin = pow2_margin;
+        jobs[nj].scale_out = sx;
+        ++nj;
+        if (!w_is_fp8) {
+            jobs[nj].x = w;
+            jobs[nj].numel = n * k;
+            jobs[nj].fp8_max = fmt_max(fmt);
+            jobs[nj].pow2_margin = pow2_margin;
+            jobs[nj].scale_out = sw;
+            ++nj;
+        }
+        rc = launch_amax_jobs(jobs, nj, scratch, stream);
+        if (rc) return rc;
+    }
+    QuantJob qx;
+    qx.x = x;
+    qx.rows = m;
+    qx.cols = k;
+    qx.fmt = fmt;
+    qx.out = x8;
+    if (dynamic) {
+        qx.scale = sx;
+    } else {
+        qx.scale = x_ring->state + x_ring->hist_len;
+        qx.ring = x_ring;
+        qx.scale_used_out = sx;
+    }
+    rc = launch_quantize(qx, stream);
+    if (rc) return rc;
+    if (!w_is_fp8) {
+        QuantJob qw;
+        qw.x = w;
+        qw.rows = n;
+        qw.cols = k;
+        qw.fmt = fmt;
+        qw.out = w8;
+        if (dynamic) {
+            qw.scale = sw;
+        } else {
+            qw.scale = w_ring->state + w_ring->hist_len;
+            qw.ring = w_ring;
+            qw.scale_used_out = sw;
+        }
+        rc = launch_quantize(qw, stream);
+        if (rc) return rc;
+    }
+    int bias_kind = 0;
+    if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt == FP8_E4M3 ? 2 : 3);
+    return gemm_launch(x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y,
+                       stream);
+}
+
+int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                        int need_grad_x, int need_grad_w, int need_grad_b, const float* sx_fwd, const float* sw_fwd,
+                        const fp8_ring_t* g_ring, float pow2_margin, float* sg_used, void* workspace,
+                        size_t workspace_bytes, void* grad_x, void* grad_w, void* grad_b, cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
+    if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (w == nullptr || grad_x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
+    if (need_grad_w && (x == nullptr || grad_w == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
+    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
+    if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
+    const bool dynamic = g_ring == nullptr;
+    if (!dynamic && ((need_grad_w && sx_fwd == nullptr) || (need_grad_x && sw_fwd == nullptr)))
+        return fail(FP8DSA_ERR_INVALID_ARG, "delayed scaling needs the forward's sx_fwd / sw_fwd");
+    if (dynamic && !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "pow2_margin must be > 0");
+    int rc = check_ring_arg(g_ring, "g_ring");
+    if (rc) return rc;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    const BwdLayout L = bwd_layout(m, k, n);
+    if (workspace_bytes < L.total)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    rc = check_device();
+    if (rc) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* g8 = ws + L.g8;
+    uint8_t* g8t = ws + L.g8t;
+    uint8_t* x8t = ws + L.x8t;
+    uint8_t* w8t = ws + L.w8t;
+    float* colsum = reinterpret_cast<float*>(ws + L.colsum);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
+    float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
+    float* sg = sg_used ? sg_used : internal;
+    const float* sx = sx_fwd;
+    const float* sw = sw_fwd;
+
+    if (dynamic) {
+        cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset scratch: ") + cudaGetErrorString(e));
+        float* sx_dyn = internal + 1;
+        float* sw_dyn = internal + 2;
+        AmaxJob jobs[3];
+        int nj = 0;
+        jobs[nj].x = g;
+        jobs[nj].numel = m * n;
+        jobs[nj].fp8_max = fmt_max(fmt);
+        jobs[nj].pow2_margin = pow2_margin;
+        jobs[nj].scale_out = sg;
+        ++nj;
+        if (need_grad_w) {
+            jobs[nj].x = x;
+            jobs[nj].numel = m * k;
+            jobs[nj].fp8_max = fmt_max(fmt);
+            jobs[nj].pow2_margin = pow2_margin;
+            jobs[nj].scale_out = sx_dyn;
+            ++nj;
+        }
+        if (need_grad_x) {
+            jobs[nj].x = w;
+            jobs[nj].numel = n * k;
+            jobs[nj].fp8_max = fmt_max(fmt);
+            jobs[nj].pow2_margin = pow2_margin;
+            jobs[nj].scale_out = sw_dyn;
+            ++nj;
+        }
+        rc = launch_amax_jobs(jobs, nj, scratch, stream);
+        if (rc) return rc;
+        sx = sx_dyn;
+        sw = sw_dyn;
+    }
+
+    // g: both orientations, ring fold, per-tile column sums for grad_b.
+    QuantJob qg;
+    qg.x = g;
+    qg.rows = m;
+    qg.cols = n;
+    qg.fmt = fmt;
+    qg.out = g8;
+    qg.out_t = g8t;
+    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    if (dynamic) {
+        qg.scale = sg;
+    } else {
+        qg.scale = g_ring->state + g_ring->hist_len;
+        qg.ring = g_ring;
+        qg.scale_used_out = sg;
+    }
+    rc = launch_quantize(qg, stream);
+    if (rc) return rc;
+    if (need_grad_w) {
+        QuantJob qx;
+        qx.x = x;
+        qx.rows = m;
+        qx.cols = k;
+        qx.fmt = fmt;
+        qx.out_t = x8t;
+        qx.scale = sx;
+        rc = launch_quantize(qx, stream);
+        if (rc) return rc;
+    }
+    if (need_grad_x) {
+        QuantJob qw;
+        qw.x = w;
+        qw.rows = n;
+        qw.cols = k;
+        qw.fmt = fmt;
+        qw.out_t = w8t;
+        qw.scale = sw;
+        rc = launch_quantize(qw, stream);
+        if (rc) return rc;
+        // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T
+        rc = gemm_launch(g8, w8t, fmt, fmt, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x,
+                         stream);
+        if (rc) return rc;
+    }
+    if (need_grad_w) {
+        // grad_w [n][k] = g8t [n][m] . (x8t [k][m])^T
+        rc = gemm_launch(g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w,
+                         stream);
+        if (rc) return rc;
+    }
+    if (need_grad_b) {
+        const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
+        rc = launch_colsum_finalize(colsum, tiles, n, grad_b, stream);
+        if (rc) return rc;
+    }
+    return FP8DSA_OK;
+}
+
+}  // extern "C"

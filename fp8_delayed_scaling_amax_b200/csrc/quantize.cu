@@ -1,0 +1,647 @@
+// FP8 quantize kernels with fused raw-domain amax and the last-block history-ring fold.
+//
+// Sources (AstrAI compare view 3e57cc8...main): csrc/kernels/fp8/quantize.cuh
+// (fp8_quantize_kernel, fp8_quantize_tiled_kernel, publish_amax), astrai/extension/fp8.py
+// (_ScaleRing, FP8Recipe.scale_from_history, _dynamic_scale) and the extension commit log
+// (amax is the max of the unscaled input; the ring is finalised in the quantize kernel's last
+// block with zero extra launches).
+//
+// B200 design:
+//  * Row-major quantize is a flat grid-stride kernel: 16 elements per thread-iteration
+//    (two or four 128-bit loads, one 128-bit store of packed fp8x4 words), two iterations
+//    in flight, grid = 8 resident 256-thread blocks per SM.
+//  * Transposed / dual quantize is tiled 128 x 128: coalesced 128-bit row loads, fp8 bytes
+//    staged in a 16 KB shared tile whose 16-byte chunks are XOR-swizzled by row group, then
+//    a register 4x4 byte transpose (PRMT) and 128-byte coalesced stores of each output row.
+//    The dual mode also writes the row-major bytes straight from registers, and can emit
+//    per-tile fp32 column sums (the bias gradient) from the values it already holds.
+//  * Each block reduces amax with warp shuffles, one atomicMax per block; with a ring, a
+//    threadfence + ticket elects the last block, which folds the amax into the window and
+//    publishes the next step.  No wait, no spin: the fold cannot stall.
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <string>
+
+#include "internal.h"
+
+namespace fp8dsa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTile = 128;
+
+// ----------------------------------------------------------------------------------------
+// Input element access
+// ----------------------------------------------------------------------------------------
+struct Bf16In {
+    using E = uint16_t;
+    using Raw = uint4;
+    static __device__ __forceinline__ float cvt(E v) { return __uint_as_float(uint32_t(v) << 16); }
+    // 8 consecutive elements (16 bytes, 16-byte aligned) as raw bits, then unpacked.
+    static __device__ __forceinline__ Raw load_raw(const E* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+    static __device__ __forceinline__ void unpack(const Raw& v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+    static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+};
+
+struct F16In {
+    using E = uint16_t;
+    using Raw = uint4;
+    static __device__ __forceinline__ float cvt(E v) { return __half2float(__ushort_as_half(v)); }
+    static __device__ __forceinline__ Raw load_raw(const E* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+    static __device__ __forceinline__ void unpack(const Raw& v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __half2float(__ushort_as_half(static_cast<uint16_t>(w[i] & 0xFFFFu)));
+            f[2 * i + 1] = __half2float(__ushort_as_half(static_cast<uint16_t>(w[i] >> 16)));
+        }
+    }
+    static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+};
+
+struct F32Raw {
+    float4 a, b;
+};
+
+struct F32In {
+    using E = float;
+    using Raw = F32Raw;
+    static __device__ __forceinline__ float cvt(E v) { return v; }
+    static __device__ __forceinline__ Raw load_raw(const E* p) {
+        return {__ldg(reinterpret_cast<const float4*>(p)), __ldg(reinterpret_cast<const float4*>(p) + 1)};
+    }
+    static __device__ __forceinline__ void unpack(const Raw& v, float (&f)[8]) {
+        f[0] = v.a.x; f[1] = v.a.y; f[2] = v.a.z; f[3] = v.a.w;
+        f[4] = v.b.x; f[5] = v.b.y; f[6] = v.b.z; f[7] = v.b.w;
+    }
+    static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+};
+
+// Arguments of the quantize kernels (one POD by value).
+struct QArgs {
+    const void* x;
+    int64_t numel, rows, cols;
+    const float* scale;        // step s; every element is multiplied by RN32(1/s)
+    uint8_t* out;              // [rows][cols] or null
+    uint8_t* out_t;            // [cols][rows] or null
+    float* amax_accum;         // block maxima land here (ring amax slot or amax_out), or null
+    float* amax_out;           // ring mode: receives the final amax
+    float* ring_state;         // null = no fold
+    int hist_len, hist_idx;
+    float fp8_max, pow2_margin;
+    float* scale_used_out;     // receives the step used, or null
+    float* colsum;             // [gridDim.y][cols] per-tile column sums, or null
+    int vec_in, vec_out, vec_out_t;
+};
+
+// Eight floats -> eight fp8 bytes (two words), updating amax over the raw values.
+template <int kFmt>
+__device__ __forceinline__ uint2 convert8(const float (&f)[8], float mult, float& amax) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    const uint32_t w0 = cvt_fp8x4<kFmt>(__fmul_rn(f[0], mult), __fmul_rn(f[1], mult),
+                                        __fmul_rn(f[2], mult), __fmul_rn(f[3], mult));
+    const uint32_t w1 = cvt_fp8x4<kFmt>(__fmul_rn(f[4], mult), __fmul_rn(f[5], mult),
+                                        __fmul_rn(f[6], mult), __fmul_rn(f[7], mult));
+    return make_uint2(w0, w1);
+}
+
+template <int kFmt>
+__device__ __forceinline__ uint8_t convert1(float v, float mult) {
+    return static_cast<uint8_t>(cvt_fp8x2<kFmt>(__fmul_rn(v, mult), 0.0f) & 0xFFu);
+}
+
+// Block-wide amax reduce, one atomic per block, then (with a ring) the last-block fold:
+// scale_used = step, hist[idx] = amax, scale = max(RN32(peak / fp8_max) / 2^m, 1e-12),
+// amax and done slots re-zeroed.  Every thread of the block must call this.
+__device__ __forceinline__ void block_finish(const QArgs& a, float amax, float step) {
+    __shared__ float red[32];
+    const int tid = threadIdx.x;
+    amax = warp_max(amax);
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    if (tid != 0) return;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    float m = red[0];
+    for (int w = 1; w < nwarps; ++w) m = fmaxf(m, red[w]);
+    if (a.amax_accum != nullptr) atomicMax(reinterpret_cast<unsigned*>(a.amax_accum), __float_as_uint(m));
+    if (a.ring_state != nullptr) {
+        float* st = a.ring_state;
+        const int n = a.hist_len;
+        unsigned* done = reinterpret_cast<unsigned*>(st + n + 3);
+        __threadfence();
+        const unsigned nblocks = gridDim.x * gridDim.y * gridDim.z;
+        const unsigned ticket = atomicAdd(done, 1u);
+        if (ticket != nblocks - 1u) return;
+        __threadfence();
+        const float am = __uint_as_float(atomicOr(reinterpret_cast<unsigned*>(st + n + 2), 0u));
+        st[n + 1] = step;
+        st[a.hist_idx] = am;
+        float peak = am;
+        for (int i = 0; i < n; ++i) peak = fmaxf(peak, __ldcg(st + i));
+        st[n] = fmaxf(__fdiv_rn(__fdiv_rn(peak, a.fp8_max), a.pow2_margin), 1e-12f);
+        st[n + 2] = 0.0f;
+        atomicExch(done, 0u);
+        if (a.amax_out != nullptr) *a.amax_out = am;
+        if (a.scale_used_out != nullptr) *a.scale_used_out = step;
+    } else if (a.scale_used_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0) {
+        *a.scale_used_out = step;
+    }
+}
+
+// ----------------------------------------------------------------------------------------
+// Row-major quantize: flat, grid-stride, 16 elements per thread per iteration.
+// ----------------------------------------------------------------------------------------
+template <class In, int kFmt>
+__global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(QArgs a) {
+    const float step = __ldg(a.scale);
+    const float mult = __frcp_rn(step);
+    const auto* x = static_cast<const typename In::E*>(a.x);
+    float amax = 0.0f;
+    const int64_t gstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t n16 = a.vec_in ? a.numel / 16 : 0;
+    for (int64_t g = tid; g < n16; g += 2 * gstride) {
+        const int64_t g1 = g + gstride;
+        const bool has1 = g1 < n16;
+        typename In::Raw r0 = In::load_raw(x + g * 16);
+        typename In::Raw r1 = In::load_raw(x + g * 16 + 8);
+        typename In::Raw r2, r3;
+        if (has1) {
+            r2 = In::load_raw(x + g1 * 16);
+            r3 = In::load_raw(x + g1 * 16 + 8);
+        }
+        float f0[8], f1[8];
+        In::unpack(r0, f0);
+        In::unpack(r1, f1);
+        const uint2 lo = convert8<kFmt>(f0, mult, amax);
+        const uint2 hi = convert8<kFmt>(f1, mult, amax);
+        *reinterpret_cast<uint4*>(a.out + g * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        if (has1) {
+            In::unpack(r2, f0);
+            In::unpack(r3, f1);
+            const uint2 lo1 = convert8<kFmt>(f0, mult, amax);
+            const uint2 hi1 = convert8<kFmt>(f1, mult, amax);
+            *reinterpret_cast<uint4*>(a.out + g1 * 16) = make_uint4(lo1.x, lo1.y, hi1.x, hi1.y);
+        }
+    }
+    for (int64_t i = n16 * 16 + tid; i < a.numel; i += gstride) {
+        const float v = In::cvt(x[i]);
+        amax = fmaxf(amax, fabsf(v));
+        a.out[i] = convert1<kFmt>(v, mult);
+    }
+    block_finish(a, amax, step);
+}
+
+// ----------------------------------------------------------------------------------------
+// Transposed / dual quantize: 128 x 128 tiles through a swizzled shared byte tile.
+// ----------------------------------------------------------------------------------------
+template <class In, int kFmt, bool kRowOut, bool kColsum>
+__global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 4) quant_tiled_kernel(QArgs a) {
+    // 128 rows x 128 bytes; the 16-byte chunk c of row r lives at chunk c ^ ((r >> 4) & 7).
+    __shared__ __align__(16) uint32_t tile[kTile * 32];
+    __shared__ float csum[kColsum ? 8 : 1][kColsum ? kTile : 1];
+
+    const float step = __ldg(a.scale);
+    const float mult = __frcp_rn(step);
+    const auto* x = static_cast<const typename In::E*>(a.x);
+    const int64_t rows = a.rows, cols = a.cols;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTile;
+    const int t = threadIdx.x;
+    const int j = t & 15;   // 8-column group of the tile
+    const int rr = t >> 4;  // row within each 16-row slab
+    const int64_t gc = c0 + 8 * j;
+    const bool interior = a.vec_in && r0 + kTile <= rows && c0 + kTile <= cols;
+
+    float amax = 0.0f;
+    float cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0f;
+
+    typename In::Raw raw[8];
+    if (interior) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) raw[i] = In::load_raw(x + (r0 + rr + 16 * i) * cols + gc);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = rr + 16 * i;
+        const int64_t gr = r0 + r;
+        float f[8];
+        if (interior) {
+            In::unpack(raw[i], f);
+        } else if (gr < rows && a.vec_in && gc + 8 <= cols) {
+            In::load8(x + gr * cols + gc, f);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                f[e] = (gr < rows && gc + e < cols) ? In::cvt(x[gr * cols + gc + e]) : 0.0f;
+        }
+        if constexpr (kColsum) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cs[e] += f[e];
+        }
+        const uint2 w = convert8<kFmt>(f, mult, amax);
+        if constexpr (kRowOut) {
+            if (gr < rows) {
+                uint8_t* dst = a.out + gr * cols + gc;
+                if (a.vec_out && gc + 8 <= cols) {
+                    *reinterpret_cast<uint2*>(dst) = w;
+                } else {
+                    const uint32_t ww[2] = {w.x, w.y};
+                    for (int e = 0; e < 8 && gc + e < cols; ++e)
+                        dst[e] = static_cast<uint8_t>(ww[e >> 2] >> (8 * (e & 3)));
+                }
+            }
+        }
+        const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
+        *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = w;
+    }
+
+    if constexpr (kColsum) {
+        // lanes l and l ^ 16 share the column group; then the 8 warps go through shared memory
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
+        if ((t & 16) == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) csum[t >> 5][8 * j + e] = cs[e];
+        }
+    }
+    __syncthreads();
+
+    if constexpr (kColsum) {
+        if (t < kTile && c0 + t < cols) {
+            float s = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) s += csum[w][t];
+            a.colsum[static_cast<int64_t>(blockIdx.y) * cols + c0 + t] = s;
+        }
+    }
+
+    // Phase 2: warp w owns tile columns 16w .. 16w+15; lane -> (column group of 4, 16 rows).
+    const int w = t >> 5, lane = t & 31;
+    const int cgl = lane & 3, rg = lane >> 2;
+    uint32_t W[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) W[i] = tile[(16 * rg + i) * 32 + ((w ^ rg) << 2) + cgl];
+    uint32_t O[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t x0 = __byte_perm(W[4 * k], W[4 * k + 1], 0x5140);
+        const uint32_t x1 = __byte_perm(W[4 * k], W[4 * k + 1], 0x7362);
+        const uint32_t y0 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x5140);
+        const uint32_t y1 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x7362);
+        O[0][k] = __byte_perm(x0, y0, 0x5410);
+        O[1][k] = __byte_perm(x0, y0, 0x7632);
+        O[2][k] = __byte_perm(x1, y1, 0x5410);
+        O[3][k] = __byte_perm(x1, y1, 0x7632);
+    }
+    const int64_t gr0 = r0 + 16 * rg;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const int64_t c = c0 + 4 * (4 * w + cgl) + jj;
+        if (c >= cols || gr0 >= rows) continue;
+        uint8_t* dst = a.out_t + c * rows + gr0;
+        if (a.vec_out_t && gr0 + 16 <= rows) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(O[jj][0], O[jj][1], O[jj][2], O[jj][3]);
+        } else {
+            for (int b = 0; b < 16 && gr0 + b < rows; ++b)
+                dst[b] = static_cast<uint8_t>(O[jj][b >> 2] >> (8 * (b & 3)));
+        }
+    }
+    block_finish(a, amax, step);
+}
+
+// ----------------------------------------------------------------------------------------
+// Amax of up to three tensors in one launch (blockIdx.y = tensor); the last block of each
+// tensor publishes its step / amax / ring seed and re-zeroes its scratch.
+// ----------------------------------------------------------------------------------------
+struct AmaxArgs {
+    const void* x[3];
+    int in_type[3];
+    int64_t numel[3];
+    float fp8_max[3], pow2_margin[3];
+    float* scale_out[3];
+    float* amax_out[3];
+    float* ring_state[3];
+    int hist_len[3], hist_idx[3];
+    uint32_t* scratch[3];  // [amax bits, done]
+    int vec[3];
+};
+
+template <class In>
+__device__ __forceinline__ float amax_range(const void* xv, int64_t numel, int vec) {
+    const auto* x = static_cast<const typename In::E*>(xv);
+    float amax = 0.0f;
+    const int64_t gstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t n16 = vec ? numel / 16 : 0;
+    for (int64_t g = tid; g < n16; g += gstride) {
+        float f0[8], f1[8];
+        In::load8(x + g * 16, f0);
+        In::load8(x + g * 16 + 8, f1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fmaxf(fabsf(f0[e]), fabsf(f1[e])));
+    }
+    for (int64_t i = n16 * 16 + tid; i < numel; i += gstride) amax = fmaxf(amax, fabsf(In::cvt(x[i])));
+    return amax;
+}
+
+__global__ void __launch_bounds__(kThreads) amax_jobs_kernel(AmaxArgs a) {
+    const int job = blockIdx.y;
+    float amax;
+    if (a.in_type[job] == FP8_IN_BF16)
+        amax = amax_range<Bf16In>(a.x[job], a.numel[job], a.vec[job]);
+    else if (a.in_type[job] == FP8_IN_F16)
+        amax = amax_range<F16In>(a.x[job], a.numel[job], a.vec[job]);
+    else
+        amax = amax_range<F32In>(a.x[job], a.numel[job], a.vec[job]);
+
+    __shared__ float red[32];
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    float m = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    uint32_t* scr = a.scratch[job];
+    atomicMax(scr, __float_as_uint(m));
+    __threadfence();
+    const unsigned ticket = atomicAdd(scr + 1, 1u);
+    if (ticket != gridDim.x - 1u) return;
+    __threadfence();
+    const float am = __uint_as_float(atomicOr(scr, 0u));
+    float peak = am;
+    if (a.ring_state[job] != nullptr) {
+        float* st = a.ring_state[job];
+        const int n = a.hist_len[job];
+        st[a.hist_idx[job]] = am;
+        for (int i = 0; i < n; ++i) peak = fmaxf(peak, __ldcg(st + i));
+        st[n] = fmaxf(__fdiv_rn(__fdiv_rn(peak, a.fp8_max[job]), a.pow2_margin[job]), 1e-12f);
+    }
+    if (a.scale_out[job] != nullptr)
+        *a.scale_out[job] = fmaxf(__fdiv_rn(__fdiv_rn(am, a.fp8_max[job]), a.pow2_margin[job]), 1e-12f);
+    if (a.amax_out[job] != nullptr) *a.amax_out[job] = am;
+    atomicExch(scr, 0u);
+    atomicExch(scr + 1, 0u);
+}
+
+__global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* partial, int64_t tiles,
+                                                                    int64_t cols, uint16_t* out) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= cols) return;
+    float s = 0.0f;
+    for (int64_t t = 0; t < tiles; ++t) s += __ldcg(partial + t * cols + c);
+    out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+}
+
+template <int kFmt, class In>
+void launch_quant_kernel(const QArgs& a, bool tiled, bool row_out, bool colsum, cudaStream_t stream) {
+    if (!tiled) {
+        const int64_t groups = (a.numel + 15) / 16;
+        const int64_t want = std::max<int64_t>(1, (groups + kThreads - 1) / kThreads);
+        const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
+        quant_flat_kernel<In, kFmt><<<blocks, kThreads, 0, stream>>>(a);
+        return;
+    }
+    const dim3 grid(static_cast<unsigned>((a.cols + kTile - 1) / kTile),
+                    static_cast<unsigned>((a.rows + kTile - 1) / kTile));
+    if (row_out) {
+        if (colsum)
+            quant_tiled_kernel<In, kFmt, true, true><<<grid, kThreads, 0, stream>>>(a);
+        else
+            quant_tiled_kernel<In, kFmt, true, false><<<grid, kThreads, 0, stream>>>(a);
+    } else {
+        if (colsum)
+            quant_tiled_kernel<In, kFmt, false, true><<<grid, kThreads, 0, stream>>>(a);
+        else
+            quant_tiled_kernel<In, kFmt, false, false><<<grid, kThreads, 0, stream>>>(a);
+    }
+}
+
+int check_ring(const fp8_ring_t* ring) {
+    if (ring == nullptr) return FP8DSA_OK;
+    if (ring->state == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "ring->state is NULL");
+    if (!aligned16(ring->state)) return fail(FP8DSA_ERR_UNSUPPORTED, "ring->state must be 16-byte aligned");
+    if (ring->hist_len < 1) return fail(FP8DSA_ERR_INVALID_ARG, "ring->hist_len must be >= 1");
+    if (ring->hist_idx < 0 || ring->hist_idx >= ring->hist_len)
+        return fail(FP8DSA_ERR_INVALID_ARG, "ring->hist_idx must be in [0, hist_len)");
+    if (!(ring->fp8_max > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "ring->fp8_max must be > 0");
+    if (!(ring->pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "ring->pow2_margin must be > 0");
+    return FP8DSA_OK;
+}
+
+}  // namespace
+
+int launch_quantize(const QuantJob& job, cudaStream_t stream) {
+    QArgs a{};
+    a.x = job.x;
+    a.rows = job.rows;
+    a.cols = job.cols;
+    a.numel = job.rows * job.cols;
+    a.scale = job.scale;
+    a.out = job.out;
+    a.out_t = job.out_t;
+    a.scale_used_out = job.scale_used_out;
+    a.colsum = job.colsum_partial;
+    const bool tiled = job.out_t != nullptr && a.numel > 0;
+    if (job.ring != nullptr) {
+        const int n = job.ring->hist_len;
+        a.ring_state = job.ring->state;
+        a.hist_len = n;
+        a.hist_idx = job.ring->hist_idx;
+        a.fp8_max = job.ring->fp8_max;
+        a.pow2_margin = job.ring->pow2_margin;
+        a.amax_accum = job.ring->state + n + 2;
+        a.amax_out = job.amax_out;
+    } else {
+        a.amax_accum = job.amax_out;
+        if (job.amax_out != nullptr) {
+            cudaError_t e = cudaMemsetAsync(job.amax_out, 0, sizeof(float), stream);
+            if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset amax: ") + cudaGetErrorString(e));
+        }
+    }
+    const int eb = in_type_bytes(job.in_type);
+    const bool rows_vec = (job.cols * eb) % 16 == 0;
+    a.vec_in = aligned16(job.x) && (tiled ? rows_vec : true);
+    a.vec_out = (job.out == nullptr) || (tiled ? ((reinterpret_cast<uintptr_t>(job.out) & 7) == 0 && job.cols % 8 == 0)
+                                               : aligned16(job.out));
+    a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
+    if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
+
+    const double bytes = static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0));
+    launch_begin(kKindQuantize, stream);
+    const bool row_out = job.out != nullptr;
+    const bool colsum = job.colsum_partial != nullptr;
+    if (job.fmt == FP8_E4M3) {
+        if (job.in_type == FP8_IN_BF16) launch_quant_kernel<0, Bf16In>(a, tiled, row_out, colsum, stream);
+        else if (job.in_type == FP8_IN_F16) launch_quant_kernel<0, F16In>(a, tiled, row_out, colsum, stream);
+        else launch_quant_kernel<0, F32In>(a, tiled, row_out, colsum, stream);
+    } else {
+        if (job.in_type == FP8_IN_BF16) launch_quant_kernel<1, Bf16In>(a, tiled, row_out, colsum, stream);
+        else if (job.in_type == FP8_IN_F16) launch_quant_kernel<1, F16In>(a, tiled, row_out, colsum, stream);
+        else launch_quant_kernel<1, F32In>(a, tiled, row_out, colsum, stream);
+    }
+    launch_end(kKindQuantize, stream, bytes);
+    return check_launch("fp8 quantize kernel");
+}
+
+int launch_amax_jobs(const AmaxJob* jobs, int njobs, uint32_t* scratch, cudaStream_t stream) {
+    AmaxArgs a{};
+    int64_t max_numel = 0;
+    double bytes = 0.0;
+    for (int i = 0; i < njobs; ++i) {
+        const AmaxJob& j = jobs[i];
+        a.x[i] = j.x;
+        a.in_type[i] = j.in_type;
+        a.numel[i] = j.numel;
+        a.fp8_max[i] = j.ring.state ? j.ring.fp8_max : j.fp8_max;
+        a.pow2_margin[i] = j.ring.state ? j.ring.pow2_margin : j.pow2_margin;
+        a.scale_out[i] = j.scale_out;
+        a.amax_out[i] = j.amax_out;
+        a.ring_state[i] = j.ring.state;
+        a.hist_len[i] = j.ring.hist_len;
+        a.hist_idx[i] = j.ring.hist_idx;
+        a.scratch[i] = j.ring.state ? reinterpret_cast<uint32_t*>(j.ring.state + j.ring.hist_len + 2)
+                                    : scratch + 4 * i;
+        a.vec[i] = aligned16(j.x);
+        max_numel = std::max(max_numel, j.numel);
+        bytes += static_cast<double>(j.numel) * in_type_bytes(j.in_type);
+    }
+    const int64_t want = std::max<int64_t>(1, (max_numel / 16 + kThreads - 1) / kThreads);
+    const int per_job = std::max(1, static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8 / njobs)));
+    launch_begin(kKindOther, stream);
+    amax_jobs_kernel<<<dim3(per_job, njobs), kThreads, 0, stream>>>(a);
+    launch_end(kKindOther, stream, bytes);
+    return check_launch("fp8 amax kernel");
+}
+
+int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,
+                           cudaStream_t stream) {
+    const unsigned blocks = static_cast<unsigned>((cols + kThreads - 1) / kThreads);
+    launch_begin(kKindOther, stream);
+    colsum_finalize_kernel<<<blocks, kThreads, 0, stream>>>(partial, tiles, cols, static_cast<uint16_t*>(out_bf16));
+    launch_end(kKindOther, stream, static_cast<double>(tiles) * cols * 4 + cols * 2);
+    return check_launch("colsum finalize kernel");
+}
+
+}  // namespace fp8dsa
+
+using namespace fp8dsa;
+
+extern "C" {
+
+int fp8_scale_ring_init(float* state, int hist_len, cudaStream_t stream) {
+    clear_error();
+    if (state == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "state is NULL");
+    if (hist_len < 1) return fail(FP8DSA_ERR_INVALID_ARG, "hist_len must be >= 1");
+    if (!aligned16(state)) return fail(FP8DSA_ERR_UNSUPPORTED, "state must be 16-byte aligned");
+    int rc = check_device();
+    if (rc) return rc;
+    cudaError_t e = cudaMemsetAsync(state, 0, sizeof(float) * (static_cast<size_t>(hist_len) + 4), stream);
+    if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset ring: ") + cudaGetErrorString(e));
+    return FP8DSA_OK;
+}
+
+int fp8_scale_ring_seed(const fp8_ring_t* ring, const void* x, fp8_in_t in_type, int64_t numel,
+                        cudaStream_t stream) {
+    clear_error();
+    if (ring == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "ring is NULL");
+    int rc = check_ring(ring);
+    if (rc) return rc;
+    if (!valid_in_type(in_type)) return fail(FP8DSA_ERR_INVALID_ARG, "bad in_type");
+    if (numel < 0) return fail(FP8DSA_ERR_INVALID_ARG, "numel must be >= 0");
+    if (numel > 0 && x == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x is NULL");
+    rc = check_device();
+    if (rc) return rc;
+    AmaxJob j;
+    j.x = x;
+    j.in_type = in_type;
+    j.numel = numel;
+    j.ring = *ring;
+    return launch_amax_jobs(&j, 1, nullptr, stream);
+}
+
+int fp8_amax_scale(const void* x, fp8_in_t in_type, int64_t numel, float fp8_max, float pow2_margin,
+                   float* scale_out, float* amax_out, uint32_t* scratch, cudaStream_t stream) {
+    clear_error();
+    if (!valid_in_type(in_type)) return fail(FP8DSA_ERR_INVALID_ARG, "bad in_type");
+    if (numel < 0) return fail(FP8DSA_ERR_INVALID_ARG, "numel must be >= 0");
+    if (numel > 0 && x == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x is NULL");
+    if (scale_out == nullptr && amax_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "no output");
+    if (scratch == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "scratch is NULL");
+    if (!aligned16(scratch)) return fail(FP8DSA_ERR_UNSUPPORTED, "scratch must be 16-byte aligned");
+    if (!(fp8_max > 0.0f) || !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "fp8_max and pow2_margin must be > 0");
+    int rc = check_device();
+    if (rc) return rc;
+    AmaxJob j;
+    j.x = x;
+    j.in_type = in_type;
+    j.numel = numel;
+    j.fp8_max = fp8_max;
+    j.pow2_margin = pow2_margin;
+    j.scale_out = scale_out;
+    j.amax_out = amax_out;
+    return launch_amax_jobs(&j, 1, scratch, stream);
+}
+
+static int quantize_common(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,
+                           fp8_fmt_t fmt, uint8_t* out, uint8_t* out_t, float* amax_out,
+                           const fp8_ring_t* ring, cudaStream_t stream) {
+    if (!valid_in_type(in_type)) return fail(FP8DSA_ERR_INVALID_ARG, "bad in_type");
+    if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
+    if (rows < 0 || cols < 0) return fail(FP8DSA_ERR_INVALID_ARG, "rows and cols must be >= 0");
+    if (rows > 0 && cols > 0 && (x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "x is NULL");
+    if (scale == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "scale is NULL");
+    if (out == nullptr && out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "output is NULL");
+    if (out_t != nullptr && (cols + kTile - 1) / kTile > 0x7FFFFFFF)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "too many columns");
+    if (out_t != nullptr && (rows + kTile - 1) / kTile > 65535)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "transposed quantize supports at most 65535*128 rows");
+    int rc = check_ring(ring);
+    if (rc) return rc;
+    rc = check_device();
+    if (rc) return rc;
+    QuantJob j;
+    j.x = x;
+    j.in_type = in_type;
+    j.rows = rows;
+    j.cols = cols;
+    j.scale = scale;
+    j.fmt = fmt;
+    j.out = out;
+    j.out_t = out_t;
+    j.amax_out = amax_out;
+    j.ring = ring;
+    return launch_quantize(j, stream);
+}
+
+int fp8_quantize(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,
+                 fp8_fmt_t fmt, int transposed, uint8_t* out, float* amax_out, const fp8_ring_t* ring,
+                 cudaStream_t stream) {
+    clear_error();
+    if (out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out is NULL");
+    return quantize_common(x, in_type, rows, cols, scale, fmt, transposed ? nullptr : out,
+                           transposed ? out : nullptr, amax_out, ring, stream);
+}
+
+int fp8_quantize_dual(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,
+                      fp8_fmt_t fmt, uint8_t* out, uint8_t* out_t, float* amax_out, const fp8_ring_t* ring,
+                      cudaStream_t stream) {
+    clear_error();
+    if (out == nullptr || out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out and out_t are required");
+    return quantize_common(x, in_type, rows, cols, scale, fmt, out, out_t, amax_out, ring, stream);
+}
+
+}  // extern "C"

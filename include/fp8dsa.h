@@ -1,0 +1,216 @@
+/*
+ * fp8dsa -- FP8 linear layer with per-tensor delayed scaling, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every entry point takes plain pointers and sizes; no C++ or PyTorch types cross
+ * it.  Citations name the AstrAI pages the operation is defined on:
+ *   [ext-log]   AstrAI commit log of astrai/extension
+ *   [compare]   AstrAI compare view 3e57cc8...main (files named after it)
+ *   [by-author] AstrAI commits by author (benchmarks, dispatch notes)
+ *
+ * Conventions shared by all calls
+ * -------------------------------
+ * - Device pointers ("dev") must be CUDA device memory of the current device; host pointers
+ *   ("host") are ordinary host memory.  The library never allocates, frees or retains any
+ *   caller buffer: the caller owns everything, including rings and workspaces.
+ * - All work is enqueued on `stream` (0 = legacy default stream) and returns without
+ *   synchronising.  No scale, amax or status value ever crosses to the host implicitly.
+ * - A "step" (quantization step, `scale`) is the dequantization multiplier: the quantize
+ *   kernels multiply by RN32(1/step), and the GEMM multiplies the accumulator by
+ *   RN32(step_a * step_b) [compare: astrai/extension/fp8.py, fp8_linear_forward].
+ * - Return value: FP8DSA_OK (0) or a negative FP8DSA_ERR_* code.  On error nothing has been
+ *   enqueued (argument checks run before any CUDA call) unless the code is
+ *   FP8DSA_ERR_CUDA, and fp8_last_error() returns a thread-local message.
+ * - fp8 bytes: E4M3FN (max 448) or E5M2 (max 57344) [compare: csrc/kernels/fp8/common.h,
+ *   FP8Format].  bf16 / f16 / f32 inputs are IEEE bit patterns.
+ */
+#ifndef FP8DSA_H
+#define FP8DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8DSA_OK 0
+#define FP8DSA_ERR_INVALID_ARG (-1)     /* null pointer, bad enum, bad size or index     */
+#define FP8DSA_ERR_UNSUPPORTED (-2)     /* alignment / stride the kernels cannot take    */
+#define FP8DSA_ERR_CUDA (-3)            /* a CUDA runtime call or launch failed          */
+#define FP8DSA_ERR_DEVICE (-4)          /* current device is not compute capability 10.x */
+#define FP8DSA_ERR_WORKSPACE (-5)       /* workspace smaller than the *_workspace_size() */
+
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_fmt_t;
+typedef enum { FP8_IN_BF16 = 0, FP8_IN_F16 = 1, FP8_IN_F32 = 2 } fp8_in_t;
+
+/* GEMM operand layouts.  First letter: A; second letter: B.
+ *   A 'N' = stored [M][K] (K contiguous)      A 'T' = stored [K][M] (M contiguous)
+ *   B 'T' = stored [N][K] (K contiguous; the nn.Linear weight)
+ *   B 'N' = stored [K][N] (N contiguous)
+ * The training GEMMs (forward, dX, dW) are all NT [compare: astrai/extension/fp8.py,
+ * _LinearFp8.backward]; NN and TN are the other layouts mm_fp8 accepts
+ * [compare: csrc/kernels/fp8/common.h, RowMajor / ColMajor tags]. */
+typedef enum { FP8_LAYOUT_NT = 0, FP8_LAYOUT_NN = 1, FP8_LAYOUT_TN = 2, FP8_LAYOUT_TT = 3 } fp8_layout_t;
+
+/* One operand's delayed-scaling history ring [compare: astrai/extension/fp8.py, _ScaleRing].
+ * `state` (dev, fp32, hist_len + 4 floats, 16-byte aligned) is laid out
+ *     [ hist[0..hist_len) | scale | scale_used | amax | done ]
+ * hist: amax history window; scale: the step the next use will quantize with;
+ * scale_used: the step the last folding kernel quantized with (its snapshot);
+ * amax, done: kernel scratch, zero between calls (self-cleaning).
+ * hist_idx in [0, hist_len) is the slot this use records into; the caller advances it
+ * host-side, (idx + 1) % hist_len, after each use.  fp8_max is 448 or 57344 for the
+ * format the ring's operand is quantized to, pow2_margin = 2^margin (> 0). */
+typedef struct {
+    float* state;
+    int hist_len;
+    int hist_idx;
+    float fp8_max;
+    float pow2_margin;
+} fp8_ring_t;
+
+/* Zero the ring's hist_len + 4 floats.  state: dev.  [compare: _ScaleRing.__init__] */
+int fp8_scale_ring_init(float* state, int hist_len, cudaStream_t stream);
+
+/* First-use seeding [compare: _ScaleRing.seed]: hist[hist_idx] = max|x| over numel
+ * elements of x (dev, in_type), then scale = max(RN32(peak / fp8_max) / pow2_margin, 1e-12)
+ * with peak the max over the window.  The pages elide seed's body; this is the reading
+ * that makes step 0 of delayed scaling equal dynamic scaling on the same tensor. */
+int fp8_scale_ring_seed(const fp8_ring_t* ring, const void* x, fp8_in_t in_type, int64_t numel,
+                        cudaStream_t stream);
+
+/* Dynamic (current-amax) step [compare: astrai/extension/fp8.py, _dynamic_scale]:
+ * *scale_out = max(RN32(max|x| / fp8_max) / pow2_margin, 1e-12) and, if amax_out is not
+ * NULL, *amax_out = max|x|.  scratch: dev, 16 bytes, 16-byte aligned, all zero before the
+ * first call; the kernel leaves it zero again (self-cleaning), so one scratch may be
+ * reused by calls ordered on one stream but not by calls that overlap. */
+int fp8_amax_scale(const void* x, fp8_in_t in_type, int64_t numel, float fp8_max,
+                   float pow2_margin, float* scale_out, float* amax_out, uint32_t* scratch,
+                   cudaStream_t stream);
+
+/* Quantize with fused raw-domain amax [compare: csrc/kernels/fp8/quantize.cuh,
+ * fp8_quantize_kernel / fp8_quantize_tiled_kernel; ext-log: amax of the unscaled input].
+ *   x: dev, rows x cols row-major, in_type; 16-byte aligned rows take the vector path.
+ *   scale: dev, one fp32 step s; each element becomes q_fmt(RN32(x * RN32(1/s))),
+ *          round-to-nearest-even, saturated to +-FP8_MAX.
+ *   transposed = 0: out is [rows][cols]; = 1: out is the [cols][rows] transpose.
+ *   amax_out: dev or NULL; receives max|x| (NaN ignored).
+ *   ring: NULL, or a ring whose fold runs in the kernel's last block: scale_used = *scale,
+ *         hist[hist_idx] = amax, scale = formula over the window, amax/done re-zeroed
+ *         [compare: quantize.cuh, publish_amax; ext-log: zero extra launches].
+ *         `scale` may point at ring->state[hist_len] (the ring's own step): every block
+ *         reads it before the last block publishes.
+ * rows * cols may be 0 (nothing is written, the ring still folds amax 0). */
+int fp8_quantize(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,
+                 fp8_fmt_t fmt, int transposed, uint8_t* out, float* amax_out,
+                 const fp8_ring_t* ring, cudaStream_t stream);
+
+/* Both orientations from one read of x [compare: astrai/extension/ops/fp8.py, quantize_dual]:
+ * out = [rows][cols], out_t = [cols][rows]; amax and ring as fp8_quantize. */
+int fp8_quantize_dual(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols,
+                      const float* scale, fp8_fmt_t fmt, uint8_t* out, uint8_t* out_t,
+                      float* amax_out, const fp8_ring_t* ring, cudaStream_t stream);
+
+/* FP8 x FP8 GEMM with dequantization and fused bias [compare: astrai/extension/ops/fp8.py,
+ * mm_fp8; csrc/kernels/fp8/gemm/epilogue.cuh]:
+ *     out[b][i][j] = RN_bf16( sum_k A[b][i][k] * B[b][k][j] * RN32(*scale_a * *scale_b) + bias[j] )
+ * accumulated in fp32 on the tensor cores (tcgen05.mma kind::f8f6f4, TMEM accumulators).
+ *   a, b: dev fp8 bytes in the stored layout named by `layout`, formats fmt_a / fmt_b (the
+ *         pages require equal formats; the tensor core takes them independently).
+ *   lda, ldb: row strides in elements of the stored matrices; multiples of 16; a, b 16-byte
+ *         aligned (TMA).  ldo: row stride of out in elements (>= n).
+ *   batch >= 1; stride_a / stride_b / stride_o: element strides between batches; 0 makes a
+ *         size-1 operand broadcast over the batch [compare: mm_fp8's batch rule].  Non-zero
+ *         operand strides are multiples of 16.
+ *   scale_a, scale_b: dev fp32 steps.
+ *   bias: NULL, or dev bf16[n] when bias_scale == NULL, or dev fp8[n] in fmt_a when
+ *         bias_scale (dev fp32) is given: dequantized as byte * *bias_scale after the operand
+ *         scaling [ext-log: FP8Params.bias_scale].
+ *   out: dev bf16.  m, n, k >= 0; k == 0 writes the bias (or zeros). */
+int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b,
+             fp8_layout_t layout, int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb,
+             int64_t ldo, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_o,
+             const float* scale_a, const float* scale_b, const void* bias,
+             const float* bias_scale, void* out, cudaStream_t stream);
+
+/* Workspace bytes linear_forward_fp8 needs for (m, k, n) (x8, w8 and scale scratch). */
+size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
+
+/* FP8 linear forward y = x w^T + bias [compare: astrai/extension/fp8.py, fp8_linear_forward]:
+ *   x: dev bf16 [m][k]; w: dev bf16 [n][k], or fp8 bytes in `fmt` when w_is_fp8 (then
+ *      w_step, dev fp32, is the step those bytes were quantized with, and w_ring is unused).
+ *   bias: NULL, dev bf16[n], or dev fp8[n] in `fmt` with bias_scale (dev fp32).
+ *   Delayed scaling: x_ring and w_ring given.  Each quantize reads its ring's step, folds the
+ *      fresh amax in its last block and publishes the next step; the GEMM dequantizes with
+ *      the steps used (the snapshot) [ext-log: snapshot sx/sw before the finalize].
+ *   Dynamic scaling: x_ring == NULL (and w_ring == NULL): the steps are measured from x and
+ *      w first (max(amax / fp8_max / pow2_margin, 1e-12)), with fp8_max of `fmt` and
+ *      pow2_margin given here.
+ *   sx_used, sw_used: dev fp32 outputs, the steps the GEMM used (the backward's sx / sw).
+ *   workspace: dev, >= linear_forward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned.
+ *   y: dev bf16 [m][n].  k and n must be multiples of 16. */
+int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* w_step,
+                       const void* bias, const float* bias_scale, int64_t m, int64_t k, int64_t n,
+                       fp8_fmt_t fmt, const fp8_ring_t* x_ring, const fp8_ring_t* w_ring,
+                       float pow2_margin, float* sx_used, float* sw_used, void* workspace,
+                       size_t workspace_bytes, void* y, cudaStream_t stream);
+
+/* Workspace bytes linear_backward_fp8 needs for (m, k, n). */
+size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
+
+/* FP8 linear backward [compare: astrai/extension/fp8.py, _LinearFp8.backward]:
+ *   g: dev bf16 [m][n] (dL/dy); x: dev bf16 [m][k]; w: dev bf16 [n][k].  fmt is the
+ *   backward format (E5M2 under the HYBRID policy) for g and the re-quantized x and w.
+ *   g is quantized once in both orientations (folding into g_ring); x and w are re-quantized
+ *   transposed with the forward's steps and fold no ring; then
+ *       grad_x [m][k] = g8 . w8T^T * RN32(sg * sw)   (NT)
+ *       grad_w [n][k] = g8T . x8T^T * RN32(sg * sx)  (NT)
+ *       grad_b [n]    = RN_bf16(sum over rows of g)
+ *   Delayed scaling: g_ring given, sx_fwd / sw_fwd (dev fp32) are the forward's steps.
+ *   Dynamic scaling: g_ring == NULL; sg, sx, sw are re-measured at fmt's FP8_MAX and
+ *   pow2_margin, and sx_fwd / sw_fwd are ignored.
+ *   need_grad_x / need_grad_w / need_grad_b select the outputs (the others may be NULL).
+ *   sg_used: dev fp32 output (the step g was quantized with), may be NULL.
+ *   workspace: dev, >= linear_backward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned.
+ *   k and n must be multiples of 16; m a multiple of 16 when grad_w is needed. */
+int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, int64_t k,
+                        int64_t n, fp8_fmt_t fmt, int need_grad_x, int need_grad_w,
+                        int need_grad_b, const float* sx_fwd, const float* sw_fwd,
+                        const fp8_ring_t* g_ring, float pow2_margin, float* sg_used,
+                        void* workspace, size_t workspace_bytes, void* grad_x, void* grad_w,
+                        void* grad_b, cudaStream_t stream);
+
+/* Device status word of the current device: 0, or a nonzero code a kernel set when a bounded
+ * wait ran out (a pipeline stall instead of a hang).  Synchronises `stream`, reads the word
+ * into *status (host) and clears it.  Not on the pages: added so no kernel can hang a GPU. */
+int fp8_get_device_status(cudaStream_t stream, int* status);
+
+/* Upper bound, in nanoseconds, of every bounded wait in the library's kernels
+ * (default 2e9 = 2 s).  Applies to launches after the call. */
+int fp8_set_wait_timeout_ns(uint64_t ns);
+
+/* Test hook for the failure path: launches one block that waits on a barrier nothing ever
+ * arrives at; the wait gives up after the timeout and sets the device status word.
+ * Not on the pages. */
+int fp8_debug_stalled_wait(cudaStream_t stream);
+
+/* Per-kernel timing: when enabled, every kernel the library launches is bracketed by CUDA
+ * events on its own stream.  fp8_profiler_read synchronises, returns the total device
+ * milliseconds and launch count of kernel class `kind` (0 quantize, 1 GEMM, 2 other) since
+ * the last reset, then resets that class.  Not on the pages (they time with CUDA events
+ * from Python; [by-author]). */
+int fp8_profiler_enable(int on);
+int fp8_profiler_read(int kind, double* total_ms, int64_t* launches, double* bytes_or_flops);
+
+/* Thread-local message describing the last error (empty string if none). */
+const char* fp8_last_error(void);
+
+/* Library version string. */
+const char* fp8dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8DSA_H */

@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports every function ``include/fp8dsa.h``
+declares, and rejects bad arguments with the documented codes before touching CUDA."""
+
+import ctypes
+
+import pytest
+
+import fp8_delayed_scaling_amax_b200 as F
+
+INVALID, UNSUPPORTED, WORKSPACE = -1, -2, -5
+
+
+def test_library_exports_every_header_symbol():
+    lib = F.lib()
+    names = F.header_functions()
+    assert len(names) >= 17
+    for name in names:
+        assert hasattr(lib, name), name
+        assert hasattr(F, name), f"binding lacks {name}"
+    assert "fp8dsa" in F.fp8dsa_version()
+
+
+def test_workspace_sizes_cover_the_buffers():
+    m, k, n = 2048, 1024, 3072
+    fwd = F.linear_forward_fp8_workspace_size(m, k, n)
+    bwd = F.linear_backward_fp8_workspace_size(m, k, n)
+    assert fwd >= m * k + n * k
+    assert bwd >= 2 * m * n + k * m + k * n + 4 * ((m + 127) // 128) * n
+    assert fwd % 256 == 0 and bwd % 256 == 0
+    assert F.linear_forward_fp8_workspace_size(-1, 1, 1) == 0
+
+
+def _rc(fn, *args):
+    return getattr(F.lib(), fn)(*args)
+
+
+def test_quantize_argument_checks():
+    lib = F.lib()
+    ring = F.fp8_ring_t(None, 16, 0, 448.0, 1.0)
+    # bad format
+    assert lib.fp8_quantize(16, 0, 4, 4, 16, 7, 0, 16, None, None, None) == INVALID
+    assert "fmt" in F.last_error()
+    # bad input type
+    assert lib.fp8_quantize(16, 9, 4, 4, 16, 0, 0, 16, None, None, None) == INVALID
+    # null scale
+    assert lib.fp8_quantize(16, 0, 4, 4, None, 0, 0, 16, None, None, None) == INVALID
+    # null out
+    assert lib.fp8_quantize(16, 0, 4, 4, 16, 0, 0, None, None, None, None) == INVALID
+    # negative size
+    assert lib.fp8_quantize(16, 0, -1, 4, 16, 0, 0, 16, None, None, None) == INVALID
+    # ring with null state
+    assert lib.fp8_quantize(16, 0, 4, 4, 16, 0, 0, 16, None, ctypes.byref(ring), None) == INVALID
+    # ring index out of range
+    ring2 = F.fp8_ring_t(256, 16, 16, 448.0, 1.0)
+    assert lib.fp8_quantize(16, 0, 4, 4, 16, 0, 0, 16, None, ctypes.byref(ring2), None) == INVALID
+    assert "hist_idx" in F.last_error()
+    # misaligned ring state
+    ring3 = F.fp8_ring_t(260, 16, 0, 448.0, 1.0)
+    assert lib.fp8_quantize(16, 0, 4, 4, 16, 0, 0, 16, None, ctypes.byref(ring3), None) == UNSUPPORTED
+    # dual needs both outputs
+    assert lib.fp8_quantize_dual(16, 0, 4, 4, 16, 0, 16, None, None, None, None) == INVALID
+
+
+def test_gemm_argument_checks():
+    lib = F.lib()
+    g = lib.fp8_gemm
+    ok = dict(a=256, b=512, fa=0, fb=0, lay=0, m=32, n=32, k=32, lda=32, ldb=32, ldo=32, batch=1,
+              sa=0, sb=0, so=0, pa=64, pb=64, bias=None, bs=None, out=1024)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return g(d["a"], d["b"], d["fa"], d["fb"], d["lay"], d["m"], d["n"], d["k"], d["lda"], d["ldb"], d["ldo"],
+                 d["batch"], d["sa"], d["sb"], d["so"], d["pa"], d["pb"], d["bias"], d["bs"], d["out"], None)
+
+    assert call(fa=3) == INVALID
+    assert call(lay=9) == INVALID
+    assert call(m=-1) == INVALID
+    assert call(out=None) == INVALID
+    assert call(pa=None) == INVALID
+    assert call(ldo=16) == INVALID                     # ldo < n
+    assert call(lda=16) == INVALID                     # lda < k for an N-layout A
+    assert call(lda=40) == UNSUPPORTED                 # not a multiple of 16
+    assert call(a=257) == UNSUPPORTED                  # misaligned operand
+    assert call(batch=2, sa=8, so=1024) == UNSUPPORTED  # batch stride not a multiple of 16
+    assert call(batch=2, so=0) == INVALID              # batches would overwrite each other
+    assert call(bias=None, bs=64) == INVALID           # bias_scale without bias
+    assert "bias_scale" in F.last_error()
+
+
+def test_linear_argument_checks():
+    lib = F.lib()
+    f = lib.linear_forward_fp8
+    ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
+    # k not a multiple of 16
+    assert f(256, 256, 0, None, None, None, 64, 60, 64, 0, None, None, 1.0, None, None, 1024, ws, 2048, None) == UNSUPPORTED
+    # workspace too small
+    assert f(256, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 1024, 16, 2048, None) == WORKSPACE
+    # misaligned workspace
+    assert f(256, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 1040, ws, 2048, None) == UNSUPPORTED
+    # fp8 weight without its step
+    assert f(256, 256, 1, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 1024, ws, 2048, None) == INVALID
+    b = lib.linear_backward_fp8
+    wsb = F.linear_backward_fp8_workspace_size(64, 64, 64)
+    # grad_w requested without x
+    assert b(256, None, 256, 64, 64, 64, 1, 0, 1, 0, None, None, None, 1.0, None, 1024, wsb, None, 4096, None, None) == INVALID
+    # delayed scaling without the forward's steps
+    ring = F.fp8_ring_t(256, 16, 0, 57344.0, 1.0)
+    assert b(256, 256, 256, 64, 64, 64, 1, 1, 1, 1, None, None, ctypes.byref(ring), 1.0, None, 1024, wsb,
+             4096, 4096, 4096, None) == INVALID
+
+
+def test_misc_argument_checks():
+    lib = F.lib()
+    assert lib.fp8_set_wait_timeout_ns(0) == INVALID
+    assert lib.fp8_profiler_read(7, None, None, None) == INVALID
+    assert lib.fp8_scale_ring_init(None, 16, None) == INVALID
+    assert lib.fp8_scale_ring_init(256, 0, None) == INVALID
+    assert lib.fp8_amax_scale(256, 0, 16, 448.0, 1.0, None, None, 256, None) == INVALID
+    assert lib.fp8_get_device_status(None, None) == INVALID
+    ring = F.Ring(None, 4)
+    for _ in range(5):
+        ring.advance()
+    assert ring.hist_idx == 1
