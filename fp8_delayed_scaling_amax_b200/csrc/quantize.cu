@@ -604,7 +604,8 @@ static int quantize_common(const void* x, fp8_in_t in_type, int64_t rows, int64_
     if (rows < 0 || cols < 0) return fail(FP8DSA_ERR_INVALID_ARG, "rows and cols must be >= 0");
     if (rows > 0 && cols > 0 && (x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "x is NULL");
     if (scale == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "scale is NULL");
-    if (out == nullptr && out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "output is NULL");
+    const bool empty = rows == 0 || cols == 0;
+    if (!empty && out == nullptr && out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "output is NULL");
     if (out_t != nullptr && (cols + kTile - 1) / kTile > 0x7FFFFFFF)
         return fail(FP8DSA_ERR_UNSUPPORTED, "too many columns");
     if (out_t != nullptr && (rows + kTile - 1) / kTile > 65535)
@@ -631,7 +632,7 @@ int fp8_quantize(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, co
                  fp8_fmt_t fmt, int transposed, uint8_t* out, float* amax_out, const fp8_ring_t* ring,
                  cudaStream_t stream) {
     clear_error();
-    if (out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out is NULL");
+    if (out == nullptr && rows > 0 && cols > 0) return fail(FP8DSA_ERR_INVALID_ARG, "out is NULL");
     return quantize_common(x, in_type, rows, cols, scale, fmt, transposed ? nullptr : out,
                            transposed ? out : nullptr, amax_out, ring, stream);
 }
@@ -640,7 +641,8 @@ int fp8_quantize_dual(const void* x, fp8_in_t in_type, int64_t rows, int64_t col
                       fp8_fmt_t fmt, uint8_t* out, uint8_t* out_t, float* amax_out, const fp8_ring_t* ring,
                       cudaStream_t stream) {
     clear_error();
-    if (out == nullptr || out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out and out_t are required");
+    if ((out == nullptr || out_t == nullptr) && rows > 0 && cols > 0)
+        return fail(FP8DSA_ERR_INVALID_ARG, "out and out_t are required");
     return quantize_common(x, in_type, rows, cols, scale, fmt, out, out_t, amax_out, ring, stream);
 }
 
