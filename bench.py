@@ -1,0 +1,602 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 linear layer with per-tensor delayed scaling on B200.
+
+One *step* is the whole hot path over one batch: the forward and backward (dX, dW, bias
+gradient) of every linear of a 12-layer, dim-1024 transformer trained at batch 4 x 512
+tokens (M = 2048 rows); per layer the (K, N) = (1024, 3072), (1024, 1024), (1024, 4096),
+(4096, 1024) projections.  HYBRID formats (E4M3 forward, E5M2 backward), delayed scaling with
+history 16 and margin 0 (every quantize folds its amax into its ring in its last block),
+bias fused into the forward GEMM.  Per linear and step: 3 quantizes + 1 GEMM forward,
+3 quantizes + 2 GEMMs + 1 column-sum backward.
+
+Timing: every layer has its own weights, activations and gradients (about 3 GB, far above
+the 126 MB L2).  The step is captured as CUDA graphs (one per history-ring slot, since the
+slot index is a host-side argument) and replayed; device time from CUDA events with a
+synchronize on both sides, max over ranks.  Per-kernel durations for the roofline come from
+the library's own CUDA-event profiler over instrumented eager steps of the same workload.
+
+``--impl reference`` times the CPU oracle (the plain restatement of the method, on the host
+cores) on a bounded sample of the same workload: one training linear per step.
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; N > 1 under torchrun runs one
+independent replica per GPU (the path has no exchange step: weak scaling).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 GEMM TFLOP/s (fwd/dX/dW) + quantize GB/s, % of B200 roofline"
+UNIT = "TFLOP/s"
+HIST = 16
+WORKLOAD = ("training linears of a 12-layer dim-1024 transformer at B4xT512 (M=2048), HYBRID "
+            "(E4M3 fwd, E5M2 bwd), delayed scaling history 16 margin 0, bias, fwd+dX+dW+grad_b")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=600)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-sweeps", action="store_true")
+    p.add_argument("--kernel", default=None, choices=["gemm", "quantize"],
+                   help="time one kernel on one shape instead of the step (small cases for ncu)")
+    p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS")
+    p.add_argument("--qmode", default="dual", choices=["row", "t", "dual"])
+    return p.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------
+def oracle_linear_step(k, n, seed):
+    """The oracle's forward + backward of one training linear; returns (seconds, flops)."""
+    import numpy as np
+    import workloads as W
+    from oracle import linear as L
+    from oracle import scaling as S
+
+    m = W.TRAINING_TOKENS
+    t = W.training_linear(m, k, n, seed)
+    bits = {key: W.bf16_bits(t[key]) for key in ("x", "w", "b", "g")}
+    rx, rw, rg = S.Ring(HIST, "e4m3"), S.Ring(HIST, "e4m3"), S.Ring(HIST, "e5m2")
+    f32 = {key: t[key].float().numpy() for key in ("x", "w", "g")}
+    rx.seed(f32["x"])
+    rw.seed(f32["w"])
+    rg.seed(f32["g"])
+    t0 = time.perf_counter()
+    f = L.forward(bits["x"], bits["w"], bits["b"], "e4m3", rx, rw)
+    L.backward(bits["g"], bits["x"], bits["w"], "e5m2", f["sx"], f["sw"], rg)
+    dt = time.perf_counter() - t0
+    del np
+    return dt, 3 * 2.0 * m * k * n
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline():
+    import workloads as W
+    total_t, total_f = 0.0, 0.0
+    for i, (k, n) in enumerate(W.TRAINING_LINEARS):
+        dt, fl = oracle_linear_step(k, n, seed=7000 + i)
+        total_t += dt
+        total_f += fl
+    return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": "one transformer layer (its 4 training linears, M=2048) forward + backward through the "
+                      f"numpy oracle (fp64 GEMMs): {total_f / 1e9:.1f} GFLOP in {total_t:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import workloads as W
+    for i in range(args.warmup):
+        k, n = W.TRAINING_LINEARS[i % 4]
+        oracle_linear_step(k, n, seed=8000 + i)
+    total_t, total_f = 0.0, 0.0
+    for i in range(args.steps):
+        k, n = W.TRAINING_LINEARS[i % 4]
+        dt, fl = oracle_linear_step(k, n, seed=9000 + i)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    sample = (f"one training linear (M=2048, (K,N) cycling over the 4 shapes) forward + backward per step "
+              f"through the numpy oracle; {args.steps} steps, {total_t:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t * 1e3 / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": "one linear per step"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+# GPU workload
+# ---------------------------------------------------------------------------------------
+class Linear:
+    def __init__(self, F, W, torch, m, k, n, seed, dev):
+        self.F, self.m, self.k, self.n = F, m, k, n
+        t = W.training_linear(m, k, n, seed, device=dev)
+        self.x, self.w, self.b, self.g = t["x"], t["w"], t["b"], t["g"]
+        bf = torch.bfloat16
+        self.y = torch.empty((m, n), dtype=bf, device=dev)
+        self.gx = torch.empty((m, k), dtype=bf, device=dev)
+        self.gw = torch.empty((n, k), dtype=bf, device=dev)
+        self.gb = torch.empty((n,), dtype=bf, device=dev)
+        self.fws_n = F.linear_forward_fp8_workspace_size(m, k, n)
+        self.bws_n = F.linear_backward_fp8_workspace_size(m, k, n)
+        self.fws = torch.empty(self.fws_n, dtype=torch.uint8, device=dev)
+        self.bws = torch.empty(self.bws_n, dtype=torch.uint8, device=dev)
+        self.state = torch.zeros((3, HIST + 4), dtype=torch.float32, device=dev)
+        self.steps = torch.zeros(4, dtype=torch.float32, device=dev)  # sx, sw, sg
+        for i in range(3):
+            F.fp8_scale_ring_init(self.state[i], HIST)
+        self.rx = F.Ring(self.state[0], HIST, F.FP8_E4M3)
+        self.rw = F.Ring(self.state[1], HIST, F.FP8_E4M3)
+        self.rg = F.Ring(self.state[2], HIST, F.FP8_E5M2)
+        F.fp8_scale_ring_seed(self.rx, self.x, F.FP8_IN_BF16, self.x.numel())
+        F.fp8_scale_ring_seed(self.rw, self.w, F.FP8_IN_BF16, self.w.numel())
+        F.fp8_scale_ring_seed(self.rg, self.g, F.FP8_IN_BF16, self.g.numel())
+
+    def set_slot(self, idx):
+        self.rx.hist_idx = self.rw.hist_idx = self.rg.hist_idx = idx
+
+    def fwd(self):
+        F = self.F
+        F.linear_forward_fp8(self.x, self.w, 0, None, self.b, None, self.m, self.k, self.n, F.FP8_E4M3, self.rx,
+                             self.rw, 1.0, self.steps[0:1], self.steps[1:2], self.fws, self.fws_n, self.y)
+
+    def bwd(self):
+        F = self.F
+        F.linear_backward_fp8(self.g, self.x, self.w, self.m, self.k, self.n, F.FP8_E5M2, 1, 1, 1,
+                              self.steps[0:1], self.steps[1:2], self.rg, 1.0, self.steps[2:3], self.bws,
+                              self.bws_n, self.gx, self.gw, self.gb)
+
+    @property
+    def gemm_flops(self):
+        return 3 * 2.0 * self.m * self.k * self.n
+
+    @property
+    def quant_bytes(self):
+        m, k, n = self.m, self.k, self.n
+        # fwd: x, w row-major (2 B in, 1 B out); bwd: g dual (2 + 1 + 1), x^T, w^T (2 + 1)
+        return 3 * (m * k + n * k) + 4 * m * n + 3 * (m * k + n * k)
+
+
+def build_workload(F, W, torch, dev, seed_base):
+    lins = []
+    for layer in range(W.TRAINING_LAYERS):
+        for j, (k, n) in enumerate(W.TRAINING_LINEARS):
+            lins.append(Linear(F, W, torch, W.TRAINING_TOKENS, k, n, seed_base + 100 * layer + 10 * j, dev))
+    return lins
+
+
+def run_step(lins, slot):
+    for lin in lins:
+        lin.set_slot(slot)
+    for lin in lins:
+        lin.fwd()
+    for lin in reversed(lins):
+        lin.bwd()
+
+
+# ---------------------------------------------------------------------------------------
+# Clocks and peaks
+# ---------------------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def start_clock_sampler(torch, dev):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    ids = [v.strip() for v in vis.split(",") if v.strip()] if vis else []
+    target = ids[dev.index] if dev.index is not None and dev.index < len(ids) else str(dev.index or 0)
+    cmd = ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+    if target:
+        cmd += ["-i", target]
+    try:
+        return subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    except Exception:
+        return None
+
+
+def stop_clock_sampler(proc):
+    if proc is None:
+        return None
+    proc.terminate()
+    try:
+        out, _ = proc.communicate(timeout=10)
+    except Exception:
+        proc.kill()
+        return None
+    sm, mx, reasons = [], [], set()
+    names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    for line in out.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[5:9]):
+            if val.lower().startswith("active"):
+                reasons.add(name)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on the
+    current GEMM source (its hash is recorded there); otherwise None."""
+    import hashlib
+    summary = os.path.join(ROOT, "profiles", "fp8_gemm_training_linears_traffic.txt")
+    src = os.path.join(ROOT, "fp8_delayed_scaling_amax_b200", "csrc", "gemm.cu")
+    try:
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        vals = {}
+        with open(summary) as f:
+            for line in f:
+                if "=" in line and not line.lstrip().startswith("#"):
+                    key, v = line.split("=", 1)
+                    vals[key.strip()] = v.strip()
+        if vals.get("gemm_source_sha256_16") != h:
+            return None
+        return float(vals["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------------
+# Single-kernel timing: rotate enough input sets that the bytes touched exceed twice the L2,
+# so every launch reads its operands from HBM.
+# ---------------------------------------------------------------------------------------
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _graph_time(torch, launch, iters, warmup, slots=1):
+    """Capture `iters` back-to-back launches in CUDA graphs and time their replay, so host
+    launch cost does not show up in the device time.  `slots` > 1 captures one graph per
+    history-ring slot (the slot index is a host argument baked into the capture)."""
+    cap = torch.cuda.Stream()
+    for i in range(warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for sl in range(slots):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(iters):
+                launch(i)
+        graphs.append(g)
+    graphs[0].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for g in graphs:
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (iters * slots)
+
+
+def time_gemm(F, W, torch, dev, m, n, k, iters=20, warmup=5, batch=1, bcast_b=False):
+    per_set = batch * m * k + (1 if bcast_b else batch) * n * k + batch * m * n * 2
+    nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
+    sets = []
+    for i in range(nsets):
+        a = W.fp8_bytes((batch, m, k), seed=31 + i, device=dev)
+        b = W.fp8_bytes((1 if bcast_b else batch, n, k), seed=57 + i, device=dev)
+        out = torch.empty((batch, m, n), dtype=torch.bfloat16, device=dev)
+        sets.append((a, b, out))
+    sa = torch.tensor([0.75], device=dev)
+    sb = torch.tensor([1.5], device=dev)
+    bias = W.normal_bf16((n,), 0.1, seed=5, device=dev)
+
+    def launch(i):
+        a, b, out = sets[i % nsets]
+        F.fp8_gemm(a, b, 0, 0, F.FP8_LAYOUT_NT, m, n, k, k, k, n, batch, m * k if batch > 1 else 0,
+                   0 if (bcast_b or batch == 1) else n * k, m * n, sa, sb, bias, None, out)
+
+    ms = _graph_time(torch, launch, iters, warmup)
+    return {"ms": ms, "tflops": 2.0 * batch * m * n * k / (ms * 1e-3) / 1e12, "sets": nsets}
+
+
+def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5):
+    per_set = rows * cols * (2 + (2 if mode == "dual" else 1))
+    nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
+    sets = []
+    for i in range(nsets):
+        x = W.normal_bf16((rows, cols), 1.0, seed=80 + i, device=dev)
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+        out_t = torch.empty((cols, rows), dtype=torch.uint8, device=dev)
+        st = torch.zeros(HIST + 4, dtype=torch.float32, device=dev)
+        F.fp8_scale_ring_init(st, HIST)
+        ring = F.Ring(st, HIST, F.FP8_E4M3)
+        F.fp8_scale_ring_seed(ring, x, F.FP8_IN_BF16, x.numel())
+        sets.append((x, out, out_t, ring))
+
+    def launch(i):
+        x, out, out_t, ring = sets[i % nsets]
+        step = ring.state[HIST:HIST + 1]
+        if mode == "row":
+            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, 0, out, None, ring)
+        elif mode == "t":
+            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, 1, out_t, None, ring)
+        else:
+            F.fp8_quantize_dual(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, out, out_t, None, ring)
+        ring.advance()
+
+    ms = _graph_time(torch, launch, iters, warmup)
+    nbytes = rows * cols * (2 + (2 if mode == "dual" else 1))
+    return {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "sets": nsets}
+
+
+def run_kernel_mode(args):
+    import torch
+    import fp8_delayed_scaling_amax_b200 as F
+    import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dims = [int(v) for v in args.shape.split(",")]
+    peaks = measured_peaks()
+    if args.kernel == "gemm":
+        m, n, k = dims
+        r = time_gemm(F, W, torch, dev, m, n, k, iters=args.steps, warmup=args.warmup)
+        r.update(kernel="fp8_gemm", shape=[m, n, k], frac=r["tflops"] / (2 * peaks["bf16_tflops"]))
+    else:
+        rows, cols = dims
+        r = time_quantize(F, W, torch, dev, rows, cols, args.qmode, iters=args.steps, warmup=args.warmup)
+        r.update(kernel=f"fp8_quantize_{args.qmode}", shape=[rows, cols], frac=r["gbs"] / peaks["hbm_gbs"])
+    r["status"] = F.fp8_get_device_status()
+    print(json.dumps(r), flush=True)
+    return 0
+
+
+def run_sweeps(F, W, torch, dev):
+    """Square NT GEMMs (pre-quantized E4M3, bias on), the skinny / batched shapes, and the
+    quantize bandwidth sweep, each timed alone with operands rotated through HBM."""
+    peaks = measured_peaks()
+    burst_fp8 = 2.0 * peaks["bf16_tflops"]
+    out = {"gemm_square": {}, "gemm_skinny_batched": {}, "quantize": {}}
+    for s in W.SQUARE_SIZES:
+        r = time_gemm(F, W, torch, dev, s, s, s, iters=20 if s < 8192 else 10)
+        out["gemm_square"][str(s)] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
+                                      "frac": round(r["tflops"] / burst_fp8, 4)}
+    for ba, bb, m, n, k in W.SKINNY_BATCHED:
+        batch = max(ba, bb)
+        r = time_gemm(F, W, torch, dev, m, n, k, batch=batch, bcast_b=(bb == 1 and batch > 1))
+        key = f"{batch}x{m}x{n}x{k}" + ("(B bcast)" if bb == 1 and batch > 1 else "")
+        out["gemm_skinny_batched"][key] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
+                                           "frac": round(r["tflops"] / burst_fp8, 4)}
+    for rows, cols in ((4096, 4096), (8192, 8192), (16384, 16384)):
+        for mode in ("row", "t", "dual"):
+            r = time_quantize(F, W, torch, dev, rows, cols, mode)
+            out["quantize"][f"{mode}_{rows}x{cols}"] = {"gbs": round(r["gbs"], 1), "us": round(r["ms"] * 1e3, 2),
+                                                       "frac": round(r["gbs"] / peaks["hbm_gbs"], 4)}
+    out["peaks"] = {"fp8_tflops_burst": burst_fp8, "hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"]}
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.kernel is not None:
+        return run_kernel_mode(args) if rank == 0 else 0
+
+    import torch
+    import torch.distributed as dist
+
+    import fp8_delayed_scaling_amax_b200 as F
+    import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    F.lib()
+
+    lins = build_workload(F, W, torch, dev, seed_base=100000 * rank)
+    flops_step = sum(l.gemm_flops for l in lins)
+    qbytes_step = sum(l.quant_bytes for l in lins)
+
+    # eager warm step (module load, attributes), then one graph per ring slot
+    run_step(lins, 0)
+    torch.cuda.synchronize()
+    assert F.fp8_get_device_status() == 0
+    cap = torch.cuda.Stream()
+    graphs = []
+    for slot in range(HIST):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            run_step(lins, slot)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    counter = [1]  # the eager warm step used slot 0
+
+    def replay():
+        graphs[counter[0] % HIST].replay()
+        counter[0] += 1
+
+    for t in range(args.warmup):
+        replay()
+    torch.cuda.synchronize()
+    sampler = start_clock_sampler(torch, dev) if rank == 0 or world == 1 else None
+    time.sleep(0.6)  # let the sampler start before the timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for t in range(args.steps):
+        replay()
+    end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = stop_clock_sampler(sampler)
+    ms = start.elapsed_time(end)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    status = F.fp8_get_device_status()
+
+    # per-kernel durations: the same step captured again with the library's profiler on
+    # (an event-record node on each side of every kernel), each of the 16 slot graphs
+    # replayed once, then every event pair read back
+    F.fp8_profiler_read(0), F.fp8_profiler_read(1), F.fp8_profiler_read(2)
+    F.fp8_profiler_enable(True)
+    timed_graphs = []
+    for slot in range(HIST):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            run_step(lins, slot)
+        timed_graphs.append(g)
+    F.fp8_profiler_enable(False)
+    for t in range(HIST):
+        timed_graphs[counter[0] % HIST].replay()
+        counter[0] += 1
+    torch.cuda.synchronize()
+    n_instr = HIST
+    q_ms, q_n, q_bytes = F.fp8_profiler_read(0)
+    g_ms, g_n, g_flops = F.fp8_profiler_read(1)
+    o_ms, o_n, _ = F.fp8_profiler_read(2)
+    launches_per_step = (q_n + g_n + o_n) / n_instr
+
+    # end to end through the public API: activations and gradients copied in from pinned host
+    # memory every step, bias gradients and the used steps read back every step
+    e2e = None
+    if not args.no_e2e:
+        host_in = [(l.x, torch.empty_like(l.x, device="cpu").pin_memory(), l.g,
+                    torch.empty_like(l.g, device="cpu").pin_memory()) for l in lins]
+        host_out = [(l.gb, torch.empty_like(l.gb, device="cpu").pin_memory(), l.steps,
+                     torch.empty_like(l.steps, device="cpu").pin_memory()) for l in lins]
+        for dx, hx, dg, hg in host_in:
+            hx.copy_(dx)
+            hg.copy_(dg)
+        h2d = sum(l.x.numel() * 2 + l.g.numel() * 2 for l in lins)
+        d2h = sum(l.gb.numel() * 2 + l.steps.numel() * 4 for l in lins)
+        e2e_steps = max(3, min(args.steps, 40))
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for t in range(e2e_steps):
+            for dx, hx, dg, hg in host_in:
+                dx.copy_(hx, non_blocking=True)
+                dg.copy_(hg, non_blocking=True)
+            replay()
+            for dgb, hgb, dst, hst in host_out:
+                hgb.copy_(dgb, non_blocking=True)
+                hst.copy_(dst, non_blocking=True)
+        e2.record()
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": flops_step * e2e_steps * world / (float(e_ms.item()) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+    del graphs, timed_graphs
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = measured_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]  # fp8 dense = 2 x bf16 (nominal 4.5 / 2.25 PF)
+    gemm_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else 0.0
+    quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9 if q_ms > 0 else 0.0
+    traffic = gemm_traffic_per_launch()
+    value = flops_step * args.steps * world / (ms_max * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": W.TRAINING_LAYERS, "tokens": W.TRAINING_TOKENS,
+                   "linears_kn": [list(kn) for kn in W.TRAINING_LINEARS],
+                   "l2": "inputs larger than L2: every layer has its own x, w, g (about 3 GB working set)",
+                   "graphs": f"one CUDA graph per history slot ({HIST})",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+        "gemm_flops_per_step": flops_step, "quantize_bytes_per_step": qbytes_step,
+        "kernels": {"gemm_tflops": gemm_tflops, "gemm_ms_per_step": g_ms / n_instr,
+                    "quantize_gbs": quant_gbs, "quantize_ms_per_step": q_ms / n_instr,
+                    "other_ms_per_step": o_ms / n_instr,
+                    "quantize_frac_of_hbm": quant_gbs / peaks["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp8_peak,
+                     "traffic": traffic,
+                     "peak_note": f"fp8 dense = 2 x {peaks['source']} sustained bf16 "
+                                  f"({peaks['bf16_tflops_sustained']} TFLOP/s), of {peaks['source']}"},
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "device_status": status,
+    }
+    if clocks:
+        line["clocks"] = clocks
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_sweeps:
+        line["sweeps"] = run_sweeps(F, W, torch, dev)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

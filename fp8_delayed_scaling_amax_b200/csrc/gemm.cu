@@ -16,8 +16,9 @@
 //    TMEM accumulator; tcgen05.commit releases each stage and, per tile, hands the
 //    accumulator to the epilogue.  Two accumulators (2 x BN TMEM columns) let the epilogue
 //    of tile i overlap the MMAs of tile i + 1;
-//  * warps 2-5 = epilogue: tcgen05.ld 32 columns at a time, fma with the combined scale and
-//    the bias, round to bf16, 128-bit stores;
+//  * warps 2-5 = epilogue: tcgen05.ld 64 columns at a time, fma with the combined scale and
+//    the bias, round to bf16, stage each warp's 32 x 64 box in 128-byte-swizzled shared
+//    memory and write it with a TMA bulk-tensor store (double-buffered per warp);
 //  * every wait is bounded (globaltimer); on expiry the CTA records a status code, drains its
 //    in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -40,15 +41,18 @@ constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
 constexpr int kThreads = 192; // 6 warps
 constexpr int kEpiThreads = 128;
 
+constexpr int kOutBox = 64;                       // output columns per TMA store (128 bytes of bf16)
+constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 columns
+
 template <int BN>
 struct Cfg {
     static constexpr int kStages = BN == 256 ? 4 : 6;
     static constexpr int kAStage = kBM * kBK;
     static constexpr int kBStage = BN * kBK;
     static constexpr int kTmemCols = 2 * BN;
+    static constexpr int kOutBytes = 4 * 2 * kOutStageBytes;  // 4 epilogue warps x 2 buffers
     static constexpr int kBarBytes = 256;
-    static constexpr int kBiasBytes = 4 * BN * 4;  // one bias copy per epilogue warp
-    static constexpr int kSmem = 1024 + kStages * (kAStage + kBStage) + kBarBytes + kBiasBytes;
+    static constexpr int kSmem = 1024 + kStages * (kAStage + kBStage) + kOutBytes + kBarBytes;
 };
 
 struct GemmArgs {
@@ -60,6 +64,7 @@ struct GemmArgs {
     uint16_t* out;
     int64_t ldo, stride_o;
     int vec_out;
+    int tma_out;  // stage the tile in shared memory and write it with TMA bulk-tensor stores
     const void* bias;
     int bias_kind;  // 0 none, 1 bf16, 2 fp8 e4m3 * bias_scale, 3 fp8 e5m2 * bias_scale
     const float* bias_scale;
@@ -101,21 +106,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                    const GemmArgs g) {
+                    const __grid_constant__ CUtensorMap tma_o, const GemmArgs g) {
     using C = Cfg<BN>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + S * C::kAStage;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::kBStage);
+    uint8_t* sOut = sB + S * C::kBStage;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kOutBytes);
     uint64_t* empty = full + S;
     uint64_t* acc_full = empty + S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* bias_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -136,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tma_a);
         prefetch_tensormap(&tma_b);
+        if (g.tma_out) prefetch_tensormap(&tma_o);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -248,59 +254,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // this warp may access TMEM lanes 32q .. 32q+31
-        const int row_in_tile = q * 32 + lane;
-        float* my_bias = bias_s + (warp - 2) * BN;
+        // Warp w may read TMEM lanes 32*(w%4) .. +31, i.e. tile rows 32*(w%4) + lane.  Per 64
+        // output columns: two 32-column TMEM loads, acc * scale + bias in fp32, one bf16
+        // rounding, then either a swizzled shared-memory stage + TMA bulk store of the warp's
+        // 32 x 64 box (double-buffered), or direct 128-bit stores.
+        const int q = warp & 3;
+        uint8_t* my_stage = sOut + (warp - 2) * 2 * kOutStageBytes;
         const float sc = __fmul_rn(__ldg(g.scale_a), __ldg(g.scale_b));
         const float bsc = g.bias_kind >= 2 ? __ldg(g.bias_scale) : 0.0f;
-        int acc = 0;
+        auto bias_at = [&](int col) -> float {
+            if (col >= g.n || g.bias_kind == 0) return 0.0f;
+            if (g.bias_kind == 1) return bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(g.bias) + col));
+            const uint8_t v = __ldg(static_cast<const uint8_t*>(g.bias) + col);
+            return __fmul_rn(g.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
+        };
+        int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x) {
             int b, tm, tn;
             decode_tile(tile, g, b, tm, tn);
             const int col0 = tn * BN;
-            // this warp's copy of the tile's bias, as fp32
-            __syncwarp();
-            for (int c = lane; c < BN; c += 32) {
-                const int col = col0 + c;
-                float bv = 0.0f;
-                if (col < g.n) {
-                    if (g.bias_kind == 1)
-                        bv = bf16_bits_to_float(static_cast<const uint16_t*>(g.bias)[col]);
-                    else if (g.bias_kind == 2)
-                        bv = __fmul_rn(fp8_to_float<0>(static_cast<const uint8_t*>(g.bias)[col]), bsc);
-                    else if (g.bias_kind == 3)
-                        bv = __fmul_rn(fp8_to_float<1>(static_cast<const uint8_t*>(g.bias)[col]), bsc);
-                }
-                my_bias[c] = bv;
-            }
-            __syncwarp();
+            const int row0 = tm * kBM + q * 32;
+            const int64_t row = static_cast<int64_t>(row0) + lane;
             if (!mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue)) break;
             tc_fence_after_sync();
-            const int64_t row = static_cast<int64_t>(tm) * kBM + row_in_tile;
-            uint16_t* orow = g.out + static_cast<int64_t>(b) * g.stride_o + row * g.ldo;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t r[32];
-                tmem_load_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c), r);
+            for (int c = 0; c < BN; c += kOutBox) {
+                uint32_t r0[32], r1[32];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c);
+                tmem_load_32cols(taddr, r0);
+                tmem_load_32cols(taddr + 32, r1);
+                const float b_lo = bias_at(col0 + c + lane);
+                const float b_hi = bias_at(col0 + c + 32 + lane);
                 tmem_wait_ld();
-                const int colg = col0 + c;
-                if (row < g.m && colg < g.n) {
-                    uint32_t packed[16];
+                uint32_t packed[32];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float v0 = fmaf(__uint_as_float(r[2 * e]), sc, my_bias[c + 2 * e]);
-                        const float v1 = fmaf(__uint_as_float(r[2 * e + 1]), sc, my_bias[c + 2 * e + 1]);
-                        packed[e] = pack_bf16x2(v0, v1);
+                for (int e = 0; e < 16; ++e) {
+                    const float v0 = fmaf(__uint_as_float(r0[2 * e]), sc, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e));
+                    const float v1 = fmaf(__uint_as_float(r0[2 * e + 1]), sc, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e + 1));
+                    packed[e] = pack_bf16x2(v0, v1);
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float v0 = fmaf(__uint_as_float(r1[2 * e]), sc, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e));
+                    const float v1 = fmaf(__uint_as_float(r1[2 * e + 1]), sc, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e + 1));
+                    packed[16 + e] = pack_bf16x2(v0, v1);
+                }
+                const int colg = col0 + c;
+                if (g.tma_out) {
+                    uint8_t* sb = my_stage + buf * kOutStageBytes;
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used this buffer has read it
+                    __syncwarp();
+                    // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r % 8)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && row0 < g.m && colg < g.n) {
+                        tma_store_3d(&tma_o, sb, colg, row0, b);
+                        bulk_commit_group();
                     }
-                    if (g.vec_out && colg + 32 <= g.n) {
+                    buf ^= 1;
+                } else if (row < g.m && colg < g.n) {
+                    uint16_t* orow = g.out + static_cast<int64_t>(b) * g.stride_o + row * g.ldo;
+                    if (g.vec_out && colg + kOutBox <= g.n) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + colg);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
+                        for (int v = 0; v < 8; ++v)
                             dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                     } else {
-                        for (int e = 0; e < 32 && colg + e < g.n; ++e)
-                            orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
+#pragma unroll
+                        for (int e = 0; e < kOutBox; ++e)
+                            if (colg + e < g.n) orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
                     }
                 }
             }
@@ -311,6 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_phase ^= 1u;
             }
         }
+        if (g.tma_out && lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before_sync();
@@ -352,18 +381,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D uint8 tensor map: dims {inner, outer, batch}, row stride `ld` bytes, batch stride
-// `bstride` bytes, box {128, box_outer, 1}, 128-byte swizzle, zero fill out of bounds.
-int make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t batch, int64_t ld,
-             int64_t bstride, int box_outer) {
+// 3-D tensor map: dims {inner, outer, batch} elements, row stride `ld` bytes, batch stride
+// `bstride` bytes, box {box_inner, box_outer, 1}, 128-byte swizzle, zero fill out of bounds.
+int make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner, int64_t outer,
+             int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_outer) {
     auto fn = encode_fn();
     if (fn == nullptr) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
                                 static_cast<cuuint64_t>(batch)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(bstride)};
-    const cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_outer), 1u};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
@@ -371,7 +400,8 @@ int make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, i
 }
 
 template <int BN>
-int launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& g, int64_t batch, cudaStream_t stream) {
+int launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, GemmArgs& g, int64_t batch,
+              cudaStream_t stream) {
     using C = Cfg<BN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -387,21 +417,17 @@ int launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& g, int64_t
     if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
     g.num_tiles = static_cast<int>(tiles);
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
-    fp8_gemm_kernel<BN><<<grid, kThreads, C::kSmem, stream>>>(ma, mb, g);
+    fp8_gemm_kernel<BN><<<grid, kThreads, C::kSmem, stream>>>(ma, mb, mo, g);
     return FP8DSA_OK;
 }
 
-// Choose the tile width: fewer waves x narrower tiles wins; ties go to the wider tile
-// (half the operand traffic per flop).
+// Tile width: 128 x 256 tiles unless the problem is at most 128 wide.  A 128 x 128 x 32 MMA
+// reads as many operand bytes from shared memory per flop as the TMA writes into it, and was
+// measured far slower than the 256-wide tile even where it quantizes the waves better.
 int choose_bn(int64_t m, int64_t n, int64_t batch) {
-    if (n <= 128) return 128;
-    const int64_t sms = sm_count();
-    const int64_t tm = (m + kBM - 1) / kBM;
-    const int64_t t256 = tm * ((n + 255) / 256) * batch;
-    const int64_t t128 = tm * ((n + 127) / 128) * batch;
-    const int64_t cost256 = ((t256 + sms - 1) / sms) * 256;
-    const int64_t cost128 = ((t128 + sms - 1) / sms) * 128;
-    return cost128 < cost256 ? 128 : 256;
+    (void)m;
+    (void)batch;
+    return n <= 128 ? 128 : 256;
 }
 
 }  // namespace
@@ -425,18 +451,28 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
     const bool b_bat = stride_b != 0 && batch > 1;
     const int bn = choose_bn(m, n, batch);
 
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo;
     int rc;
+    const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
     if (!a_mn)
-        rc = make_map(&ma, a, k, m, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * m, kBM);
+        rc = make_map(&ma, u8, a, k, m, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * m, 128, kBM);
     else
-        rc = make_map(&ma, a, m, k, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * k, kBK);
+        rc = make_map(&ma, u8, a, m, k, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * k, 128, kBK);
     if (rc) return rc;
     if (!b_mn)
-        rc = make_map(&mb, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, bn);
+        rc = make_map(&mb, u8, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, 128, bn);
     else
-        rc = make_map(&mb, b, n, k, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * k, kBK);
+        rc = make_map(&mb, u8, b, n, k, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * k, 128, kBK);
     if (rc) return rc;
+    // TMA stores need 16-byte aligned rows and batches of the output
+    const bool tma_out = aligned16(out) && ldo % 8 == 0 && (batch == 1 || stride_o % 8 == 0);
+    if (tma_out) {
+        rc = make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, n, m, batch, ldo * 2,
+                      batch > 1 ? stride_o * 2 : ldo * 2 * m, kOutBox, 32);
+        if (rc) return rc;
+    } else {
+        mo = ma;  // unused placeholder
+    }
 
     GemmArgs g{};
     g.m = static_cast<int>(m);
@@ -455,6 +491,7 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
     g.ldo = ldo;
     g.stride_o = stride_o;
     g.vec_out = aligned16(out) && ldo % 8 == 0 && stride_o % 8 == 0;
+    g.tma_out = tma_out;
     g.bias = bias;
     g.bias_kind = bias_kind;
     g.bias_scale = bias_scale;
@@ -464,7 +501,7 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
     if (rc) return rc;
 
     launch_begin(kKindGemm, stream);
-    rc = bn == 256 ? launch_bn<256>(ma, mb, g, batch, stream) : launch_bn<128>(ma, mb, g, batch, stream);
+    rc = bn == 256 ? launch_bn<256>(ma, mb, mo, g, batch, stream) : launch_bn<128>(ma, mb, mo, g, batch, stream);
     if (rc) return rc;
     launch_end(kKindGemm, stream, flops);
     return check_launch("fp8 gemm kernel");

@@ -121,6 +121,29 @@ __device__ __forceinline__ uint8_t convert1(float v, float mult) {
     return static_cast<uint8_t>(cvt_fp8x2<kFmt>(__fmul_rn(v, mult), 0.0f) & 0xFFu);
 }
 
+// Device-scope acquire-release fetch-add: orders this thread's earlier writes (its block's
+// amax) before the increment, and later reads after it.
+__device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
+
+constexpr int kHistPrefetch = 64;
+
+__device__ __forceinline__ float* hist_smem() {
+    __shared__ float s_hist[kHistPrefetch];
+    return s_hist;
+}
+
+// Called at kernel start: copy the ring's history window (it does not change during the
+// kernel; only the last block writes it, at the very end) into shared memory, so the fold
+// does not pay one dependent L2 round trip per slot.  Visible after block_finish's barrier.
+__device__ __forceinline__ void ring_prefetch(const QArgs& a) {
+    if (a.ring_state != nullptr && a.hist_len <= kHistPrefetch && static_cast<int>(threadIdx.x) < a.hist_len)
+        hist_smem()[threadIdx.x] = __ldcg(a.ring_state + threadIdx.x);
+}
+
 // Block-wide amax reduce, one atomic per block, then (with a ring) the last-block fold:
 // scale_used = step, hist[idx] = amax, scale = max(RN32(peak / fp8_max) / 2^m, 1e-12),
 // amax and done slots re-zeroed.  Every thread of the block must call this.
@@ -139,16 +162,20 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
         float* st = a.ring_state;
         const int n = a.hist_len;
         unsigned* done = reinterpret_cast<unsigned*>(st + n + 3);
-        __threadfence();
         const unsigned nblocks = gridDim.x * gridDim.y * gridDim.z;
-        const unsigned ticket = atomicAdd(done, 1u);
+        const unsigned ticket = ticket_acq_rel(done);
         if (ticket != nblocks - 1u) return;
-        __threadfence();
         const float am = __uint_as_float(atomicOr(reinterpret_cast<unsigned*>(st + n + 2), 0u));
         st[n + 1] = step;
         st[a.hist_idx] = am;
         float peak = am;
-        for (int i = 0; i < n; ++i) peak = fmaxf(peak, __ldcg(st + i));
+        if (n <= kHistPrefetch) {
+            const float* h = hist_smem();
+            for (int i = 0; i < n; ++i)
+                if (i != a.hist_idx) peak = fmaxf(peak, h[i]);
+        } else {
+            for (int i = 0; i < n; ++i) peak = fmaxf(peak, __ldcg(st + i));
+        }
         st[n] = fmaxf(__fdiv_rn(__fdiv_rn(peak, a.fp8_max), a.pow2_margin), 1e-12f);
         st[n + 2] = 0.0f;
         atomicExch(done, 0u);
@@ -164,6 +191,7 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
 // ----------------------------------------------------------------------------------------
 template <class In, int kFmt>
 __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(QArgs a) {
+    ring_prefetch(a);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
@@ -212,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 
     __shared__ __align__(16) uint32_t tile[kTile * 32];
     __shared__ float csum[kColsum ? 8 : 1][kColsum ? kTile : 1];
 
+    ring_prefetch(a);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
@@ -377,10 +406,8 @@ __global__ void __launch_bounds__(kThreads) amax_jobs_kernel(AmaxArgs a) {
     for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
     uint32_t* scr = a.scratch[job];
     atomicMax(scr, __float_as_uint(m));
-    __threadfence();
-    const unsigned ticket = atomicAdd(scr + 1, 1u);
+    const unsigned ticket = ticket_acq_rel(scr + 1);
     if (ticket != gridDim.x - 1u) return;
-    __threadfence();
     const float am = __uint_as_float(atomicOr(scr, 0u));
     float peak = am;
     if (a.ring_state[job] != nullptr) {
@@ -401,8 +428,20 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
                                                                     int64_t cols, uint16_t* out) {
     const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (c >= cols) return;
+    // in-order sum (deterministic); the loads are independent and issued four at a time
     float s = 0.0f;
-    for (int64_t t = 0; t < tiles; ++t) s += __ldcg(partial + t * cols + c);
+    int64_t t = 0;
+    for (; t + 4 <= tiles; t += 4) {
+        const float v0 = __ldcg(partial + t * cols + c);
+        const float v1 = __ldcg(partial + (t + 1) * cols + c);
+        const float v2 = __ldcg(partial + (t + 2) * cols + c);
+        const float v3 = __ldcg(partial + (t + 3) * cols + c);
+        s += v0;
+        s += v1;
+        s += v2;
+        s += v3;
+    }
+    for (; t < tiles; ++t) s += __ldcg(partial + t * cols + c);
     out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
 }
 

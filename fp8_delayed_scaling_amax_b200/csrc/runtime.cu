@@ -102,19 +102,29 @@ int wait_ctl(WaitCtl* ctl) {
     return FP8DSA_OK;
 }
 
+// Record `e` on `stream`.  Inside a stream capture the record becomes an external event-record
+// node of the graph, so every replay of the graph timestamps it again.
+void record_event(cudaEvent_t e, cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, stream);
+}
+
 void launch_begin(int kind, cudaStream_t stream) {
     (void)kind;
     if (!g_profile.load()) return;
     std::lock_guard<std::mutex> lock(g_mutex);
     t_pending_start = take_event();
-    cudaEventRecord(t_pending_start, stream);
+    record_event(t_pending_start, stream);
 }
 
 void launch_end(int kind, cudaStream_t stream, double work) {
     if (!g_profile.load() || t_pending_start == nullptr) return;
     std::lock_guard<std::mutex> lock(g_mutex);
     cudaEvent_t stop = take_event();
-    cudaEventRecord(stop, stream);
+    record_event(stop, stream);
     g_timed[kind].push_back({t_pending_start, stop, work});
     t_pending_start = nullptr;
 }

@@ -196,10 +196,11 @@ int fp8_set_wait_timeout_ns(uint64_t ns);
 int fp8_debug_stalled_wait(cudaStream_t stream);
 
 /* Per-kernel timing: when enabled, every kernel the library launches is bracketed by CUDA
- * events on its own stream.  fp8_profiler_read synchronises, returns the total device
- * milliseconds and launch count of kernel class `kind` (0 quantize, 1 GEMM, 2 other) since
- * the last reset, then resets that class.  Not on the pages (they time with CUDA events
- * from Python; [by-author]). */
+ * events on its own stream (inside a stream capture, by external event-record nodes, so each
+ * replay of the graph re-times them).  fp8_profiler_read synchronises, returns the total
+ * device milliseconds, launch count and algorithmic bytes (quantize, other) or flops (GEMM)
+ * of kernel class `kind` (0 quantize, 1 GEMM, 2 other) recorded since the last read, then
+ * resets that class.  Not on the pages (they time with CUDA events from Python; [by-author]). */
 int fp8_profiler_enable(int on);
 int fp8_profiler_read(int kind, double* total_ms, int64_t* launches, double* bytes_or_flops);
 
