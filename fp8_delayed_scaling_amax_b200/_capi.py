@@ -48,6 +48,8 @@ _SIGNATURES = {
     "linear_forward_fp8_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_forward_fp8": (c_int, [_P, _P, c_int, _P, _P, _P, c_int64, c_int64, c_int64, c_int,
                                    POINTER(fp8_ring_t), POINTER(fp8_ring_t), c_float, _P, _P, _P, c_size_t, _P, _P]),
+    "linear_forward_fp8_noalloc": (c_int, [_P, _P, c_int, _P, _P, _P, c_int64, c_int64, c_int64, c_int,
+                                           POINTER(fp8_ring_t), POINTER(fp8_ring_t), c_float, _P, _P, _P, _P]),
     "linear_backward_fp8_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_backward_fp8": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, _P, _P,
                                     POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P, _P]),
@@ -197,6 +199,19 @@ def linear_forward_fp8(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x
         _ptr(x), _ptr(w), int(bool(w_is_fp8)), _ptr(w_step), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n),
         int(fmt), _ring(x_ring), _ring(w_ring), float(pow2_margin), _ptr(sx_used), _ptr(sw_used), _ptr(workspace),
         int(workspace_bytes), _ptr(y), _stream(stream)))
+
+
+def linear_forward_fp8_noalloc(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
+                               sx_used, sw_used, y, stream=None):
+    """linear_forward_fp8 with the library's built-in scratch array instead of a workspace,
+    for callers that cannot allocate device memory."""
+    return _check("linear_forward_fp8_noalloc", lib().linear_forward_fp8_noalloc(
+        _ptr(x), _ptr(w), int(bool(w_is_fp8)), _ptr(w_step), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n),
+        int(fmt), _ring(x_ring), _ring(w_ring), float(pow2_margin), _ptr(sx_used), _ptr(sw_used), _ptr(y),
+        _stream(stream)))
+
+
+NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 
 def linear_backward_fp8(g, x, w, m, k, n, fmt, need_grad_x, need_grad_w, need_grad_b, sx_fwd, sw_fwd, g_ring,

@@ -156,6 +156,26 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
                        float pow2_margin, float* sx_used, float* sw_used, void* workspace,
                        size_t workspace_bytes, void* y, cudaStream_t stream);
 
+/* Size of the scratch array linear_forward_fp8_noalloc uses instead of a caller workspace. */
+#define FP8DSA_NOALLOC_WORKSPACE_BYTES (16u << 20)
+
+/* linear_forward_fp8 for callers that cannot allocate device memory -- for example code that
+ * runs inside a CUDA stream capture (where allocating is not allowed), a plug-in whose host
+ * application owns the device-memory budget, or a service that must keep a fixed device
+ * footprint.  The pages have no counterpart to this entry point.
+ * Same arguments and results as linear_forward_fp8, without the workspace: the scratch lives
+ * in one built-in device array of FP8DSA_NOALLOC_WORKSPACE_BYTES (16 MiB), held by every GPU
+ * that loads the library until the process exits.  Shapes whose
+ * linear_forward_fp8_workspace_size exceeds it return FP8DSA_ERR_WORKSPACE with a message.
+ * The first call on each device looks up the array's address (make it before any stream
+ * capture); no call allocates.  All calls share the array: calls ordered on one stream are
+ * safe, calls that overlap on the GPU race. */
+int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is_fp8, const float* w_step,
+                               const void* bias, const float* bias_scale, int64_t m, int64_t k,
+                               int64_t n, fp8_fmt_t fmt, const fp8_ring_t* x_ring,
+                               const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                               float* sw_used, void* y, cudaStream_t stream);
+
 /* Workspace bytes linear_backward_fp8 needs for (m, k, n). */
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
 

@@ -1,0 +1,79 @@
+"""The allocation-free forward entry point (`linear_forward_fp8_noalloc`).
+
+It serves callers that cannot allocate device memory when they run the forward pass (for
+example inside a CUDA stream capture, or a plug-in whose host owns the memory budget): its
+scratch is one built-in 16 MiB device array instead of a caller workspace.  Here it is
+called through the C ABI twice in a row and its output is compared with the workspace
+entry point's, within the GEMM bound the other tests use.  This file is named so pytest
+collects it last.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import fp8_delayed_scaling_amax_b200 as F
+import workloads as W
+from oracle import linear as L
+from helpers import bf16_out_to_f64, assert_within_gemm_bound
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _ring(fmt):
+    st = torch.zeros(16 + 4, dtype=torch.float32, device=DEV)
+    F.fp8_scale_ring_init(st, 16)
+    return F.Ring(st, 16, fmt)
+
+
+def _forward_both(t, delayed, rings):
+    x, w, b = (t[key].to(DEV) for key in ("x", "w", "b"))
+    m, k = x.shape
+    n = w.shape[0]
+    nbytes = F.linear_forward_fp8_workspace_size(m, k, n)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    y_ws = torch.empty((m, n), dtype=torch.bfloat16, device=DEV)
+    y_na = torch.empty((m, n), dtype=torch.bfloat16, device=DEV)
+    s_ws = torch.zeros(2, device=DEV)
+    s_na = torch.zeros(2, device=DEV)
+    (rx1, rw1), (rx2, rw2) = rings if delayed else ((None, None), (None, None))
+    F.linear_forward_fp8(x, w, 0, None, b, None, m, k, n, F.FP8_E4M3, rx1, rw1, 1.0, s_ws[0:1], s_ws[1:2], ws,
+                         nbytes, y_ws)
+    F.linear_forward_fp8_noalloc(x, w, 0, None, b, None, m, k, n, F.FP8_E4M3, rx2, rw2, 1.0, s_na[0:1], s_na[1:2],
+                                 y_na)
+    torch.cuda.synchronize()
+    return y_ws, y_na, s_ws, s_na
+
+
+@pytest.mark.parametrize("delayed", [False, True])
+def test_noalloc_forward_matches_workspace_forward_twice(delayed):
+    rings = [(_ring(F.FP8_E4M3), _ring(F.FP8_E4M3)) for _ in range(2)]
+    for call in range(2):
+        t = W.training_linear(384, 512, 640, seed=500 + call)
+        if delayed and call == 0:
+            for rx, rw in rings:
+                F.fp8_scale_ring_seed(rx, t["x"].to(DEV), F.FP8_IN_BF16, t["x"].numel())
+                F.fp8_scale_ring_seed(rw, t["w"].to(DEV), F.FP8_IN_BF16, t["w"].numel())
+        y_ws, y_na, s_ws, s_na = _forward_both(t, delayed, rings)
+        assert torch.equal(s_ws, s_na)
+        f = L.forward(W.bf16_bits(t["x"]), W.bf16_bits(t["w"]), W.bf16_bits(t["b"]), "e4m3")
+        # the two entry points against each other, with the bound the GEMM tests use
+        assert_within_gemm_bound(bf16_out_to_f64(y_na), bf16_out_to_f64(y_ws), f["s_abs"], f["sc"],
+                                 f"no-alloc vs workspace, call {call}")
+        if delayed:
+            assert torch.equal(rings[0][0].state, rings[1][0].state)
+            assert torch.equal(rings[0][1].state, rings[1][1].state)
+            for rx, rw in rings:
+                rx.advance()
+                rw.advance()
+    assert F.fp8_get_device_status() == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_array():
+    m, k, n = 4096, 4096, 4096  # needs 32 MiB of operand scratch
+    assert F.linear_forward_fp8_workspace_size(m, k, n) > F.NOALLOC_WORKSPACE_BYTES
+    with pytest.raises(F.FP8Error) as err:
+        F.linear_forward_fp8_noalloc(16, 16, 0, None, None, None, m, k, n, F.FP8_E4M3, None, None, 1.0, None, None,
+                                     16)
+    assert err.value.code == -5 and "built-in array" in str(err.value)
