@@ -56,6 +56,7 @@ _SIGNATURES = {
     "fp8_get_device_status": (c_int, [_P, POINTER(c_int)]),
     "fp8_set_wait_timeout_ns": (c_int, [c_uint64]),
     "fp8_debug_stalled_wait": (c_int, [_P]),
+    "fp8_set_pdl": (c_int, [c_int]),
     "fp8_profiler_enable": (c_int, [c_int]),
     "fp8_profiler_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double)]),
     "fp8_last_error": (c_char_p, []),
@@ -230,6 +231,10 @@ def fp8_get_device_status(stream=None) -> int:
 
 def fp8_set_wait_timeout_ns(ns: int):
     return _check("fp8_set_wait_timeout_ns", lib().fp8_set_wait_timeout_ns(int(ns)))
+
+
+def fp8_set_pdl(enabled: bool = True):
+    return _check("fp8_set_pdl", lib().fp8_set_pdl(int(bool(enabled))))
 
 
 def fp8_debug_stalled_wait(stream=None):

@@ -44,15 +44,20 @@ constexpr int kEpiThreads = 128;
 constexpr int kOutBox = 64;                       // output columns per TMA store (128 bytes of bf16)
 constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 columns
 
-template <int BN>
+// kPair: a 2-CTA cluster computes a 256 x BN tile with one M = 256 MMA across both SMs; each CTA
+// holds 128 rows of A and BN/2 rows of B, so each SM's shared memory feeds half the B operand.
+template <int BN, bool kPair>
 struct Cfg {
-    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kTileM = kPair ? 2 * kBM : kBM;
+    static constexpr int kBRows = kPair ? BN / 2 : BN;  // rows of B (along N) this CTA loads
     static constexpr int kAStage = kBM * kBK;
-    static constexpr int kBStage = BN * kBK;
+    static constexpr int kBStage = kBRows * kBK;
+    static constexpr int kStages = (kAStage + kBStage) <= 32768 ? 6 : 4;
     static constexpr int kTmemCols = 2 * BN;
     static constexpr int kOutBytes = 4 * 2 * kOutStageBytes;  // 4 epilogue warps x 2 buffers
     static constexpr int kBarBytes = 256;
     static constexpr int kSmem = 1024 + kStages * (kAStage + kBStage) + kOutBytes + kBarBytes;
+    static constexpr uint32_t kTxBytes = (kPair ? 2u : 1u) * (kAStage + kBStage);
 };
 
 struct GemmArgs {
@@ -103,11 +108,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN>
+__device__ __forceinline__ float bias_value(const GemmArgs& g, int col, float bsc) {
+    if (col >= g.n || g.bias_kind == 0) return 0.0f;
+    if (g.bias_kind == 1) return bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(g.bias) + col));
+    const uint8_t v = __ldg(static_cast<const uint8_t*>(g.bias) + col);
+    return __fmul_rn(g.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
+}
+
+template <int BN, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                     const __grid_constant__ CUtensorMap tma_o, const GemmArgs g) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, kPair>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -124,6 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    pdl_trigger();
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -132,7 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full + a, 1);
-            mbar_init(acc_empty + a, kEpiThreads);
+            // the leader's accumulator is released by both CTAs' epilogue threads
+            mbar_init(acc_empty + a, kEpiThreads * (kPair ? 2 : 1));
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -144,13 +162,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (g.tma_out) prefetch_tensormap(&tma_o);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::kTmemCols);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(tmem_slot, C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();  // the peer's loads target the leader's initialised barriers
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // the operands and steps come from the previous kernels
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
@@ -159,29 +184,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;  // per-stage: ever issued, parity of the last issue
             bool ok = true;
-            for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
+            for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
                 int b, tm, tn;
                 decode_tile(tile, g, b, tm, tn);
                 const int ba = g.a_batched ? b : 0;
                 const int bb = g.b_batched ? b : 0;
+                const int arow = tm * C::kTileM + static_cast<int>(rank) * kBM;
+                const int brow = tn * BN + static_cast<int>(rank) * C::kBRows;
                 for (int kb = 0; kb < g.k_blocks; ++kb) {
                     if (!mbar_wait_bounded(empty + stage, phase ^ 1u, g.wait, abort_flag, kStatusWaitProducer)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full + stage, C::kAStage + C::kBStage);
+                    if (leader) mbar_arrive_expect_tx(full + stage, C::kTxBytes);
                     uint8_t* a_dst = sA + stage * C::kAStage;
                     uint8_t* b_dst = sB + stage * C::kBStage;
-                    if (!g.a_mn)
-                        tma_load_3d(a_dst, &tma_a, full + stage, kb * kBK, tm * kBM, ba);
-                    else
-                        tma_load_3d(a_dst, &tma_a, full + stage, tm * kBM, kb * kBK, ba);
-                    if (!g.b_mn) {
-                        tma_load_3d(b_dst, &tma_b, full + stage, kb * kBK, tn * BN, bb);
-                    } else {
+                    if constexpr (kPair) {
+                        const uint32_t fb = mapa_shared(smem_addr(full + stage), 0);
+                        if (!g.a_mn)
+                            tma_load_3d_pair(a_dst, &tma_a, fb, kb * kBK, arow, ba);
+                        else
+                            tma_load_3d_pair(a_dst, &tma_a, fb, arow, kb * kBK, ba);
+                        if (!g.b_mn) {
+                            tma_load_3d_pair(b_dst, &tma_b, fb, kb * kBK, brow, bb);
+                        } else {
 #pragma unroll
-                        for (int h = 0; h < BN / 128; ++h)
-                            tma_load_3d(b_dst + h * 128 * kBK, &tma_b, full + stage, tn * BN + h * 128, kb * kBK, bb);
+                            for (int h = 0; h < C::kBRows / 128; ++h)
+                                tma_load_3d_pair(b_dst + h * 128 * kBK, &tma_b, fb, brow + h * 128, kb * kBK, bb);
+                        }
+                    } else {
+                        if (!g.a_mn)
+                            tma_load_3d(a_dst, &tma_a, full + stage, kb * kBK, arow, ba);
+                        else
+                            tma_load_3d(a_dst, &tma_a, full + stage, arow, kb * kBK, ba);
+                        if (!g.b_mn) {
+                            tma_load_3d(b_dst, &tma_b, full + stage, kb * kBK, brow, bb);
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < C::kBRows / 128; ++h)
+                                tma_load_3d(b_dst + h * 128 * kBK, &tma_b, full + stage, brow + h * 128, kb * kBK, bb);
+                        }
                     }
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -191,8 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (!ok) {
-                // Let every copy already in flight land before the CTA can exit.
+            if (!ok && leader) {
+                // Let every copy already in flight land before the CTAs can exit (the leader's
+                // full barriers also count the peer's bytes).
                 for (int s = 0; s < S; ++s)
                     if (issued & (1u << s))
                         mbar_wait_bounded(full + s, (issued_parity >> s) & 1u, g.wait, nullptr, kStatusWaitDrain);
@@ -200,92 +243,112 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
-        int stage = 0, acc = 0;
-        uint32_t phase = 0, acc_phase = 0;
-        bool ok = true;
-        constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
-        for (int tile = blockIdx.x; tile < g.num_tiles && ok; tile += gridDim.x) {
-            if (!mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag, kStatusWaitMma)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait_bounded(full + stage, phase, g.wait, abort_flag, kStatusWaitMma)) {
+        // ------------------------------------------------------------------ MMA issuer (leader)
+        if (leader) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
+            for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
+                const bool got = kPair ? mbar_wait_bounded_cluster(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
+                                                                   kStatusWaitMma)
+                                       : mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
+                                                           kStatusWaitMma);
+                if (!got) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t a_base = smem_addr(sA + stage * C::kAStage);
-                    const uint32_t b_base = smem_addr(sB + stage * C::kBStage);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        // K-major: step 32 bytes along the swizzled row; MN-major: step 32 rows.
-                        const uint64_t ad = g.a_mn ? smem_desc(a_base + kk * kUmmaK * 128, C::kAStage, 1024)
-                                                   : smem_desc(a_base + kk * kUmmaK, 16, 1024);
-                        const uint64_t bd = g.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
-                                                   : smem_desc(b_base + kk * kUmmaK, 16, 1024);
-                        umma_f8f6f4(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait_bounded(full + stage, phase, g.wait, abort_flag, kStatusWaitMma)) {
+                        ok = false;
+                        break;
                     }
-                    umma_commit(empty + stage);
+                    tc_fence_after_sync();
+                    if (lane == 0) {
+                        const uint32_t a_base = smem_addr(sA + stage * C::kAStage);
+                        const uint32_t b_base = smem_addr(sB + stage * C::kBStage);
+#pragma unroll
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            // K-major: step 32 bytes along the swizzled row; MN-major: step 32 rows.
+                            const uint64_t ad = g.a_mn ? smem_desc(a_base + kk * kUmmaK * 128, C::kAStage, 1024)
+                                                       : smem_desc(a_base + kk * kUmmaK, 16, 1024);
+                            const uint64_t bd = g.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
+                                                       : smem_desc(b_base + kk * kUmmaK, 16, 1024);
+                            if constexpr (kPair)
+                                umma_f8f6f4_pair(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                            else
+                                umma_f8f6f4(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        if constexpr (kPair)
+                            umma_commit_pair_multicast(empty + stage, 0x3);
+                        else
+                            umma_commit(empty + stage);
+                    }
+                    __syncwarp();
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) {
+                    if constexpr (kPair)
+                        umma_commit_pair_multicast(acc_full + acc, 0x3);
+                    else
+                        umma_commit(acc_full + acc);
                 }
                 __syncwarp();
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
                 }
             }
-            if (!ok) break;
-            if (lane == 0) umma_commit(acc_full + acc);
-            __syncwarp();
-            if (++acc == 2) {
-                acc = 0;
-                acc_phase ^= 1u;
+            // Every MMA this thread issued must complete before TMEM is released.
+            if (lane == 0) {
+                if constexpr (kPair)
+                    umma_commit_pair(drain);
+                else
+                    umma_commit(drain);
+                mbar_wait_bounded(drain, 0, g.wait, nullptr, kStatusWaitDrain);
             }
-        }
-        // Every MMA this thread issued must complete before TMEM is released.
-        if (lane == 0) {
-            umma_commit(drain);
-            mbar_wait_bounded(drain, 0, g.wait, nullptr, kStatusWaitDrain);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ epilogue
-        // Warp w may read TMEM lanes 32*(w%4) .. +31, i.e. tile rows 32*(w%4) + lane.  Per 64
-        // output columns: two 32-column TMEM loads, acc * scale + bias in fp32, one bf16
-        // rounding, then either a swizzled shared-memory stage + TMA bulk store of the warp's
-        // 32 x 64 box (double-buffered), or direct 128-bit stores.
+        // Warp w may read TMEM lanes 32*(w%4) .. +31, i.e. rows 32*(w%4) + lane of this CTA's
+        // 128-row half of the tile.  Per 64 output columns: two 32-column TMEM loads,
+        // acc * scale + bias in fp32, one bf16 rounding, then either a swizzled shared-memory
+        // stage + TMA bulk store of the warp's 32 x 64 box (double-buffered), or direct
+        // 128-bit stores.
         const int q = warp & 3;
         uint8_t* my_stage = sOut + (warp - 2) * 2 * kOutStageBytes;
         const float sc = __fmul_rn(__ldg(g.scale_a), __ldg(g.scale_b));
         const float bsc = g.bias_kind >= 2 ? __ldg(g.bias_scale) : 0.0f;
-        auto bias_at = [&](int col) -> float {
-            if (col >= g.n || g.bias_kind == 0) return 0.0f;
-            if (g.bias_kind == 1) return bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(g.bias) + col));
-            const uint8_t v = __ldg(static_cast<const uint8_t*>(g.bias) + col);
-            return __fmul_rn(g.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
-        };
+        const uint32_t acc_empty_leader0 = kPair ? mapa_shared(smem_addr(acc_empty), 0) : 0u;
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x) {
+        for (int tile = unit; tile < g.num_tiles; tile += units) {
             int b, tm, tn;
             decode_tile(tile, g, b, tm, tn);
             const int col0 = tn * BN;
-            const int row0 = tm * kBM + q * 32;
+            const int row0 = tm * C::kTileM + static_cast<int>(rank) * kBM + q * 32;
             const int64_t row = static_cast<int64_t>(row0) + lane;
+            // this tile's bias, column col0 + 32 j + lane in bias_r[j], loaded before the wait
+            float bias_r[BN / 32];
+#pragma unroll
+            for (int j = 0; j < BN / 32; ++j) bias_r[j] = bias_value(g, col0 + 32 * j + lane, bsc);
             if (!mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue)) break;
             tc_fence_after_sync();
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < BN; c += kOutBox) {
                 uint32_t r0[32], r1[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c);
                 tmem_load_32cols(taddr, r0);
                 tmem_load_32cols(taddr + 32, r1);
-                const float b_lo = bias_at(col0 + c + lane);
-                const float b_hi = bias_at(col0 + c + 32 + lane);
+                const float b_lo = bias_r[c / 32];
+                const float b_hi = bias_r[c / 32 + 1];
                 tmem_wait_ld();
                 uint32_t packed[32];
 #pragma unroll
@@ -332,7 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(acc_empty + acc);
+            if constexpr (kPair) {
+                if (leader)
+                    mbar_arrive(acc_empty + acc);
+                else
+                    mbar_arrive_cluster(acc_empty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+            } else {
+                mbar_arrive(acc_empty + acc);
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -344,13 +414,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();  // neither CTA releases TMEM or exits while the peer still uses it
     tc_fence_after_sync();
-    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    if (warp == 1) {
+        if constexpr (kPair)
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        else
+            tmem_dealloc(tmem_base, C::kTmemCols);
+    }
 }
 
 // k == 0: the product is empty; out = bias (or 0), rounded to bf16.
 __global__ void bias_fill_kernel(uint16_t* out, int64_t m, int64_t n, int64_t ldo, int64_t stride_o, int64_t batch,
                                  const void* bias, int bias_kind, const float* bias_scale) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = batch * m * n;
     const float bsc = bias_kind >= 2 ? __ldg(bias_scale) : 0.0f;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -399,35 +477,66 @@ int make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int6
     return FP8DSA_OK;
 }
 
-template <int BN>
-int launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, GemmArgs& g, int64_t batch,
-              cudaStream_t stream) {
-    using C = Cfg<BN>;
+template <int BN, bool kPair>
+int launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, GemmArgs& g, int64_t batch,
+               cudaStream_t stream) {
+    using C = Cfg<BN, kPair>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
+    static int max_units = 0;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (attr_err != cudaSuccess) return;
+        if (kPair) {
+            // how many 2-CTA clusters of this kernel fit on the device at once
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 2;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(2 * 74, 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = C::kSmem;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, kPair>, &cfg) == cudaSuccess && n > 0)
+                max_units = n;
+            cudaGetLastError();
+        }
     });
     if (attr_err != cudaSuccess)
         return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(attr_err));
+    g.tiles_m = static_cast<int>((g.m + C::kTileM - 1) / C::kTileM);
     g.tiles_n = (g.n + BN - 1) / BN;
-    g.idesc |= (static_cast<uint32_t>(BN >> 3) << 17);
-    const int64_t per = static_cast<int64_t>(g.tiles_m) * g.tiles_n;
-    const int64_t tiles = per * batch;
+    g.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
+    const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n * batch;
     if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
     g.num_tiles = static_cast<int>(tiles);
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count()));
-    fp8_gemm_kernel<BN><<<grid, kThreads, C::kSmem, stream>>>(ma, mb, mo, g);
+    const int units = kPair ? (max_units > 0 ? max_units : sm_count() / 2) : sm_count();
+    const int grid_units = static_cast<int>(std::min<int64_t>(tiles, units));
+    cudaError_t e = launch_ex(fp8_gemm_kernel<BN, kPair>, dim3(static_cast<unsigned>(grid_units * (kPair ? 2 : 1))),
+                              dim3(kThreads), C::kSmem, stream, kPair ? 2 : 1, ma, mb, mo, g);
+    if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("fp8 gemm launch: ") + cudaGetErrorString(e));
     return FP8DSA_OK;
 }
 
-// Tile width: 128 x 256 tiles unless the problem is at most 128 wide.  A 128 x 128 x 32 MMA
-// reads as many operand bytes from shared memory per flop as the TMA writes into it, and was
-// measured far slower than the 256-wide tile even where it quantizes the waves better.
+// Tile shape: 256 x 256 tiles on CTA pairs when M > 128 (each SM then reads half of the B
+// operand from its shared memory); 128 x 256 on one CTA otherwise; 128-wide tiles only when N
+// is at most 128.  A 128 x 128 x 32 MMA reads as many operand bytes from shared memory per flop
+// as the TMA writes into it, and measured far slower than the 256-wide tile.
 int choose_bn(int64_t m, int64_t n, int64_t batch) {
     (void)m;
     (void)batch;
     return n <= 128 ? 128 : 256;
+}
+
+bool choose_pair(int64_t m, int64_t n, int b_mn) {
+    if (m <= kBM) return false;
+    if (n <= 128) return false;  // pair tiles keep 256 columns (128 per CTA: one MN-major swizzle block)
+    (void)b_mn;
+    return true;
 }
 
 }  // namespace
@@ -442,14 +551,16 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
         const int64_t total = batch * m * n;
         const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 8));
         launch_begin(kKindOther, stream);
-        bias_fill_kernel<<<blocks, 256, 0, stream>>>(static_cast<uint16_t*>(out), m, n, ldo, stride_o, batch, bias,
-                                                     bias_kind, bias_scale);
+        launch_ex(bias_fill_kernel, dim3(blocks), dim3(256), 0, stream, 1, static_cast<uint16_t*>(out), m, n, ldo,
+                  stride_o, batch, bias, bias_kind, bias_scale);
         launch_end(kKindOther, stream, static_cast<double>(total) * 2);
         return check_launch("bias fill kernel");
     }
     const bool a_bat = stride_a != 0 && batch > 1;
     const bool b_bat = stride_b != 0 && batch > 1;
     const int bn = choose_bn(m, n, batch);
+    const bool pair = bn == 256 && choose_pair(m, n, b_mn);
+    const int b_rows = pair ? bn / 2 : bn;  // rows of B each CTA loads
 
     CUtensorMap ma, mb, mo;
     int rc;
@@ -460,7 +571,7 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
         rc = make_map(&ma, u8, a, m, k, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * k, 128, kBK);
     if (rc) return rc;
     if (!b_mn)
-        rc = make_map(&mb, u8, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, 128, bn);
+        rc = make_map(&mb, u8, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, 128, b_rows);
     else
         rc = make_map(&mb, u8, b, n, k, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * k, 128, kBK);
     if (rc) return rc;
@@ -478,15 +589,13 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
     g.m = static_cast<int>(m);
     g.n = static_cast<int>(n);
     g.k = static_cast<int>(k);
-    g.tiles_m = static_cast<int>((m + kBM - 1) / kBM);
     g.k_blocks = static_cast<int>((k + kBK - 1) / kBK);
     g.a_batched = a_bat;
     g.b_batched = b_bat;
     g.a_mn = a_mn;
     g.b_mn = b_mn;
     g.idesc = (1u << 4) | (static_cast<uint32_t>(fmt_a) << 7) | (static_cast<uint32_t>(fmt_b) << 10) |
-              (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
-              (static_cast<uint32_t>(kBM >> 4) << 24);
+              (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
     g.out = static_cast<uint16_t*>(out);
     g.ldo = ldo;
     g.stride_o = stride_o;
@@ -501,7 +610,11 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
     if (rc) return rc;
 
     launch_begin(kKindGemm, stream);
-    rc = bn == 256 ? launch_bn<256>(ma, mb, mo, g, batch, stream) : launch_bn<128>(ma, mb, mo, g, batch, stream);
+    if (pair)
+        rc = launch_cfg<256, true>(ma, mb, mo, g, batch, stream);
+    else
+        rc = bn == 256 ? launch_cfg<256, false>(ma, mb, mo, g, batch, stream)
+                       : launch_cfg<128, false>(ma, mb, mo, g, batch, stream);
     if (rc) return rc;
     launch_end(kKindGemm, stream, flops);
     return check_launch("fp8 gemm kernel");

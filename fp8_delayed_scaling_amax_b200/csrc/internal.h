@@ -8,7 +8,7 @@
 #include <cstdint>
 #include <string>
 
-#include "../../include/fp8dsa.h"
+#include "fp8dsa.h"
 #include "device.cuh"
 
 namespace fp8dsa {
@@ -36,6 +36,39 @@ void launch_end(int kind, cudaStream_t stream, double work);
 
 // After a launch: map a launch failure to FP8DSA_ERR_CUDA.
 int check_launch(const char* what);
+
+// Whether library kernels are launched with programmatic dependent launch (default on).
+bool pdl_enabled();
+
+// Launch `kernel` with optional 1-D cluster size and, when enabled, programmatic stream
+// serialization (the kernel overlaps its launch and prologue with the previous kernel's tail;
+// every library kernel waits in pdl_wait before touching data an earlier kernel wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      int cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    if (cluster_x > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl_enabled()) {
+        at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -83,6 +116,9 @@ struct QuantJob {
     float* colsum_partial = nullptr;  // [ceil(rows/128)][cols] fp32 column sums (tiled only)
 };
 int launch_quantize(const QuantJob& job, cudaStream_t stream);
+// Up to three tensors in one launch (same format, input type and orientation); each tensor
+// keeps its own amax, ticket and ring fold.
+int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream);
 
 // grad_b[c] = RN_bf16(sum_t partial[t][c]) in a fixed order.
 int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,

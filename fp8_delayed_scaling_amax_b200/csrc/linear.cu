@@ -8,9 +8,9 @@
 // grad_w = g8T . x8T^T, both NT; grad_b = column sum of g).
 //
 // Launches per call (delayed scaling):
-//   forward : quantize x (ring fold) + quantize w (ring fold) + GEMM                  = 3
-//   backward: dual quantize g (ring fold + per-tile column sums) + transposed quantize x
-//             + transposed quantize w + GEMM dX + GEMM dW + column-sum finalize       = 6
+//   forward : one quantize launch for x and w (each folds its own ring) + GEMM           = 2
+//   backward: one quantize launch for g (both orientations, ring fold, per-tile column
+//             sums), x^T and w^T + GEMM dX + GEMM dW + column-sum finalize            = 4
 // The snapshot of each step is written by the folding kernel itself (no clone launches), so
 // the GEMM dequantizes with exactly the step the bytes were quantized with.
 #include <cuda_runtime.h>
@@ -168,8 +168,9 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
         qx.ring = x_ring;
         qx.scale_used_out = sx;
     }
-    rc = launch_quantize(qx, stream);
-    if (rc) return rc;
+    QuantJob fwd_jobs[2];
+    int nfj = 0;
+    fwd_jobs[nfj++] = qx;
     if (!w_is_fp8) {
         QuantJob qw;
         qw.x = w;
@@ -184,9 +185,11 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
             qw.ring = w_ring;
             qw.scale_used_out = sw;
         }
-        rc = launch_quantize(qw, stream);
-        if (rc) return rc;
+        fwd_jobs[nfj++] = qw;
     }
+    // x and w in one launch, each with its own amax, ticket and ring fold
+    rc = launch_quantize_batch(fwd_jobs, nfj, stream);
+    if (rc) return rc;
     int bias_kind = 0;
     if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt == FP8_E4M3 ? 2 : 3);
     return gemm_launch(x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y,
@@ -283,8 +286,10 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         qg.ring = g_ring;
         qg.scale_used_out = sg;
     }
-    rc = launch_quantize(qg, stream);
-    if (rc) return rc;
+    // g (both orientations), x^T and w^T in one launch
+    QuantJob bwd_jobs[3];
+    int nbj = 0;
+    bwd_jobs[nbj++] = qg;
     if (need_grad_w) {
         QuantJob qx;
         qx.x = x;
@@ -293,8 +298,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         qx.fmt = fmt;
         qx.out_t = x8t;
         qx.scale = sx;
-        rc = launch_quantize(qx, stream);
-        if (rc) return rc;
+        bwd_jobs[nbj++] = qx;
     }
     if (need_grad_x) {
         QuantJob qw;
@@ -304,8 +308,11 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         qw.fmt = fmt;
         qw.out_t = w8t;
         qw.scale = sw;
-        rc = launch_quantize(qw, stream);
-        if (rc) return rc;
+        bwd_jobs[nbj++] = qw;
+    }
+    rc = launch_quantize_batch(bwd_jobs, nbj, stream);
+    if (rc) return rc;
+    if (need_grad_x) {
         // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T
         rc = gemm_launch(g8, w8t, fmt, fmt, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x,
                          stream);

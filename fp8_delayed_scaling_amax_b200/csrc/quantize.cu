@@ -100,8 +100,17 @@ struct QArgs {
     int hist_len, hist_idx;
     float fp8_max, pow2_margin;
     float* scale_used_out;     // receives the step used, or null
-    float* colsum;             // [gridDim.y][cols] per-tile column sums, or null
+    float* colsum;             // [row tiles][cols] per-tile column sums (tiled kernel), or null
     int vec_in, vec_out, vec_out_t;
+    unsigned nblocks;          // blocks working on this tensor (the ticket count of its fold)
+    int tile_begin, tiles_x;   // tiled kernel: first block of this tensor, column tiles
+};
+
+// Up to three tensors quantized by one launch; each keeps its own amax, ticket and fold.
+constexpr int kMaxJobs = 3;
+struct QBatch {
+    QArgs job[kMaxJobs];
+    int njobs;
 };
 
 // Eight floats -> eight fp8 bytes (two words), updating amax over the raw values.
@@ -147,7 +156,7 @@ __device__ __forceinline__ void ring_prefetch(const QArgs& a) {
 // Block-wide amax reduce, one atomic per block, then (with a ring) the last-block fold:
 // scale_used = step, hist[idx] = amax, scale = max(RN32(peak / fp8_max) / 2^m, 1e-12),
 // amax and done slots re-zeroed.  Every thread of the block must call this.
-__device__ __forceinline__ void block_finish(const QArgs& a, float amax, float step) {
+__device__ __forceinline__ void block_finish(const QArgs& a, float amax, float step, bool first_block) {
     __shared__ float red[32];
     const int tid = threadIdx.x;
     amax = warp_max(amax);
@@ -162,9 +171,8 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
         float* st = a.ring_state;
         const int n = a.hist_len;
         unsigned* done = reinterpret_cast<unsigned*>(st + n + 3);
-        const unsigned nblocks = gridDim.x * gridDim.y * gridDim.z;
         const unsigned ticket = ticket_acq_rel(done);
-        if (ticket != nblocks - 1u) return;
+        if (ticket != a.nblocks - 1u) return;
         const float am = __uint_as_float(atomicOr(reinterpret_cast<unsigned*>(st + n + 2), 0u));
         st[n + 1] = step;
         st[a.hist_idx] = am;
@@ -181,7 +189,7 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
         atomicExch(done, 0u);
         if (a.amax_out != nullptr) *a.amax_out = am;
         if (a.scale_used_out != nullptr) *a.scale_used_out = step;
-    } else if (a.scale_used_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0) {
+    } else if (a.scale_used_out != nullptr && first_block) {
         *a.scale_used_out = step;
     }
 }
@@ -190,7 +198,10 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
 // Row-major quantize: flat, grid-stride, 16 elements per thread per iteration.
 // ----------------------------------------------------------------------------------------
 template <class In, int kFmt>
-__global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(QArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_constant__ QBatch batch) {
+    pdl_trigger();
+    pdl_wait();
+    const QArgs& a = batch.job[blockIdx.y];  // one grid row of blocks per tensor
     ring_prefetch(a);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
@@ -228,25 +239,35 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(QArgs a) {
         amax = fmaxf(amax, fabsf(v));
         a.out[i] = convert1<kFmt>(v, mult);
     }
-    block_finish(a, amax, step);
+    block_finish(a, amax, step, blockIdx.x == 0);
 }
 
 // ----------------------------------------------------------------------------------------
 // Transposed / dual quantize: 128 x 128 tiles through a swizzled shared byte tile.
 // ----------------------------------------------------------------------------------------
-template <class In, int kFmt, bool kRowOut, bool kColsum>
-__global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 4) quant_tiled_kernel(QArgs a) {
+template <class In, int kFmt>
+__global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 3)
+    quant_tiled_kernel(const __grid_constant__ QBatch batch) {
     // 128 rows x 128 bytes; the 16-byte chunk c of row r lives at chunk c ^ ((r >> 4) & 7).
     __shared__ __align__(16) uint32_t tile[kTile * 32];
-    __shared__ float csum[kColsum ? 8 : 1][kColsum ? kTile : 1];
+    __shared__ float csum[8][kTile];
 
+    pdl_trigger();
+    pdl_wait();
+    int jb = 0;
+    while (jb + 1 < batch.njobs && static_cast<int>(blockIdx.x) >= batch.job[jb + 1].tile_begin) ++jb;
+    const QArgs& a = batch.job[jb];
+    const bool row_out = a.out != nullptr;
+    const bool colsum = a.colsum != nullptr;
     ring_prefetch(a);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
     const int64_t rows = a.rows, cols = a.cols;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile;
-    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTile;
+    const int local = static_cast<int>(blockIdx.x) - a.tile_begin;
+    const int tile_y = local / a.tiles_x;
+    const int64_t r0 = static_cast<int64_t>(tile_y) * kTile;
+    const int64_t c0 = static_cast<int64_t>(local % a.tiles_x) * kTile;
     const int t = threadIdx.x;
     const int j = t & 15;   // 8-column group of the tile
     const int rr = t >> 4;  // row within each 16-row slab
@@ -277,12 +298,12 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 
             for (int e = 0; e < 8; ++e)
                 f[e] = (gr < rows && gc + e < cols) ? In::cvt(x[gr * cols + gc + e]) : 0.0f;
         }
-        if constexpr (kColsum) {
+        if (colsum) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) cs[e] += f[e];
         }
         const uint2 w = convert8<kFmt>(f, mult, amax);
-        if constexpr (kRowOut) {
+        if (row_out) {
             if (gr < rows) {
                 uint8_t* dst = a.out + gr * cols + gc;
                 if (a.vec_out && gc + 8 <= cols) {
@@ -298,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 
         *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = w;
     }
 
-    if constexpr (kColsum) {
+    if (colsum) {
         // lanes l and l ^ 16 share the column group; then the 8 warps go through shared memory
 #pragma unroll
         for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
@@ -309,12 +330,12 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 
     }
     __syncthreads();
 
-    if constexpr (kColsum) {
+    if (colsum) {
         if (t < kTile && c0 + t < cols) {
             float s = 0.0f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) s += csum[w][t];
-            a.colsum[static_cast<int64_t>(blockIdx.y) * cols + c0 + t] = s;
+            a.colsum[static_cast<int64_t>(tile_y) * cols + c0 + t] = s;
         }
     }
 
@@ -349,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 
                 dst[b] = static_cast<uint8_t>(O[jj][b >> 2] >> (8 * (b & 3)));
         }
     }
-    block_finish(a, amax, step);
+    block_finish(a, amax, step, local == 0);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -388,6 +409,8 @@ __device__ __forceinline__ float amax_range(const void* xv, int64_t numel, int v
 }
 
 __global__ void __launch_bounds__(kThreads) amax_jobs_kernel(AmaxArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int job = blockIdx.y;
     float amax;
     if (a.in_type[job] == FP8_IN_BF16)
@@ -426,6 +449,8 @@ __global__ void __launch_bounds__(kThreads) amax_jobs_kernel(AmaxArgs a) {
 
 __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* partial, int64_t tiles,
                                                                     int64_t cols, uint16_t* out) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (c >= cols) return;
     // in-order sum (deterministic); the loads are independent and issued four at a time
@@ -446,27 +471,11 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
 }
 
 template <int kFmt, class In>
-void launch_quant_kernel(const QArgs& a, bool tiled, bool row_out, bool colsum, cudaStream_t stream) {
-    if (!tiled) {
-        const int64_t groups = (a.numel + 15) / 16;
-        const int64_t want = std::max<int64_t>(1, (groups + kThreads - 1) / kThreads);
-        const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
-        quant_flat_kernel<In, kFmt><<<blocks, kThreads, 0, stream>>>(a);
-        return;
-    }
-    const dim3 grid(static_cast<unsigned>((a.cols + kTile - 1) / kTile),
-                    static_cast<unsigned>((a.rows + kTile - 1) / kTile));
-    if (row_out) {
-        if (colsum)
-            quant_tiled_kernel<In, kFmt, true, true><<<grid, kThreads, 0, stream>>>(a);
-        else
-            quant_tiled_kernel<In, kFmt, true, false><<<grid, kThreads, 0, stream>>>(a);
-    } else {
-        if (colsum)
-            quant_tiled_kernel<In, kFmt, false, true><<<grid, kThreads, 0, stream>>>(a);
-        else
-            quant_tiled_kernel<In, kFmt, false, false><<<grid, kThreads, 0, stream>>>(a);
-    }
+void launch_quant_kernel(const QBatch& b, bool tiled, dim3 grid, cudaStream_t stream) {
+    if (tiled)
+        launch_ex(quant_tiled_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+    else
+        launch_ex(quant_flat_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
 }
 
 int check_ring(const fp8_ring_t* ring) {
@@ -483,58 +492,92 @@ int check_ring(const fp8_ring_t* ring) {
 
 }  // namespace
 
-int launch_quantize(const QuantJob& job, cudaStream_t stream) {
-    QArgs a{};
-    a.x = job.x;
-    a.rows = job.rows;
-    a.cols = job.cols;
-    a.numel = job.rows * job.cols;
-    a.scale = job.scale;
-    a.out = job.out;
-    a.out_t = job.out_t;
-    a.scale_used_out = job.scale_used_out;
-    a.colsum = job.colsum_partial;
-    const bool tiled = job.out_t != nullptr && a.numel > 0;
-    if (job.ring != nullptr) {
-        const int n = job.ring->hist_len;
-        a.ring_state = job.ring->state;
-        a.hist_len = n;
-        a.hist_idx = job.ring->hist_idx;
-        a.fp8_max = job.ring->fp8_max;
-        a.pow2_margin = job.ring->pow2_margin;
-        a.amax_accum = job.ring->state + n + 2;
-        a.amax_out = job.amax_out;
-    } else {
-        a.amax_accum = job.amax_out;
-        if (job.amax_out != nullptr) {
-            cudaError_t e = cudaMemsetAsync(job.amax_out, 0, sizeof(float), stream);
-            if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset amax: ") + cudaGetErrorString(e));
+int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream) {
+    if (njobs < 1 || njobs > kMaxJobs) return fail(FP8DSA_ERR_INVALID_ARG, "quantize batch of 1..3 tensors");
+    const fp8_fmt_t fmt = jobs[0].fmt;
+    const fp8_in_t in_type = jobs[0].in_type;
+    const bool tiled = jobs[0].out_t != nullptr;
+    for (int i = 1; i < njobs; ++i)
+        if (jobs[i].fmt != fmt || jobs[i].in_type != in_type || (jobs[i].out_t != nullptr) != tiled)
+            return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares format, input type and orientation");
+    QBatch b{};
+    b.njobs = njobs;
+    const int eb = in_type_bytes(in_type);
+    double bytes = 0.0;
+    int64_t max_groups = 0;
+    int64_t tiles_total = 0;
+    for (int i = 0; i < njobs; ++i) {
+        const QuantJob& job = jobs[i];
+        QArgs& a = b.job[i];
+        a.x = job.x;
+        a.rows = job.rows;
+        a.cols = job.cols;
+        a.numel = job.rows * job.cols;
+        a.scale = job.scale;
+        a.out = job.out;
+        a.out_t = job.out_t;
+        a.scale_used_out = job.scale_used_out;
+        a.colsum = job.colsum_partial;
+        if (job.ring != nullptr) {
+            const int n = job.ring->hist_len;
+            a.ring_state = job.ring->state;
+            a.hist_len = n;
+            a.hist_idx = job.ring->hist_idx;
+            a.fp8_max = job.ring->fp8_max;
+            a.pow2_margin = job.ring->pow2_margin;
+            a.amax_accum = job.ring->state + n + 2;
+            a.amax_out = job.amax_out;
+        } else {
+            a.amax_accum = job.amax_out;
+            if (job.amax_out != nullptr) {
+                cudaError_t e = cudaMemsetAsync(job.amax_out, 0, sizeof(float), stream);
+                if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset amax: ") + cudaGetErrorString(e));
+            }
+        }
+        const bool rows_vec = (job.cols * eb) % 16 == 0;
+        a.vec_in = aligned16(job.x) && (tiled ? rows_vec : true);
+        a.vec_out = (job.out == nullptr) ||
+                    (tiled ? ((reinterpret_cast<uintptr_t>(job.out) & 7) == 0 && job.cols % 8 == 0) : aligned16(job.out));
+        a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
+        if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
+        bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0));
+        if (tiled) {
+            // an empty tensor still gets one block, whose fold records amax 0
+            const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);
+            const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
+            a.tiles_x = static_cast<int>(tx);
+            a.tile_begin = static_cast<int>(tiles_total);
+            a.nblocks = static_cast<unsigned>(tx * ty);
+            tiles_total += tx * ty;
+        } else {
+            max_groups = std::max(max_groups, (a.numel + 15) / 16);
         }
     }
-    const int eb = in_type_bytes(job.in_type);
-    const bool rows_vec = (job.cols * eb) % 16 == 0;
-    a.vec_in = aligned16(job.x) && (tiled ? rows_vec : true);
-    a.vec_out = (job.out == nullptr) || (tiled ? ((reinterpret_cast<uintptr_t>(job.out) & 7) == 0 && job.cols % 8 == 0)
-                                               : aligned16(job.out));
-    a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
-    if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
-
-    const double bytes = static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0));
-    launch_begin(kKindQuantize, stream);
-    const bool row_out = job.out != nullptr;
-    const bool colsum = job.colsum_partial != nullptr;
-    if (job.fmt == FP8_E4M3) {
-        if (job.in_type == FP8_IN_BF16) launch_quant_kernel<0, Bf16In>(a, tiled, row_out, colsum, stream);
-        else if (job.in_type == FP8_IN_F16) launch_quant_kernel<0, F16In>(a, tiled, row_out, colsum, stream);
-        else launch_quant_kernel<0, F32In>(a, tiled, row_out, colsum, stream);
+    dim3 grid;
+    if (tiled) {
+        if (tiles_total > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many tiles");
+        grid = dim3(static_cast<unsigned>(tiles_total));
     } else {
-        if (job.in_type == FP8_IN_BF16) launch_quant_kernel<1, Bf16In>(a, tiled, row_out, colsum, stream);
-        else if (job.in_type == FP8_IN_F16) launch_quant_kernel<1, F16In>(a, tiled, row_out, colsum, stream);
-        else launch_quant_kernel<1, F32In>(a, tiled, row_out, colsum, stream);
+        const int64_t want = std::max<int64_t>(1, (max_groups + kThreads - 1) / kThreads);
+        const int per_job = static_cast<int>(std::min<int64_t>(want, std::max<int64_t>(1, static_cast<int64_t>(sm_count()) * 8 / njobs)));
+        for (int i = 0; i < njobs; ++i) b.job[i].nblocks = static_cast<unsigned>(per_job);
+        grid = dim3(static_cast<unsigned>(per_job), static_cast<unsigned>(njobs));
+    }
+    launch_begin(kKindQuantize, stream);
+    if (fmt == FP8_E4M3) {
+        if (in_type == FP8_IN_BF16) launch_quant_kernel<0, Bf16In>(b, tiled, grid, stream);
+        else if (in_type == FP8_IN_F16) launch_quant_kernel<0, F16In>(b, tiled, grid, stream);
+        else launch_quant_kernel<0, F32In>(b, tiled, grid, stream);
+    } else {
+        if (in_type == FP8_IN_BF16) launch_quant_kernel<1, Bf16In>(b, tiled, grid, stream);
+        else if (in_type == FP8_IN_F16) launch_quant_kernel<1, F16In>(b, tiled, grid, stream);
+        else launch_quant_kernel<1, F32In>(b, tiled, grid, stream);
     }
     launch_end(kKindQuantize, stream, bytes);
     return check_launch("fp8 quantize kernel");
 }
+
+int launch_quantize(const QuantJob& job, cudaStream_t stream) { return launch_quantize_batch(&job, 1, stream); }
 
 int launch_amax_jobs(const AmaxJob* jobs, int njobs, uint32_t* scratch, cudaStream_t stream) {
     AmaxArgs a{};
@@ -561,7 +604,7 @@ int launch_amax_jobs(const AmaxJob* jobs, int njobs, uint32_t* scratch, cudaStre
     const int64_t want = std::max<int64_t>(1, (max_numel / 16 + kThreads - 1) / kThreads);
     const int per_job = std::max(1, static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8 / njobs)));
     launch_begin(kKindOther, stream);
-    amax_jobs_kernel<<<dim3(per_job, njobs), kThreads, 0, stream>>>(a);
+    launch_ex(amax_jobs_kernel, dim3(per_job, njobs), dim3(kThreads), 0, stream, 1, a);
     launch_end(kKindOther, stream, bytes);
     return check_launch("fp8 amax kernel");
 }
@@ -570,7 +613,8 @@ int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, vo
                            cudaStream_t stream) {
     const unsigned blocks = static_cast<unsigned>((cols + kThreads - 1) / kThreads);
     launch_begin(kKindOther, stream);
-    colsum_finalize_kernel<<<blocks, kThreads, 0, stream>>>(partial, tiles, cols, static_cast<uint16_t*>(out_bf16));
+    launch_ex(colsum_finalize_kernel, dim3(blocks), dim3(kThreads), 0, stream, 1, partial, tiles, cols,
+              static_cast<uint16_t*>(out_bf16));
     launch_end(kKindOther, stream, static_cast<double>(tiles) * cols * 4 + cols * 2);
     return check_launch("colsum finalize kernel");
 }
@@ -647,8 +691,8 @@ static int quantize_common(const void* x, fp8_in_t in_type, int64_t rows, int64_
     if (!empty && out == nullptr && out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "output is NULL");
     if (out_t != nullptr && (cols + kTile - 1) / kTile > 0x7FFFFFFF)
         return fail(FP8DSA_ERR_UNSUPPORTED, "too many columns");
-    if (out_t != nullptr && (rows + kTile - 1) / kTile > 65535)
-        return fail(FP8DSA_ERR_UNSUPPORTED, "transposed quantize supports at most 65535*128 rows");
+    if (out_t != nullptr && ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile) > 0x7FFFFFFF)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
     int rc = check_ring(ring);
     if (rc) return rc;
     rc = check_device();

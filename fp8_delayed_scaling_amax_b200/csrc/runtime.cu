@@ -24,6 +24,7 @@ int g_cc_major[kMaxDevices];      // 0 = not queried yet
 int g_sms[kMaxDevices];
 int* g_status_ptr[kMaxDevices];   // device address of g_status on each device
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<int> g_pdl{1};
 
 // Per-kernel timing.
 struct TimedLaunch {
@@ -51,6 +52,8 @@ cudaEvent_t take_event() {
 
 // The status word bounded waits report into (one per device, one per loaded module).
 __device__ int g_status;
+
+bool pdl_enabled() { return g_pdl.load() != 0; }
 
 int fail(int code, const std::string& msg) {
     t_last_error = msg;
@@ -198,6 +201,11 @@ int fp8_debug_stalled_wait(cudaStream_t stream) {
     if (rc) return rc;
     stalled_wait_kernel<<<1, 32, 0, stream>>>(ctl);
     return check_launch("stalled_wait_kernel");
+}
+
+int fp8_set_pdl(int enabled) {
+    g_pdl.store(enabled != 0 ? 1 : 0);
+    return FP8DSA_OK;
 }
 
 int fp8_profiler_enable(int on) {

@@ -210,6 +210,12 @@ int fp8_get_device_status(cudaStream_t stream, int* status);
  * (default 2e9 = 2 s).  Applies to launches after the call. */
 int fp8_set_wait_timeout_ns(uint64_t ns);
 
+/* Launch the library's kernels with programmatic dependent launch (default 1 = on): each
+ * kernel's launch and set-up overlap the tail of the previous kernel on the stream, and it
+ * waits for that kernel's results before reading them.  0 launches them plainly.  Applies to
+ * launches after the call (and to stream captures made after it).  Not on the pages. */
+int fp8_set_pdl(int enabled);
+
 /* Test hook for the failure path: launches one block that waits on a barrier nothing ever
  * arrives at; the wait gives up after the timeout and sets the device status word.
  * Not on the pages. */
