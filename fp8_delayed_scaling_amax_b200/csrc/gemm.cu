@@ -16,9 +16,14 @@
 //    TMEM accumulator; tcgen05.commit releases each stage and, per tile, hands the
 //    accumulator to the epilogue.  Two accumulators (2 x BN TMEM columns) let the epilogue
 //    of tile i overlap the MMAs of tile i + 1;
-//  * warps 2-5 = epilogue: tcgen05.ld 64 columns at a time, fma with the combined scale and
-//    the bias, round to bf16, stage each warp's 32 x 64 box in 128-byte-swizzled shared
-//    memory and write it with a TMA bulk-tensor store (double-buffered per warp);
+//  * warps 2.. = epilogue (8 warps where shared memory allows, two per TMEM lane quarter, else
+//    4): tcgen05.ld 64 columns at a time, fma with the combined scale and the bias, round to
+//    bf16, stage each warp's 32 x 64 box in 128-byte-swizzled shared memory and write it with
+//    a TMA bulk-tensor store (double-buffered per warp);
+//  * CTA pairs: 256 x 256 tiles with one tcgen05.mma.cta_group::2 (M = 256) spanning both SMs,
+//    each SM holding 128 rows of A and half of B; pair loads complete on the leader's barriers;
+//  * one launch may carry two GEMMs over one tile space (the backward's dX and dW), and its
+//    epilogue warps can first reduce the bias-gradient column sums (a side job, no launch).
 //  * every wait is bounded (globaltimer); on expiry the CTA records a status code, drains its
 //    in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -38,31 +43,40 @@ namespace {
 constexpr int kBM = 128;      // tile rows (TMEM lanes)
 constexpr int kBK = 128;      // K bytes per stage (one 128-byte swizzle row)
 constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
-constexpr int kThreads = 192; // 6 warps
-constexpr int kEpiThreads = 128;
 
 constexpr int kOutBox = 64;                       // output columns per TMA store (128 bytes of bf16)
 constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 columns
+constexpr int kSmemLimit = 232448;                // dynamic shared memory per CTA on sm_100
+constexpr int kMaxProblems = 2;
 
 // kPair: a 2-CTA cluster computes a 256 x BN tile with one M = 256 MMA across both SMs; each CTA
 // holds 128 rows of A and BN/2 rows of B, so each SM's shared memory feeds half the B operand.
+// Epilogue warps: 8 (two per TMEM lane quarter, each owning half the columns) when the stages
+// leave room for their staging buffers, else 4.
 template <int BN, bool kPair>
 struct Cfg {
     static constexpr int kTileM = kPair ? 2 * kBM : kBM;
     static constexpr int kBRows = kPair ? BN / 2 : BN;  // rows of B (along N) this CTA loads
     static constexpr int kAStage = kBM * kBK;
     static constexpr int kBStage = kBRows * kBK;
-    static constexpr int kStages = (kAStage + kBStage) <= 32768 ? 6 : 4;
-    static constexpr int kTmemCols = 2 * BN;
-    static constexpr int kOutBytes = 4 * 2 * kOutStageBytes;  // 4 epilogue warps x 2 buffers
+    static constexpr int kEpiWarps = (kAStage + kBStage) <= 32768 ? 8 : 4;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kEpiThreads = 32 * kEpiWarps;
+    static constexpr int kEpiCols = BN / (kEpiWarps / 4);  // columns of the tile each epilogue warp owns
+    static constexpr int kOutBytes = kEpiWarps * 2 * kOutStageBytes;
     static constexpr int kBarBytes = 256;
-    static constexpr int kSmem = 1024 + kStages * (kAStage + kBStage) + kOutBytes + kBarBytes;
+    static constexpr int kFixed = 1024 + kOutBytes + kBarBytes;
+    static constexpr int kStagesFit = (kSmemLimit - kFixed) / (kAStage + kBStage);
+    static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
+    static constexpr int kSmem = kFixed + kStages * (kAStage + kBStage);
     static constexpr uint32_t kTxBytes = (kPair ? 2u : 1u) * (kAStage + kBStage);
+    static_assert(kStages >= 3, "too few pipeline stages");
 };
 
-struct GemmArgs {
-    int m, n, k;
-    int tiles_m, tiles_n, num_tiles, k_blocks;
+// One GEMM of a launch (a launch may carry two, e.g. dX and dW, over one tile space).
+struct GemmProblem {
+    int m, n, k_blocks;
+    int tiles_m, tiles_n, tile_begin;
     int a_batched, b_batched;
     int a_mn, b_mn;
     uint32_t idesc;
@@ -75,6 +89,21 @@ struct GemmArgs {
     const float* bias_scale;
     const float* scale_a;
     const float* scale_b;
+};
+
+// Optional side job of the epilogue warps, done before their first tile: the bias gradient
+// out[c] = RN_bf16(sum_t partial[t][c]), summed in order t = 0, 1, ...
+struct ColsumJob {
+    const float* partial;
+    int tiles, cols;
+    uint16_t* out;
+};
+
+struct GemmArgs {
+    GemmProblem p[kMaxProblems];
+    int nprob;
+    int num_tiles;
+    ColsumJob colsum;
     WaitCtl wait;
 };
 
@@ -89,15 +118,19 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-__device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& b, int& tm, int& tn) {
+// Tile -> (problem, batch, tile row, tile column); grouped raster of 8 tile rows per problem.
+__device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& pi, int& b, int& tm, int& tn) {
     constexpr int kGroupM = 8;
-    const int per = g.tiles_m * g.tiles_n;
-    b = tile / per;
-    const int r = tile - b * per;
-    const int group = kGroupM * g.tiles_n;
+    pi = (g.nprob > 1 && tile >= g.p[1].tile_begin) ? 1 : 0;
+    const GemmProblem& P = g.p[pi];
+    const int t = tile - P.tile_begin;
+    const int per = P.tiles_m * P.tiles_n;
+    b = t / per;
+    const int r = t - b * per;
+    const int group = kGroupM * P.tiles_n;
     const int gi = r / group;
     const int first_m = gi * kGroupM;
-    const int gm = min(g.tiles_m - first_m, kGroupM);
+    const int gm = min(P.tiles_m - first_m, kGroupM);
     const int within = r - gi * group;
     tm = first_m + within % gm;
     tn = within / gm;
@@ -108,17 +141,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float bias_value(const GemmArgs& g, int col, float bsc) {
-    if (col >= g.n || g.bias_kind == 0) return 0.0f;
-    if (g.bias_kind == 1) return bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(g.bias) + col));
-    const uint8_t v = __ldg(static_cast<const uint8_t*>(g.bias) + col);
-    return __fmul_rn(g.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
+__device__ __forceinline__ float bias_value(const GemmProblem& P, int col, float bsc) {
+    if (col >= P.n || P.bias_kind == 0) return 0.0f;
+    if (P.bias_kind == 1) return bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(P.bias) + col));
+    const uint8_t v = __ldg(static_cast<const uint8_t*>(P.bias) + col);
+    return __fmul_rn(P.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
 }
 
 template <int BN, bool kPair>
-__global__ void __launch_bounds__(kThreads, 1)
-    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                    const __grid_constant__ CUtensorMap tma_o, const GemmArgs g) {
+__global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a0, const __grid_constant__ CUtensorMap tma_b0,
+                    const __grid_constant__ CUtensorMap tma_o0, const __grid_constant__ CUtensorMap tma_a1,
+                    const __grid_constant__ CUtensorMap tma_b1, const __grid_constant__ CUtensorMap tma_o1,
+                    const __grid_constant__ GemmArgs g) {
     using C = Cfg<BN, kPair>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -134,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+    pdl_trigger();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    pdl_trigger();
     const uint32_t rank = kPair ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
     const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
@@ -150,23 +185,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full + a, 1);
             // the leader's accumulator is released by both CTAs' epilogue threads
-            mbar_init(acc_empty + a, kEpiThreads * (kPair ? 2 : 1));
+            mbar_init(acc_empty + a, C::kEpiThreads * (kPair ? 2 : 1));
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tma_a);
-        prefetch_tensormap(&tma_b);
-        if (g.tma_out) prefetch_tensormap(&tma_o);
+        prefetch_tensormap(&tma_a0);
+        prefetch_tensormap(&tma_b0);
+        if (g.p[0].tma_out) prefetch_tensormap(&tma_o0);
+        if (g.nprob > 1) {
+            prefetch_tensormap(&tma_a1);
+            prefetch_tensormap(&tma_b1);
+            if (g.p[1].tma_out) prefetch_tensormap(&tma_o1);
+        }
     }
     if (warp == 1) {
         if constexpr (kPair) {
-            tmem_alloc_pair(tmem_slot, C::kTmemCols);
+            tmem_alloc_pair(tmem_slot, 2 * BN);
             tmem_relinquish_pair();
         } else {
-            tmem_alloc(tmem_slot, C::kTmemCols);
+            tmem_alloc(tmem_slot, 2 * BN);
             tmem_relinquish();
         }
     }
@@ -185,13 +225,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t issued = 0, issued_parity = 0;  // per-stage: ever issued, parity of the last issue
             bool ok = true;
             for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
-                int b, tm, tn;
-                decode_tile(tile, g, b, tm, tn);
-                const int ba = g.a_batched ? b : 0;
-                const int bb = g.b_batched ? b : 0;
+                int pi, b, tm, tn;
+                decode_tile(tile, g, pi, b, tm, tn);
+                const GemmProblem& P = g.p[pi];
+                const CUtensorMap* ta = pi ? &tma_a1 : &tma_a0;
+                const CUtensorMap* tb = pi ? &tma_b1 : &tma_b0;
+                const int ba = P.a_batched ? b : 0;
+                const int bb = P.b_batched ? b : 0;
                 const int arow = tm * C::kTileM + static_cast<int>(rank) * kBM;
                 const int brow = tn * BN + static_cast<int>(rank) * C::kBRows;
-                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                for (int kb = 0; kb < P.k_blocks; ++kb) {
                     if (!mbar_wait_bounded(empty + stage, phase ^ 1u, g.wait, abort_flag, kStatusWaitProducer)) {
                         ok = false;
                         break;
@@ -201,28 +244,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* b_dst = sB + stage * C::kBStage;
                     if constexpr (kPair) {
                         const uint32_t fb = mapa_shared(smem_addr(full + stage), 0);
-                        if (!g.a_mn)
-                            tma_load_3d_pair(a_dst, &tma_a, fb, kb * kBK, arow, ba);
+                        if (!P.a_mn)
+                            tma_load_3d_pair(a_dst, ta, fb, kb * kBK, arow, ba);
                         else
-                            tma_load_3d_pair(a_dst, &tma_a, fb, arow, kb * kBK, ba);
-                        if (!g.b_mn) {
-                            tma_load_3d_pair(b_dst, &tma_b, fb, kb * kBK, brow, bb);
+                            tma_load_3d_pair(a_dst, ta, fb, arow, kb * kBK, ba);
+                        if (!P.b_mn) {
+                            tma_load_3d_pair(b_dst, tb, fb, kb * kBK, brow, bb);
                         } else {
 #pragma unroll
                             for (int h = 0; h < C::kBRows / 128; ++h)
-                                tma_load_3d_pair(b_dst + h * 128 * kBK, &tma_b, fb, brow + h * 128, kb * kBK, bb);
+                                tma_load_3d_pair(b_dst + h * 128 * kBK, tb, fb, brow + h * 128, kb * kBK, bb);
                         }
                     } else {
-                        if (!g.a_mn)
-                            tma_load_3d(a_dst, &tma_a, full + stage, kb * kBK, arow, ba);
+                        if (!P.a_mn)
+                            tma_load_3d(a_dst, ta, full + stage, kb * kBK, arow, ba);
                         else
-                            tma_load_3d(a_dst, &tma_a, full + stage, arow, kb * kBK, ba);
-                        if (!g.b_mn) {
-                            tma_load_3d(b_dst, &tma_b, full + stage, kb * kBK, brow, bb);
+                            tma_load_3d(a_dst, ta, full + stage, arow, kb * kBK, ba);
+                        if (!P.b_mn) {
+                            tma_load_3d(b_dst, tb, full + stage, kb * kBK, brow, bb);
                         } else {
 #pragma unroll
                             for (int h = 0; h < C::kBRows / 128; ++h)
-                                tma_load_3d(b_dst + h * 128 * kBK, &tma_b, full + stage, brow + h * 128, kb * kBK, bb);
+                                tma_load_3d(b_dst + h * 128 * kBK, tb, full + stage, brow + h * 128, kb * kBK, bb);
                         }
                     }
                     issued |= 1u << stage;
@@ -250,6 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
             for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
+                int pi, b, tm, tn;
+                decode_tile(tile, g, pi, b, tm, tn);
+                const GemmProblem& P = g.p[pi];
                 const bool got = kPair ? mbar_wait_bounded_cluster(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
                                                                    kStatusWaitMma)
                                        : mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
@@ -260,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                for (int kb = 0; kb < P.k_blocks; ++kb) {
                     if (!mbar_wait_bounded(full + stage, phase, g.wait, abort_flag, kStatusWaitMma)) {
                         ok = false;
                         break;
@@ -272,14 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                             // K-major: step 32 bytes along the swizzled row; MN-major: step 32 rows.
-                            const uint64_t ad = g.a_mn ? smem_desc(a_base + kk * kUmmaK * 128, C::kAStage, 1024)
+                            const uint64_t ad = P.a_mn ? smem_desc(a_base + kk * kUmmaK * 128, C::kAStage, 1024)
                                                        : smem_desc(a_base + kk * kUmmaK, 16, 1024);
-                            const uint64_t bd = g.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
+                            const uint64_t bd = P.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
                                                        : smem_desc(b_base + kk * kUmmaK, 16, 1024);
                             if constexpr (kPair)
-                                umma_f8f6f4_pair(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                                umma_f8f6f4_pair(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
                             else
-                                umma_f8f6f4(d_tmem, ad, bd, g.idesc, (kb | kk) != 0 ? 1u : 0u);
+                                umma_f8f6f4(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
                         }
                         if constexpr (kPair)
                             umma_commit_pair_multicast(empty + stage, 0x3);
@@ -318,33 +364,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------------ epilogue
         // Warp w may read TMEM lanes 32*(w%4) .. +31, i.e. rows 32*(w%4) + lane of this CTA's
-        // 128-row half of the tile.  Per 64 output columns: two 32-column TMEM loads,
-        // acc * scale + bias in fp32, one bf16 rounding, then either a swizzled shared-memory
-        // stage + TMA bulk store of the warp's 32 x 64 box (double-buffered), or direct
-        // 128-bit stores.
+        // 128-row half of the tile; with 8 epilogue warps, warps w and w+4 split the columns.
+        // Per 64 output columns: two 32-column TMEM loads, acc * scale + bias in fp32, one
+        // bf16 rounding, then either a swizzled shared-memory stage + TMA bulk store of the
+        // warp's 32 x 64 box (double-buffered), or direct 128-bit stores.
+        const int ew = warp - 2;
         const int q = warp & 3;
-        uint8_t* my_stage = sOut + (warp - 2) * 2 * kOutStageBytes;
-        const float sc = __fmul_rn(__ldg(g.scale_a), __ldg(g.scale_b));
-        const float bsc = g.bias_kind >= 2 ? __ldg(g.bias_scale) : 0.0f;
+        const int cbase = (ew >> 2) * C::kEpiCols;
+        uint8_t* my_stage = sOut + ew * 2 * kOutStageBytes;
+
+        // side job: the bias gradient from the per-tile column sums (before the first tile)
+        if (g.colsum.tiles > 0) {
+            const int et = ew * 32 + lane;
+            const int per_cta = C::kEpiThreads;
+            for (int c = static_cast<int>(blockIdx.x) * per_cta + et; c < g.colsum.cols;
+                 c += static_cast<int>(gridDim.x) * per_cta) {
+                const float* col = g.colsum.partial + c;
+                float sum = 0.0f;
+                int t = 0;
+                for (; t + 4 <= g.colsum.tiles; t += 4) {
+                    const float v0 = __ldcg(col + static_cast<int64_t>(t) * g.colsum.cols);
+                    const float v1 = __ldcg(col + static_cast<int64_t>(t + 1) * g.colsum.cols);
+                    const float v2 = __ldcg(col + static_cast<int64_t>(t + 2) * g.colsum.cols);
+                    const float v3 = __ldcg(col + static_cast<int64_t>(t + 3) * g.colsum.cols);
+                    sum += v0;
+                    sum += v1;
+                    sum += v2;
+                    sum += v3;
+                }
+                for (; t < g.colsum.tiles; ++t) sum += __ldcg(col + static_cast<int64_t>(t) * g.colsum.cols);
+                g.colsum.out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+            }
+        }
+
+        float sc[kMaxProblems], bsc[kMaxProblems];
+#pragma unroll
+        for (int i = 0; i < kMaxProblems; ++i) {
+            sc[i] = 0.0f;
+            bsc[i] = 0.0f;
+            if (i < g.nprob) {
+                sc[i] = __fmul_rn(__ldg(g.p[i].scale_a), __ldg(g.p[i].scale_b));
+                bsc[i] = g.p[i].bias_kind >= 2 ? __ldg(g.p[i].bias_scale) : 0.0f;
+            }
+        }
         const uint32_t acc_empty_leader0 = kPair ? mapa_shared(smem_addr(acc_empty), 0) : 0u;
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         for (int tile = unit; tile < g.num_tiles; tile += units) {
-            int b, tm, tn;
-            decode_tile(tile, g, b, tm, tn);
-            const int col0 = tn * BN;
+            int pi, b, tm, tn;
+            decode_tile(tile, g, pi, b, tm, tn);
+            const GemmProblem& P = g.p[pi];
+            const CUtensorMap* to = pi ? &tma_o1 : &tma_o0;
+            const float scale = pi ? sc[1] : sc[0];
+            const int col0 = tn * BN + cbase;
             const int row0 = tm * C::kTileM + static_cast<int>(rank) * kBM + q * 32;
             const int64_t row = static_cast<int64_t>(row0) + lane;
-            // this tile's bias, column col0 + 32 j + lane in bias_r[j], loaded before the wait
-            float bias_r[BN / 32];
+            // this warp's bias columns col0 + 32 j + lane in bias_r[j], loaded before the wait
+            float bias_r[C::kEpiCols / 32];
 #pragma unroll
-            for (int j = 0; j < BN / 32; ++j) bias_r[j] = bias_value(g, col0 + 32 * j + lane, bsc);
+            for (int j = 0; j < C::kEpiCols / 32; ++j) bias_r[j] = bias_value(P, col0 + 32 * j + lane, pi ? bsc[1] : bsc[0]);
             if (!mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue)) break;
             tc_fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < BN; c += kOutBox) {
+            for (int c = 0; c < C::kEpiCols; c += kOutBox) {
                 uint32_t r0[32], r1[32];
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c);
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                       static_cast<uint32_t>(acc * BN + cbase + c);
                 tmem_load_32cols(taddr, r0);
                 tmem_load_32cols(taddr + 32, r1);
                 const float b_lo = bias_r[c / 32];
@@ -353,18 +438,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t packed[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float v0 = fmaf(__uint_as_float(r0[2 * e]), sc, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e));
-                    const float v1 = fmaf(__uint_as_float(r0[2 * e + 1]), sc, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e + 1));
+                    const float v0 = fmaf(__uint_as_float(r0[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e));
+                    const float v1 = fmaf(__uint_as_float(r0[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e + 1));
                     packed[e] = pack_bf16x2(v0, v1);
                 }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float v0 = fmaf(__uint_as_float(r1[2 * e]), sc, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e));
-                    const float v1 = fmaf(__uint_as_float(r1[2 * e + 1]), sc, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e + 1));
+                    const float v0 = fmaf(__uint_as_float(r1[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e));
+                    const float v1 = fmaf(__uint_as_float(r1[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e + 1));
                     packed[16 + e] = pack_bf16x2(v0, v1);
                 }
                 const int colg = col0 + c;
-                if (g.tma_out) {
+                if (P.tma_out) {
                     uint8_t* sb = my_stage + buf * kOutStageBytes;
                     if (lane == 0) bulk_wait_group_read<1>();  // the store that last used this buffer has read it
                     __syncwarp();
@@ -375,14 +460,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0 && row0 < g.m && colg < g.n) {
-                        tma_store_3d(&tma_o, sb, colg, row0, b);
+                    if (lane == 0 && row0 < P.m && colg < P.n) {
+                        tma_store_3d(to, sb, colg, row0, b);
                         bulk_commit_group();
                     }
                     buf ^= 1;
-                } else if (row < g.m && colg < g.n) {
-                    uint16_t* orow = g.out + static_cast<int64_t>(b) * g.stride_o + row * g.ldo;
-                    if (g.vec_out && colg + kOutBox <= g.n) {
+                } else if (row < P.m && colg < P.n) {
+                    uint16_t* orow = P.out + static_cast<int64_t>(b) * P.stride_o + row * P.ldo;
+                    if (P.vec_out && colg + kOutBox <= P.n) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + colg);
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
@@ -390,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
 #pragma unroll
                         for (int e = 0; e < kOutBox; ++e)
-                            if (colg + e < g.n) orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
+                            if (colg + e < P.n) orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
                     }
                 }
             }
@@ -408,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_phase ^= 1u;
             }
         }
-        if (g.tma_out && lane == 0) bulk_wait_group_all();
+        if (lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
 
@@ -418,9 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     if (warp == 1) {
         if constexpr (kPair)
-            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+            tmem_dealloc_pair(tmem_base, 2 * BN);
         else
-            tmem_dealloc(tmem_base, C::kTmemCols);
+            tmem_dealloc(tmem_base, 2 * BN);
     }
 }
 
@@ -478,8 +563,7 @@ int make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int6
 }
 
 template <int BN, bool kPair>
-int launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, GemmArgs& g, int64_t batch,
-               cudaStream_t stream) {
+int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, cudaStream_t stream) {
     using C = Cfg<BN, kPair>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -496,7 +580,7 @@ int launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& 
             at[0].val.clusterDim.y = 1;
             at[0].val.clusterDim.z = 1;
             cfg.gridDim = dim3(2 * 74, 1, 1);
-            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.blockDim = dim3(C::kThreads, 1, 1);
             cfg.dynamicSmemBytes = C::kSmem;
             cfg.attrs = at;
             cfg.numAttrs = 1;
@@ -508,116 +592,166 @@ int launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& 
     });
     if (attr_err != cudaSuccess)
         return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(attr_err));
-    g.tiles_m = static_cast<int>((g.m + C::kTileM - 1) / C::kTileM);
-    g.tiles_n = (g.n + BN - 1) / BN;
-    g.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
-    const int64_t tiles = static_cast<int64_t>(g.tiles_m) * g.tiles_n * batch;
-    if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
+    int64_t tiles = 0;
+    for (int i = 0; i < g.nprob; ++i) {
+        GemmProblem& P = g.p[i];
+        P.tiles_m = (P.m + C::kTileM - 1) / C::kTileM;
+        P.tiles_n = (P.n + BN - 1) / BN;
+        P.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
+        P.tile_begin = static_cast<int>(tiles);
+        tiles += static_cast<int64_t>(P.tiles_m) * P.tiles_n * batch[i];
+        if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
+    }
     g.num_tiles = static_cast<int>(tiles);
     const int units = kPair ? (max_units > 0 ? max_units : sm_count() / 2) : sm_count();
-    const int grid_units = static_cast<int>(std::min<int64_t>(tiles, units));
+    const int grid_units = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, units)));
     cudaError_t e = launch_ex(fp8_gemm_kernel<BN, kPair>, dim3(static_cast<unsigned>(grid_units * (kPair ? 2 : 1))),
-                              dim3(kThreads), C::kSmem, stream, kPair ? 2 : 1, ma, mb, mo, g);
+                              dim3(C::kThreads), C::kSmem, stream, kPair ? 2 : 1, maps[0], maps[1], maps[2], maps[3],
+                              maps[4], maps[5], g);
     if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("fp8 gemm launch: ") + cudaGetErrorString(e));
     return FP8DSA_OK;
 }
 
-// Tile shape: 256 x 256 tiles on CTA pairs when M > 128 (each SM then reads half of the B
-// operand from its shared memory); 128 x 256 on one CTA otherwise; 128-wide tiles only when N
-// is at most 128.  A 128 x 128 x 32 MMA reads as many operand bytes from shared memory per flop
-// as the TMA writes into it, and measured far slower than the 256-wide tile.
-int choose_bn(int64_t m, int64_t n, int64_t batch) {
-    (void)m;
-    (void)batch;
-    return n <= 128 ? 128 : 256;
-}
+// Tile shape for a launch: 256 x 256 tiles on CTA pairs when every problem has M > 128 and
+// N > 128 (each SM then reads half of the B operand from its shared memory); otherwise one
+// CTA per tile, 128 x 256, or 128 x 128 when some problem is at most 128 wide.  A 128 x 128
+// MMA reads as many operand bytes from shared memory per flop as the TMA writes into it and
+// measured far slower than the 256-wide tile.
+struct TileChoice {
+    int bn;
+    bool pair;
+};
 
-bool choose_pair(int64_t m, int64_t n, int b_mn) {
-    if (m <= kBM) return false;
-    if (n <= 128) return false;  // pair tiles keep 256 columns (128 per CTA: one MN-major swizzle block)
-    (void)b_mn;
-    return true;
+TileChoice choose_tiles(const GemmDesc* d, int n) {
+    bool narrow = false, short_m = false;
+    for (int i = 0; i < n; ++i) {
+        narrow = narrow || d[i].n <= 128;
+        short_m = short_m || d[i].m <= kBM;
+    }
+    if (narrow) return {128, false};
+    return {256, !short_m};
 }
 
 }  // namespace
+
+int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
+                      int64_t colsum_cols, void* colsum_out, cudaStream_t stream) {
+    // problems with an empty product write their bias (or zeros) without the tensor cores
+    GemmDesc work[kMaxProblems];
+    int nwork = 0;
+    double flops = 0.0;
+    for (int i = 0; i < ndesc; ++i) {
+        const GemmDesc& d = descs[i];
+        if (d.m == 0 || d.n == 0 || d.batch == 0) continue;
+        if (d.k == 0) {
+            const int64_t total = d.batch * d.m * d.n;
+            const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 8));
+            launch_begin(kKindOther, stream);
+            launch_ex(bias_fill_kernel, dim3(blocks), dim3(256), 0, stream, 1, static_cast<uint16_t*>(d.out), d.m, d.n,
+                      d.ldo, d.stride_o, d.batch, d.bias, d.bias_kind, d.bias_scale);
+            launch_end(kKindOther, stream, static_cast<double>(total) * 2);
+            int rc = check_launch("bias fill kernel");
+            if (rc) return rc;
+            continue;
+        }
+        work[nwork++] = d;
+        flops += 2.0 * static_cast<double>(d.m) * d.n * d.k * d.batch;
+    }
+    const bool colsum = colsum_tiles > 0 && colsum_cols > 0;
+    if (nwork == 0) {
+        if (colsum) return launch_colsum_finalize(colsum_partial, colsum_tiles, colsum_cols, colsum_out, stream);
+        if (colsum_cols > 0 && colsum_out != nullptr) {  // no rows: the bias gradient is zero
+            cudaError_t e = cudaMemsetAsync(colsum_out, 0, sizeof(uint16_t) * colsum_cols, stream);
+            if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset grad_b: ") + cudaGetErrorString(e));
+        }
+        return FP8DSA_OK;
+    }
+    if (colsum_cols > 0x7FFFFFFF || colsum_tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "bias gradient too wide");
+    const TileChoice tc = choose_tiles(work, nwork);
+    const int b_rows = tc.pair ? tc.bn / 2 : tc.bn;  // rows of B each CTA loads
+
+    CUtensorMap maps[6];
+    GemmArgs g{};
+    int64_t batch[kMaxProblems] = {1, 1};
+    const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    for (int i = 0; i < nwork; ++i) {
+        const GemmDesc& d = work[i];
+        const bool a_bat = d.stride_a != 0 && d.batch > 1;
+        const bool b_bat = d.stride_b != 0 && d.batch > 1;
+        CUtensorMap& ma = maps[3 * i];
+        CUtensorMap& mb = maps[3 * i + 1];
+        CUtensorMap& mo = maps[3 * i + 2];
+        int rc;
+        if (!d.a_mn)
+            rc = make_map(&ma, u8, d.a, d.k, d.m, a_bat ? d.batch : 1, d.lda, a_bat ? d.stride_a : d.lda * d.m, 128, kBM);
+        else
+            rc = make_map(&ma, u8, d.a, d.m, d.k, a_bat ? d.batch : 1, d.lda, a_bat ? d.stride_a : d.lda * d.k, 128, kBK);
+        if (rc) return rc;
+        if (!d.b_mn)
+            rc = make_map(&mb, u8, d.b, d.k, d.n, b_bat ? d.batch : 1, d.ldb, b_bat ? d.stride_b : d.ldb * d.n, 128,
+                          b_rows);
+        else
+            rc = make_map(&mb, u8, d.b, d.n, d.k, b_bat ? d.batch : 1, d.ldb, b_bat ? d.stride_b : d.ldb * d.k, 128, kBK);
+        if (rc) return rc;
+        // TMA stores need 16-byte aligned rows and batches of the output
+        const bool tma_out = aligned16(d.out) && d.ldo % 8 == 0 && (d.batch == 1 || d.stride_o % 8 == 0);
+        if (tma_out) {
+            rc = make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.out, d.n, d.m, d.batch, d.ldo * 2,
+                          d.batch > 1 ? d.stride_o * 2 : d.ldo * 2 * d.m, kOutBox, 32);
+            if (rc) return rc;
+        } else {
+            mo = ma;  // unused placeholder
+        }
+        GemmProblem& P = g.p[i];
+        P.m = static_cast<int>(d.m);
+        P.n = static_cast<int>(d.n);
+        P.k_blocks = static_cast<int>((d.k + kBK - 1) / kBK);
+        P.a_batched = a_bat;
+        P.b_batched = b_bat;
+        P.a_mn = d.a_mn;
+        P.b_mn = d.b_mn;
+        P.idesc = (1u << 4) | (static_cast<uint32_t>(d.fmt_a) << 7) | (static_cast<uint32_t>(d.fmt_b) << 10) |
+                  (static_cast<uint32_t>(d.a_mn) << 15) | (static_cast<uint32_t>(d.b_mn) << 16);
+        P.out = static_cast<uint16_t*>(d.out);
+        P.ldo = d.ldo;
+        P.stride_o = d.stride_o;
+        P.vec_out = aligned16(d.out) && d.ldo % 8 == 0 && d.stride_o % 8 == 0;
+        P.tma_out = tma_out;
+        P.bias = d.bias;
+        P.bias_kind = d.bias_kind;
+        P.bias_scale = d.bias_scale;
+        P.scale_a = d.scale_a;
+        P.scale_b = d.scale_b;
+        batch[i] = d.batch;
+    }
+    for (int i = nwork; i < kMaxProblems; ++i) maps[3 * i] = maps[3 * i + 1] = maps[3 * i + 2] = maps[0];
+    g.nprob = nwork;
+    if (colsum) {
+        g.colsum.partial = colsum_partial;
+        g.colsum.tiles = static_cast<int>(colsum_tiles);
+        g.colsum.cols = static_cast<int>(colsum_cols);
+        g.colsum.out = static_cast<uint16_t*>(colsum_out);
+    }
+    int rc = wait_ctl(&g.wait);
+    if (rc) return rc;
+
+    launch_begin(kKindGemm, stream);
+    if (tc.pair)
+        rc = launch_cfg<256, true>(maps, g, batch, stream);
+    else
+        rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, stream) : launch_cfg<128, false>(maps, g, batch, stream);
+    if (rc) return rc;
+    launch_end(kKindGemm, stream, flops);
+    return check_launch("fp8 gemm kernel");
+}
 
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn, int b_mn, int64_t m,
                 int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch, int64_t stride_a,
                 int64_t stride_b, int64_t stride_o, const float* scale_a, const float* scale_b, const void* bias,
                 int bias_kind, const float* bias_scale, void* out, cudaStream_t stream) {
-    if (m == 0 || n == 0 || batch == 0) return FP8DSA_OK;
-    const double flops = 2.0 * static_cast<double>(m) * n * k * batch;
-    if (k == 0) {
-        const int64_t total = batch * m * n;
-        const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 8));
-        launch_begin(kKindOther, stream);
-        launch_ex(bias_fill_kernel, dim3(blocks), dim3(256), 0, stream, 1, static_cast<uint16_t*>(out), m, n, ldo,
-                  stride_o, batch, bias, bias_kind, bias_scale);
-        launch_end(kKindOther, stream, static_cast<double>(total) * 2);
-        return check_launch("bias fill kernel");
-    }
-    const bool a_bat = stride_a != 0 && batch > 1;
-    const bool b_bat = stride_b != 0 && batch > 1;
-    const int bn = choose_bn(m, n, batch);
-    const bool pair = bn == 256 && choose_pair(m, n, b_mn);
-    const int b_rows = pair ? bn / 2 : bn;  // rows of B each CTA loads
-
-    CUtensorMap ma, mb, mo;
-    int rc;
-    const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    if (!a_mn)
-        rc = make_map(&ma, u8, a, k, m, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * m, 128, kBM);
-    else
-        rc = make_map(&ma, u8, a, m, k, a_bat ? batch : 1, lda, a_bat ? stride_a : lda * k, 128, kBK);
-    if (rc) return rc;
-    if (!b_mn)
-        rc = make_map(&mb, u8, b, k, n, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * n, 128, b_rows);
-    else
-        rc = make_map(&mb, u8, b, n, k, b_bat ? batch : 1, ldb, b_bat ? stride_b : ldb * k, 128, kBK);
-    if (rc) return rc;
-    // TMA stores need 16-byte aligned rows and batches of the output
-    const bool tma_out = aligned16(out) && ldo % 8 == 0 && (batch == 1 || stride_o % 8 == 0);
-    if (tma_out) {
-        rc = make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, n, m, batch, ldo * 2,
-                      batch > 1 ? stride_o * 2 : ldo * 2 * m, kOutBox, 32);
-        if (rc) return rc;
-    } else {
-        mo = ma;  // unused placeholder
-    }
-
-    GemmArgs g{};
-    g.m = static_cast<int>(m);
-    g.n = static_cast<int>(n);
-    g.k = static_cast<int>(k);
-    g.k_blocks = static_cast<int>((k + kBK - 1) / kBK);
-    g.a_batched = a_bat;
-    g.b_batched = b_bat;
-    g.a_mn = a_mn;
-    g.b_mn = b_mn;
-    g.idesc = (1u << 4) | (static_cast<uint32_t>(fmt_a) << 7) | (static_cast<uint32_t>(fmt_b) << 10) |
-              (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
-    g.out = static_cast<uint16_t*>(out);
-    g.ldo = ldo;
-    g.stride_o = stride_o;
-    g.vec_out = aligned16(out) && ldo % 8 == 0 && stride_o % 8 == 0;
-    g.tma_out = tma_out;
-    g.bias = bias;
-    g.bias_kind = bias_kind;
-    g.bias_scale = bias_scale;
-    g.scale_a = scale_a;
-    g.scale_b = scale_b;
-    rc = wait_ctl(&g.wait);
-    if (rc) return rc;
-
-    launch_begin(kKindGemm, stream);
-    if (pair)
-        rc = launch_cfg<256, true>(ma, mb, mo, g, batch, stream);
-    else
-        rc = bn == 256 ? launch_cfg<256, false>(ma, mb, mo, g, batch, stream)
-                       : launch_cfg<128, false>(ma, mb, mo, g, batch, stream);
-    if (rc) return rc;
-    launch_end(kKindGemm, stream, flops);
-    return check_launch("fp8 gemm kernel");
+    GemmDesc d{a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
+               scale_a, scale_b, bias, bias_kind, bias_scale, out};
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, stream);
 }
 
 }  // namespace fp8dsa

@@ -124,6 +124,25 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream);
 int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,
                            cudaStream_t stream);
 
+// One GEMM of a launch, arguments already validated.
+struct GemmDesc {
+    const uint8_t* a;
+    const uint8_t* b;
+    int fmt_a, fmt_b, a_mn, b_mn;
+    int64_t m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o;
+    const float* scale_a;
+    const float* scale_b;
+    const void* bias;
+    int bias_kind;
+    const float* bias_scale;
+    void* out;
+};
+
+// One or two GEMMs in one persistent launch over the union of their tiles; if colsum_tiles > 0
+// the epilogue warps first write colsum_out[c] = RN_bf16(sum_t colsum_partial[t][c]).
+int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
+                      int64_t colsum_cols, void* colsum_out, cudaStream_t stream);
+
 // The GEMM entry with arguments already validated (used by the linear compositions).
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn_major,
                 int b_mn_major, int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb,

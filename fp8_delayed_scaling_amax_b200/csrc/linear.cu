@@ -10,7 +10,8 @@
 // Launches per call (delayed scaling):
 //   forward : one quantize launch for x and w (each folds its own ring) + GEMM           = 2
 //   backward: one quantize launch for g (both orientations, ring fold, per-tile column
-//             sums), x^T and w^T + GEMM dX + GEMM dW + column-sum finalize            = 4
+//             sums), x^T and w^T + one GEMM launch for dX and dW whose epilogue warps
+//             also reduce the column sums into grad_b                                 = 2
 // The snapshot of each step is written by the folding kernel itself (no clone launches), so
 // the GEMM dequantizes with exactly the step the bytes were quantized with.
 #include <cuda_runtime.h>
@@ -312,23 +313,17 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
     }
     rc = launch_quantize_batch(bwd_jobs, nbj, stream);
     if (rc) return rc;
-    if (need_grad_x) {
-        // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T
-        rc = gemm_launch(g8, w8t, fmt, fmt, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x,
-                         stream);
-        if (rc) return rc;
-    }
-    if (need_grad_w) {
-        // grad_w [n][k] = g8t [n][m] . (x8t [k][m])^T
-        rc = gemm_launch(g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w,
-                         stream);
-        if (rc) return rc;
-    }
-    if (need_grad_b) {
-        const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
-        rc = launch_colsum_finalize(colsum, tiles, n, grad_b, stream);
-        if (rc) return rc;
-    }
+    // dX and dW in one launch over both tile spaces; its epilogue warps also finish grad_b
+    GemmDesc gd[2];
+    int ng = 0;
+    if (need_grad_x)  // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T
+        gd[ng++] = GemmDesc{g8, w8t, fmt, fmt, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x};
+    if (need_grad_w)  // grad_w [n][k] = g8t [n][m] . (x8t [k][m])^T
+        gd[ng++] = GemmDesc{g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
+    const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
+    rc = gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
+                           need_grad_b ? grad_b : nullptr, stream);
+    if (rc) return rc;
     return FP8DSA_OK;
 }
 
