@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 
@@ -612,24 +613,48 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
     return FP8DSA_OK;
 }
 
-// Tile shape for a launch: 256 x 256 tiles on CTA pairs when every problem has M > 128 and
-// N > 128 (each SM then reads half of the B operand from its shared memory); otherwise one
-// CTA per tile, 128 x 256, or 128 x 128 when some problem is at most 128 wide.  A 128 x 128
-// MMA reads as many operand bytes from shared memory per flop as the TMA writes into it and
-// measured far slower than the 256-wide tile.
+// Tile shape for a launch: 256 x 256 tiles on CTA pairs (each SM loads half of the B tile)
+// whenever every problem has M > 128 and N > 128; 128 x 256 on single CTAs when some M is at
+// most 128; 128 x 128 when some N is at most 128.  Measured on B200, a 128-wide MMA tile costs
+// almost as much time per k-block as a 256-wide one (4096^3: 1.57 vs 2.40 PFLOP/s), so narrower
+// tiles do not buy back wave quantization on these shapes.
 struct TileChoice {
     int bn;
     bool pair;
 };
 
+// Tuning override: FP8DSA_GEMM_TILE = "256p", "128p", "256" or "128" forces that tile shape
+// wherever the problem admits it (read once; unset = the default choice below).
+int tile_override() {
+    static const int v = [] {
+        const char* e = std::getenv("FP8DSA_GEMM_TILE");
+        if (e == nullptr) return 0;
+        const std::string t(e);
+        if (t == "256p") return 1;
+        if (t == "128p") return 2;
+        if (t == "256") return 3;
+        if (t == "128") return 4;
+        return 0;
+    }();
+    return v;
+}
+
 TileChoice choose_tiles(const GemmDesc* d, int n) {
-    bool narrow = false, short_m = false;
+    bool narrow = false, short_m = false, b_mn = false;
     for (int i = 0; i < n; ++i) {
         narrow = narrow || d[i].n <= 128;
         short_m = short_m || d[i].m <= kBM;
+        b_mn = b_mn || d[i].b_mn;
     }
     if (narrow) return {128, false};
-    return {256, !short_m};
+    if (short_m) return {256, false};
+    switch (tile_override()) {
+        case 2: if (!b_mn) return {128, true}; break;
+        case 3: return {256, false};
+        case 4: return {128, false};
+        default: break;
+    }
+    return {256, true};
 }
 
 }  // namespace
@@ -737,7 +762,7 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
 
     launch_begin(kKindGemm, stream);
     if (tc.pair)
-        rc = launch_cfg<256, true>(maps, g, batch, stream);
+        rc = tc.bn == 256 ? launch_cfg<256, true>(maps, g, batch, stream) : launch_cfg<128, true>(maps, g, batch, stream);
     else
         rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, stream) : launch_cfg<128, false>(maps, g, batch, stream);
     if (rc) return rc;
