@@ -57,6 +57,11 @@ def parse_args():
                    help="time one kernel on one shape instead of the step (small cases for ncu)")
     p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS")
     p.add_argument("--qmode", default="dual", choices=["row", "t", "dual"])
+    p.add_argument("--gemm-split-k", type=int, default=None,
+                   help="GEMM split-K mode: 0 automatic, 1 never, 2..4 forced (library default if omitted)")
+    p.add_argument("--tiled-persist-threshold", type=int, default=None,
+                   help="tile count above which transposed / dual quantize runs persistent "
+                        "(library default if omitted)")
     return p.parse_args()
 
 
@@ -385,6 +390,8 @@ def run_kernel_mode(args):
     import workloads as W
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.tiled_persist_threshold is not None:
+        F.fp8_set_tiled_persist_threshold(args.tiled_persist_threshold)
     dims = [int(v) for v in args.shape.split(",")]
     peaks = measured_peaks()
     if args.kernel == "gemm":
@@ -445,6 +452,10 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     F.lib()
+    if args.tiled_persist_threshold is not None:
+        F.fp8_set_tiled_persist_threshold(args.tiled_persist_threshold)
+    if args.gemm_split_k is not None:
+        F.fp8_set_gemm_split_k(args.gemm_split_k)
 
     lins = build_workload(F, W, torch, dev, seed_base=100000 * rank)
     flops_step = sum(l.gemm_flops for l in lins)

@@ -57,6 +57,8 @@ _SIGNATURES = {
     "fp8_set_wait_timeout_ns": (c_int, [c_uint64]),
     "fp8_debug_stalled_wait": (c_int, [_P]),
     "fp8_set_pdl": (c_int, [c_int]),
+    "fp8_set_tiled_persist_threshold": (c_int, [c_int64]),
+    "fp8_set_gemm_split_k": (c_int, [c_int]),
     "fp8_profiler_enable": (c_int, [c_int]),
     "fp8_profiler_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double)]),
     "fp8_last_error": (c_char_p, []),
@@ -235,6 +237,14 @@ def fp8_set_wait_timeout_ns(ns: int):
 
 def fp8_set_pdl(enabled: bool = True):
     return _check("fp8_set_pdl", lib().fp8_set_pdl(int(bool(enabled))))
+
+
+def fp8_set_gemm_split_k(splits: int = 1):
+    return _check("fp8_set_gemm_split_k", lib().fp8_set_gemm_split_k(int(splits)))
+
+
+def fp8_set_tiled_persist_threshold(min_tiles: int = 1024):
+    return _check("fp8_set_tiled_persist_threshold", lib().fp8_set_tiled_persist_threshold(int(min_tiles)))
 
 
 def fp8_debug_stalled_wait(stream=None):

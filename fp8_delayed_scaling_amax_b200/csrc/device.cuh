@@ -18,6 +18,8 @@ enum DeviceStatus : int {
     kStatusWaitMma = 0x102,        // GEMM MMA warp gave up waiting for operands / accumulator
     kStatusWaitEpilogue = 0x103,   // GEMM epilogue gave up waiting for an accumulator
     kStatusWaitDrain = 0x104,      // a drain wait (in-flight copies / MMAs) gave up
+    kStatusWaitQuantize = 0x105,   // tiled quantize gave up waiting for an input tile
+    kStatusWaitSplit = 0x106,      // split-K owner gave up waiting for its partial sums
     kStatusWaitDebug = 0x1FF,      // the deliberate stalled-wait test hook
 };
 
@@ -217,6 +219,35 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Device-scope release increment / acquire load of a global counter (split-K hand-off).
+__device__ __forceinline__ void counter_add_release(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t counter_load_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *p >= target (device-scope acquire).  Returns false, raising `abort_flag` and
+// recording `code`, if that takes longer than the timeout, or at once if `abort_flag` is
+// already raised.
+__device__ __forceinline__ bool counter_wait_bounded(const uint32_t* p, uint32_t target, const WaitCtl& ctl,
+                                                     volatile int* abort_flag, int code) {
+    if (counter_load_acquire(p) >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (counter_load_acquire(p) >= target) return true;
+        if (abort_flag != nullptr && *abort_flag) return false;
+        if (global_timer_ns() - t0 > ctl.timeout_ns) {
+            report_status(ctl, code);
+            if (abort_flag != nullptr) *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // CTA pairs (2-CTA clusters): one MMA spans both SMs' tensor cores, M = 256.
 // ---------------------------------------------------------------------------------------
@@ -355,6 +386,38 @@ __device__ __forceinline__ float fp8_to_float(uint8_t v) {
         asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(in));
     const uint16_t lo = static_cast<uint16_t>(h2 & 0xFFFFu);
     return __half2float(__ushort_as_half(lo));
+}
+
+// Packed running maximum of |x| over two bf16 (resp. f16) lanes: each lane of the result has
+// magnitude max(|acc|, |v|) (its sign is the xor of the operands' signs and carries no
+// meaning); a NaN operand lane returns the other lane's value, so NaN never enters.
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t acc, uint32_t v) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(v));
+    return r;
+}
+__device__ __forceinline__ uint32_t max_abs_f16x2(uint32_t acc, uint32_t v) {
+    uint32_t r;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(v));
+    return r;
+}
+
+// a = RN32(a * m), b = RN32(b * m) in one packed instruction.
+__device__ __forceinline__ void mul2_rn(float& a, float& b, float m) {
+    unsigned long long p, q;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(q) : "f"(m));
+    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(p) : "l"(q));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
+}
+
+// a = RN32(a + c), b = RN32(b + d) in one packed instruction.
+__device__ __forceinline__ void add2_rn(float& a, float& b, float c, float d) {
+    unsigned long long p, q;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(q) : "f"(c), "f"(d));
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(p) : "l"(q));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {

@@ -32,9 +32,11 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "internal.h"
 
@@ -77,7 +79,9 @@ struct Cfg {
 // One GEMM of a launch (a launch may carry two, e.g. dX and dW, over one tile space).
 struct GemmProblem {
     int m, n, k_blocks;
-    int tiles_m, tiles_n, tile_begin;
+    int tiles_m, tiles_n, tile_begin, tiles;  // tiles: all tiles of the problem (batch included)
+    int k_splits;                             // K ranges per tile (1 = no split)
+    int contrib_begin, owner_begin;           // first contributor unit / first owner (see decode_unit)
     int a_batched, b_batched;
     int a_mn, b_mn;
     uint32_t idesc;
@@ -104,6 +108,10 @@ struct GemmArgs {
     GemmProblem p[kMaxProblems];
     int nprob;
     int num_tiles;
+    int num_units, contrib_units;  // work units (tile, K range); the first contrib_units are split-K contributors
+    int splitk;                    // some problem has k_splits > 1
+    float* partial;                // split-K fp32 partial tiles: [contrib unit][CTA of the pair][BN/4][128][4]
+    uint32_t* counters;            // split-K arrivals per (tile, CTA of the pair); zero at launch
     ColsumJob colsum;
     WaitCtl wait;
 };
@@ -137,6 +145,67 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& pi
     tn = within / gm;
 }
 
+// Work unit -> (problem, tile, split, k-block range).  Without split-K a unit is a whole tile.
+// With it, tile t of problem p is cut into p.k_splits contiguous K ranges: the range s >= 1
+// is a contributor unit, which leaves its fp32 partial sum in the workspace; the range 0 is
+// the tile's owner, which adds the contributors' partials (in order s = 1, 2, ...) to its own
+// accumulator and writes the output.  Units [0, contrib_units) are all contributors (problem
+// by problem, split-major, tiles in order), the owners follow, problem by problem.  Every
+// CTA walks its units in increasing order and every contributor precedes its owner, so an
+// owner only ever waits for units that never wait themselves.
+struct Unit {
+    int pi, tile, split, kb0, kb1;
+};
+
+template <bool kSplit>
+__device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& g) {
+    Unit r;
+    if constexpr (!kSplit) {  // one unit per tile, the whole K range
+        r.pi = (g.nprob > 1 && u >= g.p[1].tile_begin) ? 1 : 0;
+        r.tile = u;
+        r.split = 0;
+        r.kb0 = 0;
+        r.kb1 = g.p[r.pi].k_blocks;
+        return r;
+    }
+    if (u < g.contrib_units) {
+        r.pi = (g.nprob > 1 && u >= g.p[1].contrib_begin) ? 1 : 0;
+        const GemmProblem& P = g.p[r.pi];
+        const int local = u - P.contrib_begin;
+        r.split = 1 + local / P.tiles;
+        r.tile = P.tile_begin + local % P.tiles;
+    } else {
+        const int o = u - g.contrib_units;
+        r.pi = (g.nprob > 1 && o >= g.p[1].owner_begin) ? 1 : 0;
+        const GemmProblem& P = g.p[r.pi];
+        r.split = 0;
+        r.tile = P.tile_begin + (o - P.owner_begin);
+    }
+    const GemmProblem& P = g.p[r.pi];
+    r.kb0 = (r.split * P.k_blocks) / P.k_splits;
+    r.kb1 = ((r.split + 1) * P.k_blocks) / P.k_splits;
+    return r;
+}
+
+// Contributor unit index of split s (>= 1) of tile `tile` of problem P.
+__device__ __forceinline__ int contrib_slot(const GemmProblem& P, int tile, int s) {
+    return P.contrib_begin + (s - 1) * P.tiles + (tile - P.tile_begin);
+}
+
+// Named barrier over `nthreads` threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);
@@ -149,7 +218,7 @@ __device__ __forceinline__ float bias_value(const GemmProblem& P, int col, float
     return __fmul_rn(P.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
 }
 
-template <int BN, bool kPair>
+template <int BN, bool kPair, bool kSplit>
 __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a0, const __grid_constant__ CUtensorMap tma_b0,
                     const __grid_constant__ CUtensorMap tma_o0, const __grid_constant__ CUtensorMap tma_a1,
@@ -225,9 +294,10 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;  // per-stage: ever issued, parity of the last issue
             bool ok = true;
-            for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
+            for (int u = unit; u < g.num_units && ok; u += units) {
+                const Unit w = decode_unit<kSplit>(u, g);
                 int pi, b, tm, tn;
-                decode_tile(tile, g, pi, b, tm, tn);
+                decode_tile(w.tile, g, pi, b, tm, tn);
                 const GemmProblem& P = g.p[pi];
                 const CUtensorMap* ta = pi ? &tma_a1 : &tma_a0;
                 const CUtensorMap* tb = pi ? &tma_b1 : &tma_b0;
@@ -235,7 +305,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 const int bb = P.b_batched ? b : 0;
                 const int arow = tm * C::kTileM + static_cast<int>(rank) * kBM;
                 const int brow = tn * BN + static_cast<int>(rank) * C::kBRows;
-                for (int kb = 0; kb < P.k_blocks; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_bounded(empty + stage, phase ^ 1u, g.wait, abort_flag, kStatusWaitProducer)) {
                         ok = false;
                         break;
@@ -293,10 +363,9 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
-            for (int tile = unit; tile < g.num_tiles && ok; tile += units) {
-                int pi, b, tm, tn;
-                decode_tile(tile, g, pi, b, tm, tn);
-                const GemmProblem& P = g.p[pi];
+            for (int u = unit; u < g.num_units && ok; u += units) {
+                const Unit w = decode_unit<kSplit>(u, g);
+                const GemmProblem& P = g.p[w.pi];
                 const bool got = kPair ? mbar_wait_bounded_cluster(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
                                                                    kStatusWaitMma)
                                        : mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
@@ -307,7 +376,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-                for (int kb = 0; kb < P.k_blocks; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_bounded(full + stage, phase, g.wait, abort_flag, kStatusWaitMma)) {
                         ok = false;
                         break;
@@ -323,10 +392,11 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                                                        : smem_desc(a_base + kk * kUmmaK, 16, 1024);
                             const uint64_t bd = P.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
                                                        : smem_desc(b_base + kk * kUmmaK, 16, 1024);
+                            const uint32_t accumulate = (kb != w.kb0 || kk != 0) ? 1u : 0u;
                             if constexpr (kPair)
-                                umma_f8f6f4_pair(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
+                                umma_f8f6f4_pair(d_tmem, ad, bd, P.idesc, accumulate);
                             else
-                                umma_f8f6f4(d_tmem, ad, bd, P.idesc, (kb | kk) != 0 ? 1u : 0u);
+                                umma_f8f6f4(d_tmem, ad, bd, P.idesc, accumulate);
                         }
                         if constexpr (kPair)
                             umma_commit_pair_multicast(empty + stage, 0x3);
@@ -411,10 +481,15 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
         const uint32_t acc_empty_leader0 = kPair ? mapa_shared(smem_addr(acc_empty), 0) : 0u;
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
-        for (int tile = unit; tile < g.num_tiles; tile += units) {
+        constexpr int kCtas = kPair ? 2 : 1;
+        const int row_in = q * 32 + lane;  // this thread's row within the CTA's 128 rows
+        for (int u = unit; u < g.num_units; u += units) {
+            const Unit w = decode_unit<kSplit>(u, g);
             int pi, b, tm, tn;
-            decode_tile(tile, g, pi, b, tm, tn);
+            decode_tile(w.tile, g, pi, b, tm, tn);
             const GemmProblem& P = g.p[pi];
+            const bool contrib = kSplit && w.split > 0;               // leave an fp32 partial sum
+            const bool owner = kSplit && !contrib && P.k_splits > 1;  // add the partials, then write
             const CUtensorMap* to = pi ? &tma_o1 : &tma_o0;
             const float scale = pi ? sc[1] : sc[0];
             const int col0 = tn * BN + cbase;
@@ -424,8 +499,22 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             float bias_r[C::kEpiCols / 32];
 #pragma unroll
             for (int j = 0; j < C::kEpiCols / 32; ++j) bias_r[j] = bias_value(P, col0 + 32 * j + lane, pi ? bsc[1] : bsc[0]);
-            if (!mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue)) break;
+            const bool got = mbar_wait_bounded(acc_full + acc, acc_phase, g.wait, abort_flag, kStatusWaitEpilogue);
+            if constexpr (kSplit) {
+                // split-K adds named barriers below: the epilogue warps leave together
+                if (named_barrier_or(1, C::kEpiThreads, !got)) break;
+            } else if (!got) {
+                break;
+            }
             tc_fence_after_sync();
+            if (owner) {
+                // one thread waits (acquire) until the tile's contributors have all arrived
+                bool arrived = true;
+                if (ew == 0 && lane == 0)
+                    arrived = counter_wait_bounded(g.counters + 2 * w.tile + rank, static_cast<uint32_t>(P.k_splits - 1),
+                                                   g.wait, abort_flag, kStatusWaitSplit);
+                if (named_barrier_or(1, C::kEpiThreads, !arrived)) break;
+            }
 #pragma unroll
             for (int c = 0; c < C::kEpiCols; c += kOutBox) {
                 uint32_t r0[32], r1[32];
@@ -436,6 +525,43 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 const float b_lo = bias_r[c / 32];
                 const float b_hi = bias_r[c / 32 + 1];
                 tmem_wait_ld();
+                const int cc = cbase + c;  // column within the tile
+                // Partial tiles are stored as [column group of 4][row][4]: for each group the 32
+                // lanes (rows) of a warp cover 512 contiguous bytes, one coalesced access.
+                if (contrib) {
+                    float4* dst = reinterpret_cast<float4*>(g.partial) +
+                                  ((static_cast<int64_t>(u) * kCtas + rank) * (BN / 4) + cc / 4) * kBM + row_in;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        __stcg(dst + v * kBM, make_float4(__uint_as_float(r0[4 * v]), __uint_as_float(r0[4 * v + 1]),
+                                                          __uint_as_float(r0[4 * v + 2]), __uint_as_float(r0[4 * v + 3])));
+                        __stcg(dst + (8 + v) * kBM,
+                               make_float4(__uint_as_float(r1[4 * v]), __uint_as_float(r1[4 * v + 1]),
+                                           __uint_as_float(r1[4 * v + 2]), __uint_as_float(r1[4 * v + 3])));
+                    }
+                    continue;
+                }
+                if (owner) {
+                    for (int sp = 1; sp < P.k_splits; ++sp) {
+                        const float4* src =
+                            reinterpret_cast<const float4*>(g.partial) +
+                            ((static_cast<int64_t>(contrib_slot(P, w.tile, sp)) * kCtas + rank) * (BN / 4) + cc / 4) * kBM +
+                            row_in;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const float4 p0 = __ldcg(src + v * kBM);
+                            const float4 p1 = __ldcg(src + (8 + v) * kBM);
+                            r0[4 * v] = __float_as_uint(__uint_as_float(r0[4 * v]) + p0.x);
+                            r0[4 * v + 1] = __float_as_uint(__uint_as_float(r0[4 * v + 1]) + p0.y);
+                            r0[4 * v + 2] = __float_as_uint(__uint_as_float(r0[4 * v + 2]) + p0.z);
+                            r0[4 * v + 3] = __float_as_uint(__uint_as_float(r0[4 * v + 3]) + p0.w);
+                            r1[4 * v] = __float_as_uint(__uint_as_float(r1[4 * v]) + p1.x);
+                            r1[4 * v + 1] = __float_as_uint(__uint_as_float(r1[4 * v + 1]) + p1.y);
+                            r1[4 * v + 2] = __float_as_uint(__uint_as_float(r1[4 * v + 2]) + p1.z);
+                            r1[4 * v + 3] = __float_as_uint(__uint_as_float(r1[4 * v + 3]) + p1.w);
+                        }
+                    }
+                }
                 uint32_t packed[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -489,6 +615,14 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             } else {
                 mbar_arrive(acc_empty + acc);
             }
+            if (contrib) {
+                // every epilogue thread has issued its partial stores; publish them (release)
+                named_barrier(1, C::kEpiThreads);
+                if (ew == 0 && lane == 0) {
+                    __threadfence();
+                    counter_add_release(g.counters + 2 * w.tile + rank, 1u);
+                }
+            }
             if (++acc == 2) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -533,44 +667,136 @@ __global__ void bias_fill_kernel(uint16_t* out, int64_t m, int64_t n, int64_t ld
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            p = nullptr;
-        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }();
-    return fn;
-}
-
 // 3-D tensor map: dims {inner, outer, batch} elements, row stride `ld` bytes, batch stride
 // `bstride` bytes, box {box_inner, box_outer, 1}, 128-byte swizzle, zero fill out of bounds.
 int make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner, int64_t outer,
              int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_outer) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
-                                static_cast<cuuint64_t>(batch)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(bstride)};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
-    return FP8DSA_OK;
+    return encode_tensor_map(map, dtype, base, inner, outer, batch, ld, bstride, box_inner, box_outer,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int BN, bool kPair>
-int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, cudaStream_t stream) {
+// Split-K planning: k_splits in 1..kMaxSplits per problem.  The automatic choice simulates
+// the static schedule as a two-stage pipeline per CTA (or pair): the MMAs of unit i overlap
+// the epilogue of unit i - 1, and an owner's epilogue also waits for its contributors'
+// partials.  Costs are B200 measurements of this kernel: kMmaUsPerKb per 256 x 256 x 128
+// k-block, and the epilogue of a plain tile, of a contributor (fp32 partial out) and of an
+// owner (partials in).  A range keeps at least 2 k-blocks, the contributors must fit the
+// partial workspace, and ties go to fewer splits.
+constexpr int kMaxSplits = 4;
+constexpr double kSetupUs = 1.5, kMmaUsPerKb = 0.42, kEpiUs = 2.5, kEpiContribUs = 4.6, kEpiOwnerUs = 3.8,
+                 kEpiOwnerExtraUs = 0.8;
+
+int range_len(const GemmProblem& P, int splits, int s) {
+    return ((s + 1) * P.k_blocks) / splits - (s * P.k_blocks) / splits;
+}
+
+// 0 = automatic split choice, 1 = never split (default), 2..kMaxSplits = that many ranges per
+// tile wherever the workspace and K allow (set by fp8_set_gemm_split_k).
+std::atomic<int> g_split_mode{1};
+
+// Modelled makespan (us) of the unit schedule with `sp` ranges per problem on `units` CTAs.
+double simulate_plan(const GemmArgs& g, const int* sp, int units, std::vector<double>& mma_end,
+                     std::vector<double>& epi_end, std::vector<double>& contrib_end) {
+    mma_end.assign(static_cast<size_t>(units), kSetupUs);
+    epi_end.assign(static_cast<size_t>(units), kSetupUs);
+    int64_t u = 0;
+    int64_t ncontrib = 0;
+    for (int i = 0; i < g.nprob; ++i) ncontrib += static_cast<int64_t>(sp[i] - 1) * g.p[i].tiles;
+    contrib_end.assign(static_cast<size_t>(std::max<int64_t>(ncontrib, 1)), 0.0);
+    auto run = [&](double mma, double epi, double ready) {
+        const size_t c = static_cast<size_t>(u % units);
+        mma_end[c] += mma;
+        const double start = std::max(std::max(mma_end[c], epi_end[c]), ready);
+        epi_end[c] = start + epi;
+        ++u;
+        return epi_end[c];
+    };
+    int64_t cb = 0;
+    for (int i = 0; i < g.nprob; ++i)
+        for (int sj = 1; sj < sp[i]; ++sj)
+            for (int t = 0; t < g.p[i].tiles; ++t)
+                contrib_end[static_cast<size_t>(cb++)] = run(range_len(g.p[i], sp[i], sj) * kMmaUsPerKb, kEpiContribUs, 0.0);
+    cb = 0;
+    for (int i = 0; i < g.nprob; ++i) {
+        const int64_t base = cb;
+        for (int t = 0; t < g.p[i].tiles; ++t) {
+            double ready = 0.0;
+            for (int sj = 1; sj < sp[i]; ++sj)
+                ready = std::max(ready, contrib_end[static_cast<size_t>(base + static_cast<int64_t>(sj - 1) * g.p[i].tiles + t)]);
+            const double epi = sp[i] > 1 ? kEpiOwnerUs + kEpiOwnerExtraUs * (sp[i] - 2) : kEpiUs;
+            run(range_len(g.p[i], sp[i], 0) * kMmaUsPerKb, epi, ready);
+        }
+        cb += static_cast<int64_t>(sp[i] - 1) * g.p[i].tiles;
+    }
+    return *std::max_element(epi_end.begin(), epi_end.end());
+}
+
+void plan_units(GemmArgs& g, int units, int64_t max_contrib, int64_t counter_words) {
+    int best[kMaxProblems] = {1, 1};
+    const int mode = g_split_mode.load();
+    const bool room = max_contrib > 0 && counter_words >= 2 * static_cast<int64_t>(g.num_tiles) && units > 0;
+    if (room && mode >= 2) {
+        int64_t contrib = 0;
+        for (int i = 0; i < g.nprob; ++i) {
+            const int64_t extra = static_cast<int64_t>(mode - 1) * g.p[i].tiles;
+            if (g.p[i].k_blocks >= 2 * mode && contrib + extra <= max_contrib) {
+                best[i] = mode;
+                contrib += extra;
+            }
+        }
+    } else if (room && mode == 0) {
+        double best_cost = 1e300;
+        int best_sum = 1 << 30;
+        std::vector<double> mma_end, epi_end, contrib_end;
+        const int lim1 = g.nprob > 1 ? kMaxSplits : 1;
+        for (int s0 = 1; s0 <= kMaxSplits; ++s0) {
+            for (int s1 = 1; s1 <= lim1; ++s1) {
+                const int sp[kMaxProblems] = {s0, s1};
+                int64_t contrib = 0;
+                bool ok = true;
+                for (int i = 0; i < g.nprob; ++i) {
+                    if (sp[i] > 1 && g.p[i].k_blocks < 2 * sp[i]) ok = false;
+                    contrib += static_cast<int64_t>(sp[i] - 1) * g.p[i].tiles;
+                }
+                if (!ok || contrib > max_contrib) continue;
+                const double cost = simulate_plan(g, sp, units, mma_end, epi_end, contrib_end);
+                const int sum = s0 + s1;
+                if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && sum < best_sum)) {
+                    best_cost = cost;
+                    best_sum = sum;
+                    best[0] = s0;
+                    best[1] = s1;
+                }
+            }
+        }
+    }
+    int64_t cb = 0;
+    for (int i = 0; i < g.nprob; ++i) {
+        g.p[i].k_splits = best[i];
+        g.p[i].contrib_begin = static_cast<int>(cb);
+        cb += static_cast<int64_t>(best[i] - 1) * g.p[i].tiles;
+    }
+    int64_t ob = 0;
+    for (int i = 0; i < g.nprob; ++i) {
+        g.p[i].owner_begin = static_cast<int>(ob);
+        ob += g.p[i].tiles;
+    }
+    g.contrib_units = static_cast<int>(cb);
+    g.num_units = static_cast<int>(cb + ob);
+    g.splitk = cb > 0 ? 1 : 0;
+}
+
+// One-time set-up of a kernel instance: its shared-memory limit and (pairs) how many
+// 2-CTA clusters fit on the device at once.
+template <int BN, bool kPair, bool kSplit>
+cudaError_t kernel_setup(int* max_units_out) {
     using C = Cfg<BN, kPair>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     static int max_units = 0;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmem);
         if (attr_err != cudaSuccess) return;
         if (kPair) {
             // how many 2-CTA clusters of this kernel fit on the device at once
@@ -586,11 +812,21 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
             cfg.attrs = at;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, kPair>, &cfg) == cudaSuccess && n > 0)
+            if (cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, kPair, kSplit>, &cfg) == cudaSuccess && n > 0)
                 max_units = n;
             cudaGetLastError();
         }
     });
+    *max_units_out = max_units;
+    return attr_err;
+}
+
+template <int BN, bool kPair>
+int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, const SplitWorkspace* split,
+               cudaStream_t stream) {
+    using C = Cfg<BN, kPair>;
+    int max_units = 0;
+    const cudaError_t attr_err = kernel_setup<BN, kPair, false>(&max_units);
     if (attr_err != cudaSuccess)
         return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(attr_err));
     int64_t tiles = 0;
@@ -600,15 +836,38 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
         P.tiles_n = (P.n + BN - 1) / BN;
         P.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
         P.tile_begin = static_cast<int>(tiles);
-        tiles += static_cast<int64_t>(P.tiles_m) * P.tiles_n * batch[i];
-        if (tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
+        const int64_t pt = static_cast<int64_t>(P.tiles_m) * P.tiles_n * batch[i];
+        tiles += pt;
+        if (tiles > (int64_t(1) << 28)) return fail(FP8DSA_ERR_UNSUPPORTED, "too many output tiles");
+        P.tiles = static_cast<int>(pt);
     }
     g.num_tiles = static_cast<int>(tiles);
     const int units = kPair ? (max_units > 0 ? max_units : sm_count() / 2) : sm_count();
-    const int grid_units = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, units)));
-    cudaError_t e = launch_ex(fp8_gemm_kernel<BN, kPair>, dim3(static_cast<unsigned>(grid_units * (kPair ? 2 : 1))),
-                              dim3(C::kThreads), C::kSmem, stream, kPair ? 2 : 1, maps[0], maps[1], maps[2], maps[3],
-                              maps[4], maps[5], g);
+    constexpr int64_t kUnitPartialBytes = int64_t(kPair ? 2 : 1) * kBM * BN * 4;
+    if (split != nullptr && split->partial != nullptr && split->counters != nullptr) {
+        g.partial = split->partial;
+        g.counters = split->counters;
+        plan_units(g, units, static_cast<int64_t>(split->partial_bytes) / kUnitPartialBytes, split->counter_words);
+    } else {
+        plan_units(g, units, 0, 0);
+    }
+    auto kernel = fp8_gemm_kernel<BN, kPair, false>;
+    if (g.splitk) {
+        int split_units = 0;
+        const cudaError_t se = kernel_setup<BN, kPair, true>(&split_units);
+        if (se != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(se));
+        // both instances must have every cluster of the plan resident at once
+        if (kPair && split_units > 0 && split_units < units) {
+            g.partial = nullptr;
+            g.counters = nullptr;
+            plan_units(g, units, 0, 0);
+        } else {
+            kernel = fp8_gemm_kernel<BN, kPair, true>;
+        }
+    }
+    const int grid_units = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g.num_units, units)));
+    cudaError_t e = launch_ex(kernel, dim3(static_cast<unsigned>(grid_units * (kPair ? 2 : 1))), dim3(C::kThreads),
+                              C::kSmem, stream, kPair ? 2 : 1, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], g);
     if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("fp8 gemm launch: ") + cudaGetErrorString(e));
     return FP8DSA_OK;
 }
@@ -659,8 +918,27 @@ TileChoice choose_tiles(const GemmDesc* d, int n) {
 
 }  // namespace
 
+size_t splitk_partial_bytes(const int64_t* m, const int64_t* n, int nprob) {
+    // (kMaxSplits - 1) contributors per tile; a tile's partial covers its padded output area
+    size_t total = 0;
+    for (int i = 0; i < nprob; ++i) {
+        if (m[i] <= 0 || n[i] <= 0) continue;
+        total += static_cast<size_t>(kMaxSplits - 1) * static_cast<size_t>(align_up(m[i], 256)) *
+                 static_cast<size_t>(align_up(n[i], 256)) * 4u;
+    }
+    return total;
+}
+
+int64_t splitk_counter_words(const int64_t* m, const int64_t* n, int nprob) {
+    // two counters per tile of the finest tiling (128 x 128)
+    int64_t total = 0;
+    for (int i = 0; i < nprob; ++i)
+        if (m[i] > 0 && n[i] > 0) total += 2 * ((m[i] + kBM - 1) / kBM) * ((n[i] + 127) / 128);
+    return total;
+}
+
 int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
-                      int64_t colsum_cols, void* colsum_out, cudaStream_t stream) {
+                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, cudaStream_t stream) {
     // problems with an empty product write their bias (or zeros) without the tensor cores
     GemmDesc work[kMaxProblems];
     int nwork = 0;
@@ -762,12 +1040,20 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
 
     launch_begin(kKindGemm, stream);
     if (tc.pair)
-        rc = tc.bn == 256 ? launch_cfg<256, true>(maps, g, batch, stream) : launch_cfg<128, true>(maps, g, batch, stream);
+        rc = tc.bn == 256 ? launch_cfg<256, true>(maps, g, batch, split, stream)
+                          : launch_cfg<128, true>(maps, g, batch, split, stream);
     else
-        rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, stream) : launch_cfg<128, false>(maps, g, batch, stream);
+        rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, split, stream)
+                          : launch_cfg<128, false>(maps, g, batch, split, stream);
     if (rc) return rc;
     launch_end(kKindGemm, stream, flops);
     return check_launch("fp8 gemm kernel");
+}
+
+int gemm_set_split_mode(int mode) {
+    if (mode < 0 || mode > kMaxSplits) return fail(FP8DSA_ERR_INVALID_ARG, "split_k must be 0 (automatic) .. 4");
+    g_split_mode.store(mode);
+    return FP8DSA_OK;
 }
 
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn, int b_mn, int64_t m,
@@ -776,7 +1062,7 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
                 int bias_kind, const float* bias_scale, void* out, cudaStream_t stream) {
     GemmDesc d{a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
                scale_a, scale_b, bias, bias_kind, bias_scale, out};
-    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, stream);
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, nullptr, stream);
 }
 
 }  // namespace fp8dsa

@@ -34,6 +34,13 @@ enum KernelKind : int { kKindQuantize = 0, kKindGemm = 1, kKindOther = 2 };
 void launch_begin(int kind, cudaStream_t stream);
 void launch_end(int kind, cudaStream_t stream, double work);
 
+// Encode a 3-D tiled tensor map (TMA descriptor): dims {inner, outer, batch} elements, row
+// stride `ld` bytes, batch stride `bstride` bytes, box {box_inner, box_outer, 1}, the given
+// shared-memory swizzle, zero fill out of bounds.  The driver entry point is looked up once.
+int encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner,
+                      int64_t outer, int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_outer,
+                      CUtensorMapSwizzle swizzle);
+
 // After a launch: map a launch failure to FP8DSA_ERR_CUDA.
 int check_launch(const char* what);
 
@@ -118,7 +125,10 @@ struct QuantJob {
 int launch_quantize(const QuantJob& job, cudaStream_t stream);
 // Up to three tensors in one launch (same format, input type and orientation); each tensor
 // keeps its own amax, ticket and ring fold.
-int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream);
+// `zero` / `zero_words` (optional): words the launch also sets to zero (split-K counters of
+// the GEMM that follows).
+int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, uint32_t* zero = nullptr,
+                          int64_t zero_words = 0);
 
 // grad_b[c] = RN_bf16(sum_t partial[t][c]) in a fixed order.
 int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,
@@ -138,10 +148,40 @@ struct GemmDesc {
     void* out;
 };
 
+// Split-K scratch a GEMM launch may use (see gemm_launch_group): fp32 partial tiles and one
+// arrival counter per (tile, CTA of a pair), which must be zero when the GEMM starts (the
+// quantize launch that precedes it in the linear compositions zeroes them).
+struct SplitWorkspace {
+    float* partial = nullptr;
+    size_t partial_bytes = 0;
+    uint32_t* counters = nullptr;
+    int64_t counter_words = 0;
+};
+// Scratch that lets a GEMM group split any of its problems' K into up to 4 ranges: partial
+// bytes and counter words for problems of the given output shapes.
+size_t splitk_partial_bytes(const int64_t* m, const int64_t* n, int nprob);
+int64_t splitk_counter_words(const int64_t* m, const int64_t* n, int nprob);
+
 // One or two GEMMs in one persistent launch over the union of their tiles; if colsum_tiles > 0
-// the epilogue warps first write colsum_out[c] = RN_bf16(sum_t colsum_partial[t][c]).
+// the epilogue warps first write colsum_out[c] = RN_bf16(sum_t colsum_partial[t][c]).  With
+// `split` (may be null) the launch may cut tiles' K ranges across CTAs where that shortens
+// the schedule; the result differs from the unsplit one only in fp32 summation order.
 int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
-                      int64_t colsum_cols, void* colsum_out, cudaStream_t stream);
+                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, cudaStream_t stream);
+
+// Split-K mode of later GEMM launches (0 automatic, 1 never, 2..4 forced); rejects others.
+int gemm_set_split_mode(int mode);
+
+// Workspace bytes of linear_forward_fp8 without the optional split-K region.
+size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n);
+
+// linear_forward_fp8 with a choice: allow_split = false needs only the base workspace and
+// runs the GEMM without split-K.
+int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
+                        const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                        const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                        float* sw_used, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
+                        cudaStream_t stream);
 
 // The GEMM entry with arguments already validated (used by the linear compositions).
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn_major,

@@ -26,8 +26,11 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr size_t kScratchBytes = 128;  // 3 x 16 B amax scratch + 4 internal fp32 steps
 
+// Each layout ends with the optional split-K region (the GEMM's arrival counters, then its
+// fp32 partial tiles); `base` is the size without it.
 struct FwdLayout {
-    size_t x8, w8, scratch, total;
+    size_t x8, w8, scratch, base, counters, partial, total;
+    int64_t counter_words;
 };
 
 FwdLayout fwd_layout(int64_t m, int64_t k, int64_t n) {
@@ -39,12 +42,20 @@ FwdLayout fwd_layout(int64_t m, int64_t k, int64_t n) {
     off = align_up(off + static_cast<size_t>(n) * k, kAlign);
     L.scratch = off;
     off = align_up(off + kScratchBytes, kAlign);
+    L.base = off;
+    const int64_t om[1] = {m}, on[1] = {n};  // y [m][n]
+    L.counter_words = splitk_counter_words(om, on, 1);
+    L.counters = off;
+    off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(L.counter_words), kAlign);
+    L.partial = off;
+    off = align_up(off + splitk_partial_bytes(om, on, 1), kAlign);
     L.total = off;
     return L;
 }
 
 struct BwdLayout {
-    size_t g8, g8t, x8t, w8t, colsum, scratch, total;
+    size_t g8, g8t, x8t, w8t, colsum, scratch, base, counters, partial, total;
+    int64_t counter_words;
 };
 
 BwdLayout bwd_layout(int64_t m, int64_t k, int64_t n) {
@@ -63,6 +74,13 @@ BwdLayout bwd_layout(int64_t m, int64_t k, int64_t n) {
     off = align_up(off + sizeof(float) * static_cast<size_t>((m + 127) / 128) * n, kAlign);
     L.scratch = off;
     off = align_up(off + kScratchBytes, kAlign);
+    L.base = off;
+    const int64_t om[2] = {m, n}, on[2] = {k, k};  // grad_x [m][k], grad_w [n][k]
+    L.counter_words = splitk_counter_words(om, on, 2);
+    L.counters = off;
+    off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(L.counter_words), kAlign);
+    L.partial = off;
+    off = align_up(off + splitk_partial_bytes(om, on, 2), kAlign);
     L.total = off;
     return L;
 }
@@ -88,15 +106,33 @@ size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
     return fwd_layout(m, k, n).total;
 }
 
+int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
+                       const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                       const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                       float* sw_used, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
+    return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
+                               sx_used, sw_used, workspace, workspace_bytes, true, y, stream);
+}
+
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
     if (m < 0 || k < 0 || n < 0) return 0;
     return bwd_layout(m, k, n).total;
 }
 
-int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
-                       const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
-                       const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
-                       float* sw_used, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
+}  // extern "C"
+
+namespace fp8dsa {
+
+size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n) {
+    if (m < 0 || k < 0 || n < 0) return 0;
+    return fwd_layout(m, k, n).base;
+}
+
+int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
+                        const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                        const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                        float* sw_used, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
+                        cudaStream_t stream) {
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
@@ -116,8 +152,9 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
         return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
     const FwdLayout L = fwd_layout(m, k, n);
-    if (workspace_bytes < L.total)
-        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    const size_t need = allow_split ? L.total : L.base;
+    if (workspace_bytes < need)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) + " bytes");
     if (w_is_fp8 && !aligned16(w)) return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 w must be 16-byte aligned");
     rc = check_device();
     if (rc) return rc;
@@ -188,14 +225,26 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
         }
         fwd_jobs[nfj++] = qw;
     }
-    // x and w in one launch, each with its own amax, ticket and ring fold
-    rc = launch_quantize_batch(fwd_jobs, nfj, stream);
+    SplitWorkspace split;
+    if (allow_split) {
+        split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+        split.counter_words = L.counter_words;
+        split.partial = reinterpret_cast<float*>(ws + L.partial);
+        split.partial_bytes = L.total - L.partial;
+    }
+    // x and w in one launch, each with its own amax, ticket and ring fold; it also zeroes the
+    // GEMM's split-K counters
+    rc = launch_quantize_batch(fwd_jobs, nfj, stream, split.counters, split.counter_words);
     if (rc) return rc;
     int bias_kind = 0;
     if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt == FP8_E4M3 ? 2 : 3);
-    return gemm_launch(x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y,
-                       stream);
+    const GemmDesc d{x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y};
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, allow_split ? &split : nullptr, stream);
 }
+
+}  // namespace fp8dsa
+
+extern "C" {
 
 int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
                         int need_grad_x, int need_grad_w, int need_grad_b, const float* sx_fwd, const float* sw_fwd,
@@ -311,7 +360,12 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         qw.scale = sw;
         bwd_jobs[nbj++] = qw;
     }
-    rc = launch_quantize_batch(bwd_jobs, nbj, stream);
+    SplitWorkspace split;
+    split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+    split.counter_words = L.counter_words;
+    split.partial = reinterpret_cast<float*>(ws + L.partial);
+    split.partial_bytes = L.total - L.partial;
+    rc = launch_quantize_batch(bwd_jobs, nbj, stream, split.counters, split.counter_words);
     if (rc) return rc;
     // dX and dW in one launch over both tile spaces; its epilogue warps also finish grad_b
     GemmDesc gd[2];
@@ -322,7 +376,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         gd[ng++] = GemmDesc{g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
     const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
     rc = gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
-                           need_grad_b ? grad_b : nullptr, stream);
+                           need_grad_b ? grad_b : nullptr, &split, stream);
     if (rc) return rc;
     return FP8DSA_OK;
 }

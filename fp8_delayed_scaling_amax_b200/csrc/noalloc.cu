@@ -11,8 +11,9 @@
 //
 // Set-up: the first call on each device looks up that array's device address with
 // cudaGetSymbolAddress, with that device current, and caches it; make that first call
-// before any stream capture.  Afterwards the call enqueues exactly what linear_forward_fp8
-// enqueues, and it allocates nothing.  Every call shares the one array, which keeps the
+// before any stream capture.  Afterwards the call enqueues what linear_forward_fp8 enqueues,
+// except that its GEMM never splits K (the array holds only the operand buffers and the
+// scale scratch), and it allocates nothing.  Every call shares the one array, which keeps the
 // last call's contents: the operand buffers are rewritten in full by each call and the
 // dynamic-scaling amax scratch is cleared by each call, but calls that overlap on the GPU
 // (different streams without ordering between them) race on the array.
@@ -62,7 +63,7 @@ extern "C" int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is
                                           float* sw_used, void* y, cudaStream_t stream) {
     clear_error();
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    const size_t need = linear_forward_fp8_workspace_size(m, k, n);
+    const size_t need = linear_forward_base_workspace(m, k, n);
     if (need > static_cast<size_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES))
         return fail(FP8DSA_ERR_WORKSPACE, "linear_forward_fp8_noalloc: this shape needs " + std::to_string(need) +
                                               " bytes of scratch; the built-in array holds " +
@@ -72,6 +73,8 @@ extern "C" int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is
     void* ws = nullptr;
     rc = noalloc_workspace(&ws);
     if (rc) return rc;
-    return linear_forward_fp8(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
-                              sx_used, sw_used, ws, static_cast<size_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES), y, stream);
+    // the GEMM runs without split-K: the built-in array holds only the operand buffers
+    return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
+                               sx_used, sw_used, ws, static_cast<size_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES), false, y,
+                               stream);
 }

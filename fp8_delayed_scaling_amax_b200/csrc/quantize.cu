@@ -10,19 +10,24 @@
 //  * Row-major quantize is a flat grid-stride kernel: 16 elements per thread-iteration
 //    (two or four 128-bit loads, one 128-bit store of packed fp8x4 words), two iterations
 //    in flight, grid = 8 resident 256-thread blocks per SM.
-//  * Transposed / dual quantize is tiled 128 x 128: coalesced 128-bit row loads, fp8 bytes
-//    staged in a 16 KB shared tile whose 16-byte chunks are XOR-swizzled by row group, then
-//    a register 4x4 byte transpose (PRMT) and 128-byte coalesced stores of each output row.
-//    The dual mode also writes the row-major bytes straight from registers, and can emit
-//    per-tile fp32 column sums (the bias gradient) from the values it already holds.
-//  * Each block reduces amax with warp shuffles, one atomicMax per block; with a ring, a
-//    threadfence + ticket elects the last block, which folds the amax into the window and
-//    publishes the next step.  No wait, no spin: the fold cannot stall.
+//  * Transposed / dual quantize is tiled 128 x 128 and persistent (two CTAs per SM walk all
+//    tiles of the batch): each 128 x 128 input tile arrives by one TMA bulk-tensor copy into
+//    a two-stage shared-memory ring, so the next tile loads while this one is converted;
+//    fp8 bytes are staged in a 16 KB shared tile whose 16-byte chunks are XOR-swizzled by row
+//    group, then a register 4x4 byte transpose (PRMT) and 128-byte coalesced stores of each
+//    output row.  The dual mode also writes the row-major bytes straight from registers, and
+//    can emit per-tile fp32 column sums (the bias gradient) from the values it already holds.
+//  * Each block reduces amax with warp shuffles, one atomicMax per block and tensor; with a
+//    ring, an acq_rel ticket elects the last block, which folds the amax into the window and
+//    publishes the next step.  The fold itself never waits; the tiled kernel's only wait (for
+//    its input copies) is bounded and reports a status code instead of hanging.
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 #include <string>
 
 #include "internal.h"
@@ -32,6 +37,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTile = 128;
+constexpr int64_t kMaxTiles = int64_t(1) << 30;  // tile indices stay far from int overflow
 
 // ----------------------------------------------------------------------------------------
 // Input element access
@@ -51,6 +57,16 @@ struct Bf16In {
         }
     }
     static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+    static __device__ __forceinline__ Raw lds_raw(const E* p) { return *reinterpret_cast<const uint4*>(p); }
+    // running max of |x| over raw words, two lanes per instruction
+    using Acc = uint32_t;
+    static __device__ __forceinline__ Acc acc_zero() { return 0u; }
+    static __device__ __forceinline__ void acc_max(Acc& acc, const Raw& v) {
+        acc = max_abs_bf16x2(max_abs_bf16x2(acc, v.x), max_abs_bf16x2(v.y, max_abs_bf16x2(v.z, v.w)));
+    }
+    static __device__ __forceinline__ float acc_value(Acc acc) {
+        return fmaxf(fabsf(__uint_as_float(acc << 16)), fabsf(__uint_as_float(acc & 0xFFFF0000u)));
+    }
 };
 
 struct F16In {
@@ -67,6 +83,16 @@ struct F16In {
         }
     }
     static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+    static __device__ __forceinline__ Raw lds_raw(const E* p) { return *reinterpret_cast<const uint4*>(p); }
+    using Acc = uint32_t;
+    static __device__ __forceinline__ Acc acc_zero() { return 0u; }
+    static __device__ __forceinline__ void acc_max(Acc& acc, const Raw& v) {
+        acc = max_abs_f16x2(max_abs_f16x2(acc, v.x), max_abs_f16x2(v.y, max_abs_f16x2(v.z, v.w)));
+    }
+    static __device__ __forceinline__ float acc_value(Acc acc) {
+        return fmaxf(fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>(acc & 0xFFFFu)))),
+                     fabsf(__half2float(__ushort_as_half(static_cast<uint16_t>(acc >> 16)))));
+    }
 };
 
 struct F32Raw {
@@ -85,6 +111,16 @@ struct F32In {
         f[4] = v.b.x; f[5] = v.b.y; f[6] = v.b.z; f[7] = v.b.w;
     }
     static __device__ __forceinline__ void load8(const E* p, float (&f)[8]) { unpack(load_raw(p), f); }
+    static __device__ __forceinline__ Raw lds_raw(const E* p) {
+        return {reinterpret_cast<const float4*>(p)[0], reinterpret_cast<const float4*>(p)[1]};
+    }
+    using Acc = float;
+    static __device__ __forceinline__ Acc acc_zero() { return 0.0f; }
+    static __device__ __forceinline__ void acc_max(Acc& acc, const Raw& v) {
+        acc = fmaxf(acc, fmaxf(fmaxf(fmaxf(fabsf(v.a.x), fabsf(v.a.y)), fmaxf(fabsf(v.a.z), fabsf(v.a.w))),
+                               fmaxf(fmaxf(fabsf(v.b.x), fabsf(v.b.y)), fmaxf(fabsf(v.b.z), fabsf(v.b.w)))));
+    }
+    static __device__ __forceinline__ float acc_value(Acc acc) { return acc; }
 };
 
 // Arguments of the quantize kernels (one POD by value).
@@ -102,27 +138,36 @@ struct QArgs {
     float* scale_used_out;     // receives the step used, or null
     float* colsum;             // [row tiles][cols] per-tile column sums (tiled kernel), or null
     int vec_in, vec_out, vec_out_t;
+    int tma;                   // tiled kernel: input tiles arrive by TMA through map[job]
     unsigned nblocks;          // blocks working on this tensor (the ticket count of its fold)
-    int tile_begin, tiles_x;   // tiled kernel: first block of this tensor, column tiles
+    int tile_begin, tiles_x;   // tiled kernel: first tile of this tensor, column tiles
 };
 
 // Up to three tensors quantized by one launch; each keeps its own amax, ticket and fold.
 constexpr int kMaxJobs = 3;
 struct QBatch {
+    CUtensorMap map[kMaxJobs];  // tiled kernel: [rows][cols] input, box 128 x 128, no swizzle
     QArgs job[kMaxJobs];
     int njobs;
+    int tiles_total;            // tiled kernel: tiles of all jobs, concatenated
+    uint32_t* zero;             // side job of the launch's first block: zero[0 .. zero_words)
+    int64_t zero_words;
 };
 
-// Eight floats -> eight fp8 bytes (two words), updating amax over the raw values.
+// The side job: the first block of the launch clears the words (after pdl_wait, so the
+// kernel that last used them has finished).
+__device__ __forceinline__ void zero_side_job(const QBatch& b) {
+    if (b.zero_words > 0 && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int64_t i = threadIdx.x; i < b.zero_words; i += blockDim.x) b.zero[i] = 0u;
+}
+
+// Eight floats -> eight fp8 bytes (two words): each byte is the RN, saturating encoding of
+// RN32(f * mult), the products taken two per packed instruction; amax is kept by the caller.
 template <int kFmt>
-__device__ __forceinline__ uint2 convert8(const float (&f)[8], float mult, float& amax) {
+__device__ __forceinline__ uint2 quant8(float (&f)[8], float mult) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
-    const uint32_t w0 = cvt_fp8x4<kFmt>(__fmul_rn(f[0], mult), __fmul_rn(f[1], mult),
-                                        __fmul_rn(f[2], mult), __fmul_rn(f[3], mult));
-    const uint32_t w1 = cvt_fp8x4<kFmt>(__fmul_rn(f[4], mult), __fmul_rn(f[5], mult),
-                                        __fmul_rn(f[6], mult), __fmul_rn(f[7], mult));
-    return make_uint2(w0, w1);
+    for (int e = 0; e < 8; e += 2) mul2_rn(f[e], f[e + 1], mult);
+    return make_uint2(cvt_fp8x4<kFmt>(f[0], f[1], f[2], f[3]), cvt_fp8x4<kFmt>(f[4], f[5], f[6], f[7]));
 }
 
 template <int kFmt>
@@ -140,32 +185,20 @@ __device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
 
 constexpr int kHistPrefetch = 64;
 
-__device__ __forceinline__ float* hist_smem() {
-    __shared__ float s_hist[kHistPrefetch];
-    return s_hist;
-}
-
 // Called at kernel start: copy the ring's history window (it does not change during the
 // kernel; only the last block writes it, at the very end) into shared memory, so the fold
-// does not pay one dependent L2 round trip per slot.  Visible after block_finish's barrier.
-__device__ __forceinline__ void ring_prefetch(const QArgs& a) {
+// does not pay one dependent L2 round trip per slot.  Visible after the next barrier.
+__device__ __forceinline__ void ring_prefetch(const QArgs& a, float* hist) {
     if (a.ring_state != nullptr && a.hist_len <= kHistPrefetch && static_cast<int>(threadIdx.x) < a.hist_len)
-        hist_smem()[threadIdx.x] = __ldcg(a.ring_state + threadIdx.x);
+        hist[threadIdx.x] = __ldcg(a.ring_state + threadIdx.x);
 }
 
-// Block-wide amax reduce, one atomic per block, then (with a ring) the last-block fold:
-// scale_used = step, hist[idx] = amax, scale = max(RN32(peak / fp8_max) / 2^m, 1e-12),
-// amax and done slots re-zeroed.  Every thread of the block must call this.
-__device__ __forceinline__ void block_finish(const QArgs& a, float amax, float step, bool first_block) {
-    __shared__ float red[32];
-    const int tid = threadIdx.x;
-    amax = warp_max(amax);
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
-    __syncthreads();
-    if (tid != 0) return;
-    const int nwarps = (blockDim.x + 31) >> 5;
-    float m = red[0];
-    for (int w = 1; w < nwarps; ++w) m = fmaxf(m, red[w]);
+// One thread per block and tensor, with the block's amax `m`: one atomicMax, then (with a
+// ring) the ticket; the block that draws the last ticket folds: scale_used = step,
+// hist[idx] = amax, scale = max(RN32(peak / fp8_max) / 2^m, 1e-12), amax and done slots
+// re-zeroed.  `hist` is the prefetched window.
+__device__ __forceinline__ void job_finish(const QArgs& a, float m, float step, bool first_block,
+                                           const float* hist) {
     if (a.amax_accum != nullptr) atomicMax(reinterpret_cast<unsigned*>(a.amax_accum), __float_as_uint(m));
     if (a.ring_state != nullptr) {
         float* st = a.ring_state;
@@ -178,9 +211,8 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
         st[a.hist_idx] = am;
         float peak = am;
         if (n <= kHistPrefetch) {
-            const float* h = hist_smem();
             for (int i = 0; i < n; ++i)
-                if (i != a.hist_idx) peak = fmaxf(peak, h[i]);
+                if (i != a.hist_idx) peak = fmaxf(peak, hist[i]);
         } else {
             for (int i = 0; i < n; ++i) peak = fmaxf(peak, __ldcg(st + i));
         }
@@ -194,6 +226,21 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
     }
 }
 
+// Block-wide amax reduce followed by job_finish on thread 0.  Every thread must call this.
+__device__ __forceinline__ void block_finish(const QArgs& a, float amax, float step, bool first_block,
+                                             const float* hist) {
+    __shared__ float red[32];
+    const int tid = threadIdx.x;
+    amax = warp_max(amax);
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    if (tid != 0) return;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    float m = red[0];
+    for (int w = 1; w < nwarps; ++w) m = fmaxf(m, red[w]);
+    job_finish(a, m, step, first_block, hist);
+}
+
 // ----------------------------------------------------------------------------------------
 // Row-major quantize: flat, grid-stride, 16 elements per thread per iteration.
 // ----------------------------------------------------------------------------------------
@@ -201,12 +248,15 @@ template <class In, int kFmt>
 __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_constant__ QBatch batch) {
     pdl_trigger();
     pdl_wait();
+    zero_side_job(batch);
     const QArgs& a = batch.job[blockIdx.y];  // one grid row of blocks per tensor
-    ring_prefetch(a);
+    __shared__ float s_hist[kHistPrefetch];
+    ring_prefetch(a, s_hist);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
     float amax = 0.0f;
+    typename In::Acc acc = In::acc_zero();  // running max of |x| over the vector chunks
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t n16 = a.vec_in ? a.numel / 16 : 0;
@@ -221,156 +271,308 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
             r3 = In::load_raw(x + g1 * 16 + 8);
         }
         float f0[8], f1[8];
+        In::acc_max(acc, r0);
+        In::acc_max(acc, r1);
         In::unpack(r0, f0);
         In::unpack(r1, f1);
-        const uint2 lo = convert8<kFmt>(f0, mult, amax);
-        const uint2 hi = convert8<kFmt>(f1, mult, amax);
+        const uint2 lo = quant8<kFmt>(f0, mult);
+        const uint2 hi = quant8<kFmt>(f1, mult);
         *reinterpret_cast<uint4*>(a.out + g * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
         if (has1) {
+            In::acc_max(acc, r2);
+            In::acc_max(acc, r3);
             In::unpack(r2, f0);
             In::unpack(r3, f1);
-            const uint2 lo1 = convert8<kFmt>(f0, mult, amax);
-            const uint2 hi1 = convert8<kFmt>(f1, mult, amax);
+            const uint2 lo1 = quant8<kFmt>(f0, mult);
+            const uint2 hi1 = quant8<kFmt>(f1, mult);
             *reinterpret_cast<uint4*>(a.out + g1 * 16) = make_uint4(lo1.x, lo1.y, hi1.x, hi1.y);
         }
     }
+    amax = In::acc_value(acc);
     for (int64_t i = n16 * 16 + tid; i < a.numel; i += gstride) {
         const float v = In::cvt(x[i]);
         amax = fmaxf(amax, fabsf(v));
         a.out[i] = convert1<kFmt>(v, mult);
     }
-    block_finish(a, amax, step, blockIdx.x == 0);
+    block_finish(a, amax, step, blockIdx.x == 0, s_hist);
 }
 
 // ----------------------------------------------------------------------------------------
-// Transposed / dual quantize: 128 x 128 tiles through a swizzled shared byte tile.
+// Transposed / dual quantize over the 128 x 128 tiles of every tensor of the batch.
+//  * Persistent (large batches): two CTAs per SM walk all tiles; each input tile arrives by
+//    one TMA copy into a two-stage shared-memory ring, so the next tile loads while this one
+//    is converted (tensors whose rows are not 16-byte aligned are read directly instead).
+//  * One tile per CTA (small batches): three CTAs per SM, the input read straight into
+//    registers, so every resident CTA has its whole tile in flight at once.
+// Either way the fp8 bytes go through a swizzled shared byte tile for the transpose.
 // ----------------------------------------------------------------------------------------
-template <class In, int kFmt>
-__global__ void __launch_bounds__(kThreads, sizeof(typename In::Raw) > 16 ? 2 : 3)
-    quant_tiled_kernel(const __grid_constant__ QBatch batch) {
-    // 128 rows x 128 bytes; the 16-byte chunk c of row r lives at chunk c ^ ((r >> 4) & 7).
-    __shared__ __align__(16) uint32_t tile[kTile * 32];
-    __shared__ float csum[8][kTile];
+// Shared-memory layout of the tiled kernel.  Persistent: two input stages fed by TMA, the
+// fp8 byte tile, the column sums, one mbarrier per stage.  One tile per CTA: the byte tile
+// and the column sums only (its input is loaded into registers).
+template <class In, bool kPersist>
+struct TiledCfg {
+    static constexpr bool kF32 = sizeof(typename In::E) == 4;
+    static constexpr int kStages = kPersist ? 2 : 0;
+    static constexpr int kRawBytes = kTile * kTile * static_cast<int>(sizeof(typename In::E));
+    static constexpr int kOffTile = kStages * kRawBytes;       // 128 x 128 fp8 byte tile
+    static constexpr int kOffCsum = kOffTile + kTile * kTile;  // 8 x 128 fp32 column sums
+    static constexpr int kOffBar = kOffCsum + 8 * kTile * 4;   // one mbarrier per stage
+    static constexpr int kSmem = kOffBar + kStages * 8 + 1024; // + slack to align the base
+    static constexpr int kMinBlocks = kPersist ? (kF32 ? 1 : 2) : (kF32 ? 2 : 3);
+};
 
+__device__ __forceinline__ int tile_job(const QBatch& b, int tl) {
+    int jb = 0;
+    while (jb + 1 < b.njobs && tl >= b.job[jb + 1].tile_begin) ++jb;
+    return jb;
+}
+
+template <class In, int kFmt, bool kPersist>
+__global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
+    quant_tiled_kernel(const __grid_constant__ QBatch batch, const WaitCtl ctl) {
+    using C = TiledCfg<In, kPersist>;
+    using E = typename In::E;
+    extern __shared__ uint8_t dsmem[];
+    const uint32_t base = smem_addr(dsmem);
+    uint8_t* smem = dsmem + (((base + 1023u) & ~1023u) - base);
+    float(*csum)[kTile] = reinterpret_cast<float(*)[kTile]>(smem + C::kOffCsum);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    __shared__ float s_hist[kMaxJobs][kHistPrefetch];
+    __shared__ float s_red[kMaxJobs][kThreads / 32];
+    __shared__ int s_abort;
+
+    const int t = threadIdx.x;
+    const int njobs = batch.njobs;
+    if constexpr (kPersist) {
+        if (t == 0) {
+            for (int s = 0; s < C::kStages; ++s) mbar_init(&bar[s], 1);
+            fence_mbar_init();
+            s_abort = 0;
+            for (int jb = 0; jb < njobs; ++jb)
+                if (batch.job[jb].tma) prefetch_tensormap(&batch.map[jb]);
+        }
+        __syncthreads();
+    }
     pdl_trigger();
     pdl_wait();
-    int jb = 0;
-    while (jb + 1 < batch.njobs && static_cast<int>(blockIdx.x) >= batch.job[jb + 1].tile_begin) ++jb;
-    const QArgs& a = batch.job[jb];
-    const bool row_out = a.out != nullptr;
-    const bool colsum = a.colsum != nullptr;
-    ring_prefetch(a);
-    const float step = __ldg(a.scale);
-    const float mult = __frcp_rn(step);
-    const auto* x = static_cast<const typename In::E*>(a.x);
-    const int64_t rows = a.rows, cols = a.cols;
-    const int local = static_cast<int>(blockIdx.x) - a.tile_begin;
-    const int tile_y = local / a.tiles_x;
-    const int64_t r0 = static_cast<int64_t>(tile_y) * kTile;
-    const int64_t c0 = static_cast<int64_t>(local % a.tiles_x) * kTile;
-    const int t = threadIdx.x;
+    zero_side_job(batch);
+    if constexpr (kPersist) {
+        for (int jb = 0; jb < njobs; ++jb) ring_prefetch(batch.job[jb], s_hist[jb]);
+    } else {
+        const int jb = tile_job(batch, static_cast<int>(blockIdx.x));
+        ring_prefetch(batch.job[jb], s_hist[jb]);
+    }
+
+    const int total = batch.tiles_total;
+    const int gstride = static_cast<int>(gridDim.x);
+    uint32_t pending = 0;  // thread 0: stages with a load in flight
+    // Thread 0: start the load of tile `tl` into stage `s` (TMA-fed tensors only).
+    auto issue = [&](int tl, int s) {
+        const int jb = tile_job(batch, tl);
+        const QArgs& a = batch.job[jb];
+        if (!kPersist || !a.tma) return;
+        const int local = tl - a.tile_begin;
+        mbar_arrive_expect_tx(&bar[s], C::kRawBytes);
+        tma_load_3d(smem + s * C::kRawBytes, &batch.map[jb], &bar[s], (local % a.tiles_x) * kTile,
+                    (local / a.tiles_x) * kTile, 0);
+        pending |= 1u << s;
+    };
+    if (t == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            const int tl = static_cast<int>(blockIdx.x) + s * gstride;
+            if (tl < total) issue(tl, s);
+        }
+    }
+
     const int j = t & 15;   // 8-column group of the tile
     const int rr = t >> 4;  // row within each 16-row slab
-    const int64_t gc = c0 + 8 * j;
-    const bool interior = a.vec_in && r0 + kTile <= rows && c0 + kTile <= cols;
-
-    float amax = 0.0f;
-    float cs[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) cs[e] = 0.0f;
-
-    typename In::Raw raw[8];
-    if (interior) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) raw[i] = In::load_raw(x + (r0 + rr + 16 * i) * cols + gc);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = rr + 16 * i;
-        const int64_t gr = r0 + r;
-        float f[8];
-        if (interior) {
-            In::unpack(raw[i], f);
-        } else if (gr < rows && a.vec_in && gc + 8 <= cols) {
-            In::load8(x + gr * cols + gc, f);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                f[e] = (gr < rows && gc + e < cols) ? In::cvt(x[gr * cols + gc + e]) : 0.0f;
-        }
-        if (colsum) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) cs[e] += f[e];
-        }
-        const uint2 w = convert8<kFmt>(f, mult, amax);
-        if (row_out) {
-            if (gr < rows) {
-                uint8_t* dst = a.out + gr * cols + gc;
-                if (a.vec_out && gc + 8 <= cols) {
-                    *reinterpret_cast<uint2*>(dst) = w;
-                } else {
-                    const uint32_t ww[2] = {w.x, w.y};
-                    for (int e = 0; e < 8 && gc + e < cols; ++e)
-                        dst[e] = static_cast<uint8_t>(ww[e >> 2] >> (8 * (e & 3)));
-                }
-            }
-        }
-        const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
-        *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = w;
-    }
-
-    if (colsum) {
-        // lanes l and l ^ 16 share the column group; then the 8 warps go through shared memory
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
-        if ((t & 16) == 0) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) csum[t >> 5][8 * j + e] = cs[e];
-        }
-    }
-    __syncthreads();
-
-    if (colsum) {
-        if (t < kTile && c0 + t < cols) {
-            float s = 0.0f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) s += csum[w][t];
-            a.colsum[static_cast<int64_t>(tile_y) * cols + c0 + t] = s;
-        }
-    }
-
-    // Phase 2: warp w owns tile columns 16w .. 16w+15; lane -> (column group of 4, 16 rows).
     const int w = t >> 5, lane = t & 31;
     const int cgl = lane & 3, rg = lane >> 2;
-    uint32_t W[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) W[i] = tile[(16 * rg + i) * 32 + ((w ^ rg) << 2) + cgl];
-    uint32_t O[4][4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t x0 = __byte_perm(W[4 * k], W[4 * k + 1], 0x5140);
-        const uint32_t x1 = __byte_perm(W[4 * k], W[4 * k + 1], 0x7362);
-        const uint32_t y0 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x5140);
-        const uint32_t y1 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x7362);
-        O[0][k] = __byte_perm(x0, y0, 0x5410);
-        O[1][k] = __byte_perm(x0, y0, 0x7632);
-        O[2][k] = __byte_perm(x1, y1, 0x5410);
-        O[3][k] = __byte_perm(x1, y1, 0x7632);
-    }
-    const int64_t gr0 = r0 + 16 * rg;
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        const int64_t c = c0 + 4 * (4 * w + cgl) + jj;
-        if (c >= cols || gr0 >= rows) continue;
-        uint8_t* dst = a.out_t + c * rows + gr0;
-        if (a.vec_out_t && gr0 + 16 <= rows) {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(O[jj][0], O[jj][1], O[jj][2], O[jj][3]);
-        } else {
-            for (int b = 0; b < 16 && gr0 + b < rows; ++b)
-                dst[b] = static_cast<uint8_t>(O[jj][b >> 2] >> (8 * (b & 3)));
+    float am0 = 0.0f, am1 = 0.0f, am2 = 0.0f;  // this thread's amax per tensor
+    uint32_t parity = 0;                       // bit s: parity of stage s's next completion
+    bool aborted = false;
+    int it = 0;
+    for (int tl = static_cast<int>(blockIdx.x); tl < total; tl += gstride, ++it) {
+        const int s = kPersist ? it % (C::kStages > 0 ? C::kStages : 1) : 0;
+        const int jb = tile_job(batch, tl);
+        const QArgs& a = batch.job[jb];
+        const bool row_out = a.out != nullptr;
+        const bool colsum = a.colsum != nullptr;
+        const float mult = __frcp_rn(__ldg(a.scale));
+        const auto* x = static_cast<const E*>(a.x);
+        const int64_t rows = a.rows, cols = a.cols;
+        const int local = tl - a.tile_begin;
+        const int tile_y = local / a.tiles_x;
+        const int64_t r0 = static_cast<int64_t>(tile_y) * kTile;
+        const int64_t c0 = static_cast<int64_t>(local % a.tiles_x) * kTile;
+        const int64_t gc = c0 + 8 * j;
+        const bool from_smem = kPersist && a.tma != 0;
+        const bool interior = !from_smem && a.vec_in && r0 + kTile <= rows && c0 + kTile <= cols;
+        bool ok = true;
+        if (from_smem) {
+            ok = mbar_wait_bounded(&bar[s], (parity >> s) & 1u, ctl, &s_abort, kStatusWaitQuantize);
+            if (ok) {
+                parity ^= 1u << s;
+                if (t == 0) pending &= ~(1u << s);
+            }
         }
+        const E* stage = reinterpret_cast<const E*>(smem + s * C::kRawBytes);
+        // The tile's fp8 bytes, 128 rows x 128 bytes, in the first 16 KB of stage s: the
+        // 16-byte chunk c of row r lives at chunk c ^ ((r >> 4) & 7).
+        uint32_t* tile = reinterpret_cast<uint32_t*>(smem + C::kOffTile);
+
+        float tamax = 0.0f;                          // amax of the rows read element-wise
+        typename In::Acc acc = In::acc_zero();       // amax of the rows read as raw chunks
+        float cs[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] = 0.0f;
+        typename In::Raw raw[8];
+        if (from_smem) {
+            // out-of-range rows / columns of an edge tile were zero-filled by the copy
+#pragma unroll
+            for (int i = 0; i < 8; ++i) raw[i] = In::lds_raw(stage + (rr + 16 * i) * kTile + 8 * j);
+        } else if (interior) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) raw[i] = In::load_raw(x + (r0 + rr + 16 * i) * cols + gc);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rr + 16 * i;
+            const int64_t gr = r0 + r;
+            float f[8];
+            if (from_smem || interior) {
+                In::acc_max(acc, raw[i]);
+                In::unpack(raw[i], f);
+            } else {
+                if (gr < rows && a.vec_in && gc + 8 <= cols) {
+                    In::load8(x + gr * cols + gc, f);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = (gr < rows && gc + e < cols) ? In::cvt(x[gr * cols + gc + e]) : 0.0f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tamax = fmaxf(tamax, fabsf(f[e]));
+            }
+            if (colsum) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
+            }
+            const uint2 q = quant8<kFmt>(f, mult);
+            if (row_out && gr < rows) {
+                uint8_t* dst = a.out + gr * cols + gc;
+                if (a.vec_out && gc + 8 <= cols) {
+                    *reinterpret_cast<uint2*>(dst) = q;
+                } else {
+                    const uint32_t qq[2] = {q.x, q.y};
+                    for (int e = 0; e < 8 && gc + e < cols; ++e)
+                        dst[e] = static_cast<uint8_t>(qq[e >> 2] >> (8 * (e & 3)));
+                }
+            }
+            const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
+            *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = q;
+        }
+        tamax = fmaxf(tamax, In::acc_value(acc));
+        if (jb == 0)
+            am0 = fmaxf(am0, tamax);
+        else if (jb == 1)
+            am1 = fmaxf(am1, tamax);
+        else
+            am2 = fmaxf(am2, tamax);
+        if (colsum) {
+            // lanes l and l ^ 16 share the column group; then the 8 warps go through shared memory
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
+            if ((t & 16) == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) csum[w][8 * j + e] = cs[e];
+            }
+        }
+        // The byte tile is complete; every thread agrees on `ok`.
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        if (t == 0) {  // stage s has been read: refill it
+            const int nt = tl + C::kStages * gstride;
+            if (nt < total) issue(nt, s);
+        }
+
+        if (colsum && t < kTile && c0 + t < cols) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) sum += csum[v][t];
+            a.colsum[static_cast<int64_t>(tile_y) * cols + c0 + t] = sum;
+        }
+
+        // Phase 2: warp w owns tile columns 16w .. 16w+15; lane -> (column group of 4, 16 rows).
+        uint32_t W[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) W[i] = tile[(16 * rg + i) * 32 + ((w ^ rg) << 2) + cgl];
+        uint32_t O[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t x0 = __byte_perm(W[4 * k], W[4 * k + 1], 0x5140);
+            const uint32_t x1 = __byte_perm(W[4 * k], W[4 * k + 1], 0x7362);
+            const uint32_t y0 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x5140);
+            const uint32_t y1 = __byte_perm(W[4 * k + 2], W[4 * k + 3], 0x7362);
+            O[0][k] = __byte_perm(x0, y0, 0x5410);
+            O[1][k] = __byte_perm(x0, y0, 0x7632);
+            O[2][k] = __byte_perm(x1, y1, 0x5410);
+            O[3][k] = __byte_perm(x1, y1, 0x7632);
+        }
+        const int64_t gr0 = r0 + 16 * rg;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int64_t c = c0 + 4 * (4 * w + cgl) + jj;
+            if (c >= cols || gr0 >= rows) continue;
+            uint8_t* dst = a.out_t + c * rows + gr0;
+            if (a.vec_out_t && gr0 + 16 <= rows) {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(O[jj][0], O[jj][1], O[jj][2], O[jj][3]);
+            } else {
+                for (int b = 0; b < 16 && gr0 + b < rows; ++b)
+                    dst[b] = static_cast<uint8_t>(O[jj][b >> 2] >> (8 * (b & 3)));
+            }
+        }
+        __syncthreads();  // the byte tile and the column sums are free
     }
-    block_finish(a, amax, step, local == 0);
+
+    if (aborted) {
+        // A tile never arrived: let this CTA's copies in flight land, leave the fold undone
+        // (the status word reports the failure) and return.
+        if (t == 0) {
+            for (int s = 0; s < C::kStages; ++s)
+                if ((pending >> s) & 1u) mbar_wait_bounded(&bar[s], (parity >> s) & 1u, ctl, nullptr, kStatusWaitDrain);
+        }
+        return;
+    }
+
+    // Per-tensor block maxima; then one thread per tensor draws that tensor's ticket.
+    if constexpr (kPersist) {
+        am0 = warp_max(am0);
+        am1 = warp_max(am1);
+        am2 = warp_max(am2);
+        if (lane == 0) {
+            s_red[0][w] = am0;
+            s_red[1][w] = am1;
+            s_red[2][w] = am2;
+        }
+    } else {
+        // one tile, one tensor: the other two maxima are zero
+        am0 = warp_max(fmaxf(am0, fmaxf(am1, am2)));
+        if (lane == 0) s_red[0][w] = am0;
+    }
+    __syncthreads();
+    // Persistent: every CTA finishes every tensor.  One tile per CTA: only its own tensor.
+    if (t < njobs && (kPersist || t == tile_job(batch, static_cast<int>(blockIdx.x)))) {
+        const int row = kPersist ? t : 0;
+        float m = s_red[row][0];
+#pragma unroll
+        for (int v = 1; v < kThreads / 32; ++v) m = fmaxf(m, s_red[row][v]);
+        const QArgs& a = batch.job[t];
+        const bool first = kPersist ? blockIdx.x == 0 : static_cast<int>(blockIdx.x) == a.tile_begin;
+        job_finish(a, m, __ldg(a.scale), first, s_hist[t]);
+    }
 }
 
 // ----------------------------------------------------------------------------------------
@@ -471,11 +673,59 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
 }
 
 template <int kFmt, class In>
-void launch_quant_kernel(const QBatch& b, bool tiled, dim3 grid, cudaStream_t stream) {
-    if (tiled)
-        launch_ex(quant_tiled_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
-    else
-        launch_ex(quant_flat_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+void launch_flat(const QBatch& b, dim3 grid, cudaStream_t stream) {
+    launch_ex(quant_flat_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+}
+
+// Batches of more tiles than this run persistent; smaller ones one tile per CTA.
+std::atomic<int64_t> g_persist_min_tiles{1024};
+int64_t persist_min_tiles() { return g_persist_min_tiles.load(); }
+
+// Tiled launch.  Persistent: grid = min(tiles, resident CTAs) and every CTA draws one ticket
+// per tensor, so each tensor's fold counts gridDim.x blocks.  One tile per CTA: grid = tiles,
+// inputs not read by TMA, and each tensor's fold counts that tensor's tiles.
+template <int kFmt, class In, bool kPersist>
+int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
+    using C = TiledCfg<In, kPersist>;
+    auto kernel = quant_tiled_kernel<In, kFmt, kPersist>;
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    static int per_sm = 0;
+    std::call_once(once, [kernel] {
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (err == cudaSuccess) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, C::kSmem);
+    });
+    if (err != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("tiled quantize set-up: ") + cudaGetErrorString(err));
+    int grid;
+    if (kPersist) {
+        const int64_t resident = static_cast<int64_t>(sm_count()) * std::max(1, per_sm);
+        grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(b.tiles_total, resident)));
+        for (int i = 0; i < b.njobs; ++i) b.job[i].nblocks = static_cast<unsigned>(grid);
+    } else {
+        grid = b.tiles_total;
+        for (int i = 0; i < b.njobs; ++i) {
+            const int end = i + 1 < b.njobs ? b.job[i + 1].tile_begin : b.tiles_total;
+            b.job[i].nblocks = static_cast<unsigned>(end - b.job[i].tile_begin);
+            b.job[i].tma = 0;
+        }
+    }
+    launch_ex(kernel, dim3(grid), dim3(kThreads), C::kSmem, stream, 1, b, ctl);
+    return FP8DSA_OK;
+}
+
+template <int kFmt, class In>
+int launch_quant(QBatch& b, bool tiled, dim3 grid, const WaitCtl& ctl, cudaStream_t stream) {
+    if (tiled) {
+        if (b.tiles_total > persist_min_tiles()) return launch_tiled<kFmt, In, true>(b, ctl, stream);
+        return launch_tiled<kFmt, In, false>(b, ctl, stream);
+    }
+    launch_flat<kFmt, In>(b, grid, stream);
+    return FP8DSA_OK;
+}
+
+CUtensorMapDataType map_type(fp8_in_t t) {
+    return t == FP8_IN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                           : (t == FP8_IN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 int check_ring(const fp8_ring_t* ring) {
@@ -492,7 +742,7 @@ int check_ring(const fp8_ring_t* ring) {
 
 }  // namespace
 
-int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream) {
+int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, uint32_t* zero, int64_t zero_words) {
     if (njobs < 1 || njobs > kMaxJobs) return fail(FP8DSA_ERR_INVALID_ARG, "quantize batch of 1..3 tensors");
     const fp8_fmt_t fmt = jobs[0].fmt;
     const fp8_in_t in_type = jobs[0].in_type;
@@ -502,6 +752,8 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream) 
             return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares format, input type and orientation");
     QBatch b{};
     b.njobs = njobs;
+    b.zero = zero;
+    b.zero_words = zero != nullptr ? zero_words : 0;
     const int eb = in_type_bytes(in_type);
     double bytes = 0.0;
     int64_t max_groups = 0;
@@ -540,23 +792,35 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream) 
                     (tiled ? ((reinterpret_cast<uintptr_t>(job.out) & 7) == 0 && job.cols % 8 == 0) : aligned16(job.out));
         a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
         if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
+        if (tiled && a.vec_in && job.rows > 0 && job.cols > 0 && job.rows < (int64_t(1) << 31) &&
+            job.cols < (int64_t(1) << 31)) {
+            // TMA needs a 16-byte aligned base and row stride (both implied by vec_in here)
+            const int64_t ld = job.cols * eb;
+            if (encode_tensor_map(&b.map[i], map_type(in_type), job.x, job.cols, job.rows, 1, ld, ld * job.rows,
+                                  kTile, kTile, CU_TENSOR_MAP_SWIZZLE_NONE) == FP8DSA_OK)
+                a.tma = 1;
+            else
+                clear_error();  // fall back to direct loads for this tensor
+        }
         bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0));
         if (tiled) {
-            // an empty tensor still gets one block, whose fold records amax 0
+            // an empty tensor still gets one (empty) tile
             const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);
             const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
             a.tiles_x = static_cast<int>(tx);
             a.tile_begin = static_cast<int>(tiles_total);
-            a.nblocks = static_cast<unsigned>(tx * ty);
             tiles_total += tx * ty;
+            if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
         } else {
             max_groups = std::max(max_groups, (a.numel + 15) / 16);
         }
     }
     dim3 grid;
+    WaitCtl ctl{};
     if (tiled) {
-        if (tiles_total > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "too many tiles");
-        grid = dim3(static_cast<unsigned>(tiles_total));
+        b.tiles_total = static_cast<int>(tiles_total);
+        const int rc = wait_ctl(&ctl);
+        if (rc) return rc;
     } else {
         const int64_t want = std::max<int64_t>(1, (max_groups + kThreads - 1) / kThreads);
         const int per_job = static_cast<int>(std::min<int64_t>(want, std::max<int64_t>(1, static_cast<int64_t>(sm_count()) * 8 / njobs)));
@@ -564,16 +828,18 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream) 
         grid = dim3(static_cast<unsigned>(per_job), static_cast<unsigned>(njobs));
     }
     launch_begin(kKindQuantize, stream);
+    int rc;
     if (fmt == FP8_E4M3) {
-        if (in_type == FP8_IN_BF16) launch_quant_kernel<0, Bf16In>(b, tiled, grid, stream);
-        else if (in_type == FP8_IN_F16) launch_quant_kernel<0, F16In>(b, tiled, grid, stream);
-        else launch_quant_kernel<0, F32In>(b, tiled, grid, stream);
+        if (in_type == FP8_IN_BF16) rc = launch_quant<0, Bf16In>(b, tiled, grid, ctl, stream);
+        else if (in_type == FP8_IN_F16) rc = launch_quant<0, F16In>(b, tiled, grid, ctl, stream);
+        else rc = launch_quant<0, F32In>(b, tiled, grid, ctl, stream);
     } else {
-        if (in_type == FP8_IN_BF16) launch_quant_kernel<1, Bf16In>(b, tiled, grid, stream);
-        else if (in_type == FP8_IN_F16) launch_quant_kernel<1, F16In>(b, tiled, grid, stream);
-        else launch_quant_kernel<1, F32In>(b, tiled, grid, stream);
+        if (in_type == FP8_IN_BF16) rc = launch_quant<1, Bf16In>(b, tiled, grid, ctl, stream);
+        else if (in_type == FP8_IN_F16) rc = launch_quant<1, F16In>(b, tiled, grid, ctl, stream);
+        else rc = launch_quant<1, F32In>(b, tiled, grid, ctl, stream);
     }
     launch_end(kKindQuantize, stream, bytes);
+    if (rc) return rc;
     return check_launch("fp8 quantize kernel");
 }
 
@@ -689,9 +955,9 @@ static int quantize_common(const void* x, fp8_in_t in_type, int64_t rows, int64_
     if (scale == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "scale is NULL");
     const bool empty = rows == 0 || cols == 0;
     if (!empty && out == nullptr && out_t == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "output is NULL");
-    if (out_t != nullptr && (cols + kTile - 1) / kTile > 0x7FFFFFFF)
+    if (out_t != nullptr && (cols + kTile - 1) / kTile > kMaxTiles)
         return fail(FP8DSA_ERR_UNSUPPORTED, "too many columns");
-    if (out_t != nullptr && ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile) > 0x7FFFFFFF)
+    if (out_t != nullptr && ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile) > kMaxTiles)
         return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
     int rc = check_ring(ring);
     if (rc) return rc;
@@ -718,6 +984,13 @@ int fp8_quantize(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, co
     if (out == nullptr && rows > 0 && cols > 0) return fail(FP8DSA_ERR_INVALID_ARG, "out is NULL");
     return quantize_common(x, in_type, rows, cols, scale, fmt, transposed ? nullptr : out,
                            transposed ? out : nullptr, amax_out, ring, stream);
+}
+
+int fp8_set_tiled_persist_threshold(int64_t min_tiles) {
+    clear_error();
+    if (min_tiles < 0) return fail(FP8DSA_ERR_INVALID_ARG, "min_tiles must be >= 0");
+    g_persist_min_tiles.store(min_tiles);
+    return FP8DSA_OK;
 }
 
 int fp8_quantize_dual(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,

@@ -1,6 +1,8 @@
 // Library runtime: thread-local error messages, device checks, the device status word that
 // bounded waits report into, the wait timeout, optional per-kernel CUDA-event timing, and
 // the stalled-wait test hook.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -132,6 +134,36 @@ void launch_end(int kind, cudaStream_t stream, double work) {
     t_pending_start = nullptr;
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+}  // namespace
+
+int encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner,
+                      int64_t outer, int64_t batch, int64_t ld, int64_t bstride, int box_inner, int box_outer,
+                      CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
+                                static_cast<cuuint64_t>(batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(bstride)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FP8DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+    return FP8DSA_OK;
+}
+
 int check_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
@@ -201,6 +233,11 @@ int fp8_debug_stalled_wait(cudaStream_t stream) {
     if (rc) return rc;
     stalled_wait_kernel<<<1, 32, 0, stream>>>(ctl);
     return check_launch("stalled_wait_kernel");
+}
+
+int fp8_set_gemm_split_k(int splits) {
+    clear_error();
+    return gemm_set_split_mode(splits);
 }
 
 int fp8_set_pdl(int enabled) {

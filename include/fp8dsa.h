@@ -134,7 +134,9 @@ int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_
              const float* scale_a, const float* scale_b, const void* bias,
              const float* bias_scale, void* out, cudaStream_t stream);
 
-/* Workspace bytes linear_forward_fp8 needs for (m, k, n) (x8, w8 and scale scratch). */
+/* Workspace bytes linear_forward_fp8 needs for (m, k, n): x8, w8 and scale scratch, then the
+ * GEMM's split-K region (arrival counters and fp32 partial tiles for up to 4 K ranges per
+ * output tile; used only where splitting shortens the schedule). */
 size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
 
 /* FP8 linear forward y = x w^T + bias [compare: astrai/extension/fp8.py, fp8_linear_forward]:
@@ -148,8 +150,12 @@ size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
  *      w first (max(amax / fp8_max / pow2_margin, 1e-12)), with fp8_max of `fmt` and
  *      pow2_margin given here.
  *   sx_used, sw_used: dev fp32 outputs, the steps the GEMM used (the backward's sx / sw).
- *   workspace: dev, >= linear_forward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned.
- *   y: dev bf16 [m][n].  k and n must be multiples of 16. */
+ *   workspace: dev, >= linear_forward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned;
+ *      no initial contents are needed (the quantize launch clears the split-K counters).
+ *   y: dev bf16 [m][n].  k and n must be multiples of 16.
+ *   Where the GEMM cuts an output tile's K range across CTAs (split-K), the owner CTA adds
+ *   the other ranges' fp32 partial sums in a fixed order: results are deterministic and
+ *   differ from the unsplit GEMM only in fp32 summation order. */
 int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* w_step,
                        const void* bias, const float* bias_scale, int64_t m, int64_t k, int64_t n,
                        fp8_fmt_t fmt, const fp8_ring_t* x_ring, const fp8_ring_t* w_ring,
@@ -165,8 +171,9 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
  * footprint.  The pages have no counterpart to this entry point.
  * Same arguments and results as linear_forward_fp8, without the workspace: the scratch lives
  * in one built-in device array of FP8DSA_NOALLOC_WORKSPACE_BYTES (16 MiB), held by every GPU
- * that loads the library until the process exits.  Shapes whose
- * linear_forward_fp8_workspace_size exceeds it return FP8DSA_ERR_WORKSPACE with a message.
+ * that loads the library until the process exits.  The array holds the x8 / w8 operand
+ * buffers and the scale scratch (about m*k + n*k bytes), and the GEMM here never splits K;
+ * shapes whose buffers exceed the array return FP8DSA_ERR_WORKSPACE with a message.
  * The first call on each device looks up the array's address (make it before any stream
  * capture); no call allocates.  All calls share the array: calls ordered on one stream are
  * safe, calls that overlap on the GPU race. */
@@ -176,7 +183,8 @@ int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is_fp8, const
                                const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                                float* sw_used, void* y, cudaStream_t stream);
 
-/* Workspace bytes linear_backward_fp8 needs for (m, k, n). */
+/* Workspace bytes linear_backward_fp8 needs for (m, k, n): g8, g8T, x8T, w8T, the per-tile
+ * column sums and scale scratch, then the dX / dW GEMM's split-K region. */
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
 
 /* FP8 linear backward [compare: astrai/extension/fp8.py, _LinearFp8.backward]:
@@ -192,7 +200,8 @@ size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
  *   pow2_margin, and sx_fwd / sw_fwd are ignored.
  *   need_grad_x / need_grad_w / need_grad_b select the outputs (the others may be NULL).
  *   sg_used: dev fp32 output (the step g was quantized with), may be NULL.
- *   workspace: dev, >= linear_backward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned.
+ *   workspace: dev, >= linear_backward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned;
+ *      no initial contents are needed.  The dX / dW GEMM may split K as in the forward.
  *   k and n must be multiples of 16; m a multiple of 16 when grad_w is needed. */
 int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, int64_t k,
                         int64_t n, fp8_fmt_t fmt, int need_grad_x, int need_grad_w,
@@ -215,6 +224,23 @@ int fp8_set_wait_timeout_ns(uint64_t ns);
  * waits for that kernel's results before reading them.  0 launches them plainly.  Applies to
  * launches after the call (and to stream captures made after it).  Not on the pages. */
 int fp8_set_pdl(int enabled);
+
+/* Split-K in the linear compositions' GEMMs: an output tile's K range may be cut across CTAs
+ * (up to 4 ranges; contributors leave fp32 partials in the workspace, the owner adds them in a
+ * fixed order).  1 (default) never splits -- measured on B200, the extra epilogue work of the
+ * partials outweighs the shorter MMA schedule on this library's workloads; 0 splits where a
+ * model of the schedule says the launch finishes sooner; 2..4 force that many ranges per tile
+ * wherever the workspace holds the partials and every range keeps at least 256 bytes of K.
+ * Other values: FP8DSA_ERR_INVALID_ARG.  Applies to later launches (and stream captures made
+ * after the call).  Not on the pages. */
+int fp8_set_gemm_split_k(int splits);
+
+/* Transposed / dual quantize launches covering more than `min_tiles` 128 x 128 tiles (over all
+ * tensors of the launch) run on the persistent TMA-fed kernel; smaller ones run one tile per
+ * CTA.  Both give identical bytes, amax and ring updates; the choice only moves time.  Default
+ * 1024; min_tiles < 0 is rejected (FP8DSA_ERR_INVALID_ARG).  Applies to later launches.  Not
+ * on the pages. */
+int fp8_set_tiled_persist_threshold(int64_t min_tiles);
 
 /* Test hook for the failure path: launches one block that waits on a barrier nothing ever
  * arrives at; the wait gives up after the timeout and sets the device status word.

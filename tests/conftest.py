@@ -30,3 +30,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=["tile_per_cta", "persistent"])
+def tiled_path(request):
+    """Run the transposed / dual quantize on each of its two kernels: one tile per CTA, or
+    the persistent TMA-fed kernel (forced by a zero tile threshold)."""
+    import fp8_delayed_scaling_amax_b200 as F
+    F.fp8_set_tiled_persist_threshold(0 if request.param == "persistent" else 1 << 40)
+    yield request.param
+    F.fp8_set_tiled_persist_threshold(1024)

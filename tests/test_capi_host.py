@@ -117,6 +117,12 @@ def test_misc_argument_checks():
     assert lib.fp8_scale_ring_init(256, 0, None) == INVALID
     assert lib.fp8_amax_scale(256, 0, 16, 448.0, 1.0, None, None, 256, None) == INVALID
     assert lib.fp8_get_device_status(None, None) == INVALID
+    assert lib.fp8_set_tiled_persist_threshold(-1) == INVALID
+    assert lib.fp8_set_tiled_persist_threshold(1024) == 0
+    assert lib.fp8_set_gemm_split_k(-1) == INVALID
+    assert lib.fp8_set_gemm_split_k(5) == INVALID
+    assert lib.fp8_set_gemm_split_k(0) == 0
+    assert lib.fp8_set_gemm_split_k(1) == 0
     ring = F.Ring(None, 4)
     for _ in range(5):
         ring.advance()

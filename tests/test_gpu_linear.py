@@ -113,7 +113,7 @@ def test_delayed_ring_forward_eight_steps():
 
 
 @pytest.mark.parametrize("kn", W.TRAINING_LINEARS)
-def test_training_linear_delayed_hybrid(kn):
+def test_training_linear_delayed_hybrid(kn, tiled_path):
     k, n = kn
     m = W.TRAINING_TOKENS
     xr, wr = _ring(16, F.FP8_E4M3), _ring(16, F.FP8_E4M3)

@@ -62,7 +62,7 @@ def _quantize(x, in_type, s, fmt, mode, ring=None, amax=True):
 @pytest.mark.parametrize("fmt,fname", FMTS)
 @pytest.mark.parametrize("in_type,dtype", IN_TYPES)
 @pytest.mark.parametrize("mode", ["row", "t", "dual"])
-def test_quantize_bit_exact(fmt, fname, in_type, dtype, mode):
+def test_quantize_bit_exact(fmt, fname, in_type, dtype, mode, tiled_path):
     for i, shape in enumerate(SHAPES):
         x = _input(shape, dtype, seed=i + 10 * fmt)
         s = [1.0, 0.0173, 3.3e-3, 17.25][i % 4]
@@ -78,7 +78,7 @@ def test_quantize_bit_exact(fmt, fname, in_type, dtype, mode):
 
 
 @pytest.mark.parametrize("mode", ["row", "t", "dual"])
-def test_quantize_misaligned_and_strided_bases(mode):
+def test_quantize_misaligned_and_strided_bases(mode, tiled_path):
     """A base pointer off the 16-byte grid takes the element path; results are identical."""
     big = _input((129 * 77 + 1,), torch.bfloat16, seed=3).to(DEV)
     x = big[1:].view(129, 77)
@@ -91,6 +91,40 @@ def test_quantize_misaligned_and_strided_bases(mode):
     if out_t is not None:
         assert np.array_equal(np_u8(out_t), want.T)
     assert a.item() == Q.amax(xv)
+
+
+@pytest.mark.parametrize("in_type,dtype", IN_TYPES)
+@pytest.mark.parametrize("mode", ["row", "t", "dual"])
+def test_quantize_special_values(in_type, dtype, mode, tiled_path):
+    """NaN, +-inf, subnormals and signed zeros in 16-bit and 32-bit inputs, on the vector and
+    tiled paths: amax ignores NaN and is inf when an inf is present; inf saturates; every
+    non-NaN byte equals the oracle's; a NaN's byte is a NaN code (0x7F with either sign)."""
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn((256, 384), generator=g)
+    tiny = {torch.bfloat16: 3e-39, torch.float16: 3e-6, torch.float32: 1e-41}[dtype]
+    flat = x.view(-1)
+    flat[5::97] = float("nan")
+    flat[11::301] = tiny
+    flat[12::301] = -tiny
+    flat[13::211] = -0.0
+    for case in ("nan_only", "with_inf"):
+        xc = x.clone()
+        if case == "with_inf":
+            xc.view(-1)[7] = float("inf")
+            xc.view(-1)[9000] = float("-inf")
+        xd = xc.to(dtype)
+        out, out_t, a = _quantize(xd.to(DEV), in_type, 0.0173, F.FP8_E4M3, mode)
+        torch.cuda.synchronize()
+        xv = in_values_f32(xd)
+        want = Q.quantize_values(xv, 0.0173, "e4m3")
+        nan = np.isnan(xv)
+        for got, ref, mask in ((out, want, nan), (out_t, want.T, nan.T)):
+            if got is None:
+                continue
+            b = np_u8(got)
+            assert np.array_equal(b[~mask], ref[~mask]), (case, mode)
+            assert ((b[mask] & 0x7F) == 0x7F).all(), (case, mode)
+        assert a.item() == Q.amax(xv), (case, mode)
 
 
 def test_quantize_empty_and_nan():
@@ -152,7 +186,7 @@ def test_delayed_ring_sequence_bit_exact():
 
 
 @pytest.mark.parametrize("mode", ["row", "t", "dual"])
-def test_ring_fold_every_mode_and_margin(mode):
+def test_ring_fold_every_mode_and_margin(mode, tiled_path):
     ring = _ring(4, F.FP8_E5M2, margin=2)
     oring = S.Ring(4, "e5m2", margin=2)
     for t in range(6):

@@ -4,8 +4,8 @@ It serves callers that cannot allocate device memory when they run the forward p
 example inside a CUDA stream capture, or a plug-in whose host owns the memory budget): its
 scratch is one built-in 16 MiB device array instead of a caller workspace.  Here it is
 called through the C ABI twice in a row and its output is compared with the workspace
-entry point's, within the GEMM bound the other tests use.  This file is named so pytest
-collects it last.
+entry point's (run with the same unsplit GEMM schedule): within the GEMM bound the other
+tests use, and bit for bit.  This file is named so pytest collects it last.
 """
 
 import numpy as np
@@ -46,8 +46,17 @@ def _forward_both(t, delayed, rings):
     return y_ws, y_na, s_ws, s_na
 
 
+@pytest.fixture
+def unsplit_gemm():
+    """The no-alloc entry never splits the GEMM's K; with splitting also off in the workspace
+    entry both run the same kernels, so their outputs must agree bit for bit."""
+    F.fp8_set_gemm_split_k(1)
+    yield
+    F.fp8_set_gemm_split_k(1)  # the library default
+
+
 @pytest.mark.parametrize("delayed", [False, True])
-def test_noalloc_forward_matches_workspace_forward_twice(delayed):
+def test_noalloc_forward_matches_workspace_forward_twice(delayed, unsplit_gemm):
     rings = [(_ring(F.FP8_E4M3), _ring(F.FP8_E4M3)) for _ in range(2)]
     for call in range(2):
         t = W.training_linear(384, 512, 640, seed=500 + call)
@@ -61,6 +70,7 @@ def test_noalloc_forward_matches_workspace_forward_twice(delayed):
         # the two entry points against each other, with the bound the GEMM tests use
         assert_within_gemm_bound(bf16_out_to_f64(y_na), bf16_out_to_f64(y_ws), f["s_abs"], f["sc"],
                                  f"no-alloc vs workspace, call {call}")
+        assert torch.equal(y_na.view(torch.int16), y_ws.view(torch.int16)), f"call {call}"
         if delayed:
             assert torch.equal(rings[0][0].state, rings[1][0].state)
             assert torch.equal(rings[0][1].state, rings[1][1].state)
