@@ -16,8 +16,16 @@ What the pages fix (AstrAI compare view, ``astrai/extension/fp8.py``):
 * ``FP8Format.HYBRID``: E4M3 forward, E5M2 backward; the backward GEMM takes both
   operands in one format, so x and w are re-quantized to E5M2 as well.
 
+* Reuse of the forward's operands (the C++ binding of the linear backward in an
+  earlier state of the compare view): x or w already quantized by the forward is
+  passed as fp8 and its quantize kernel is skipped; its forward step still
+  dequantizes the GEMM.  There the reused bytes had to share the backward's
+  format.
+
 Readings: ``grad_b`` is the fp64 column sum rounded once to bf16; the gradient
-outputs are returned unrounded (fp64) for the bound check.
+outputs are returned unrounded (fp64) for the bound check.  ``backward_mixed``
+reads the operand reuse with independent formats (the tensor core takes A and B
+formats separately): the forward's E4M3 x8 / w8 with an E5M2 g8.
 """
 
 from __future__ import annotations
@@ -80,3 +88,33 @@ def backward(g_bits, x_bits, w_bits, fmt="e5m2", sx_fwd=None, sw_fwd=None,
     return dict(dx=dx, dx_abs=dx_abs, dx_sc=dx_sc, dw=dw, dw_abs=dw_abs, dw_sc=dw_sc,
                 grad_b=grad_b, g8=g8, g8t=g8t, x8t=x8t, w8t=w8t, sg=sg, sx=sx, sw=sw,
                 amax_g=ag)
+
+
+def backward_mixed(g_bits, x8, w8, fmt_g="e5m2", fmt_x="e4m3", fmt_w="e4m3", sx=None,
+                   sw=None, ring_g: Ring = None, margin: int = 0):
+    """Backward that reuses the forward's quantized operands as they are.
+
+    ``x8`` [m,k] and ``w8`` [n,k] are the forward's fp8 codes (formats ``fmt_x`` /
+    ``fmt_w``, steps ``sx`` / ``sw``).  Only g is quantized, row-major, in ``fmt_g``
+    (with ``ring_g``: the ring's step, folded; without: the dynamic step).  Then
+
+    * ``grad_x [m,k] = g8 @ w8 * RN32(sg*sw)``   (layout NN: B = w8 stored [n,k] = [K,N])
+    * ``grad_w [n,k] = g8^T @ x8 * RN32(sg*sx)`` (layout TN: A = g8 stored [m,n] = [K,M],
+      B = x8 stored [m,k] = [K,N])
+    * ``grad_b`` as in :func:`backward`.
+
+    Returns the same keys as :func:`backward` except the re-quantized x8T / w8T."""
+    gv = bf16_bits_to_f64(g_bits).astype(np.float32)
+    if ring_g is None:
+        sg = dynamic_scale(gv, fmt_g, margin)
+    else:
+        sg = np.float32(ring_g.scale)
+    g8, ag = quantize(gv, sg, fmt_g)
+    if ring_g is not None:
+        ring_g.fold(ag, sg)
+    sx, sw = np.float32(sx), np.float32(sw)
+    dx, dx_abs, dx_sc = gemm_ref(g8, w8, "NN", fmt_g, fmt_w, sg, sw)
+    dw, dw_abs, dw_sc = gemm_ref(g8, x8, "TN", fmt_g, fmt_x, sg, sx)
+    grad_b = round_to_bf16(np.sum(gv.astype(np.float64), axis=0))
+    return dict(dx=dx, dx_abs=dx_abs, dx_sc=dx_sc, dw=dw, dw_abs=dw_abs, dw_sc=dw_sc,
+                grad_b=grad_b, g8=g8, sg=sg, sx=sx, sw=sw, amax_g=ag)

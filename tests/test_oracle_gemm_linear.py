@@ -204,3 +204,50 @@ def test_delayed_linear_sequence_and_backward_reuses_forward_steps():
         assert bwd["sx"] == fwd["sx"] and bwd["sw"] == fwd["sw"]
         for r in (rx, rw, rg):
             r.advance()
+
+
+def test_backward_mixed_equals_exact_brute_force():
+    """E5M2 g8 times the forward's E4M3 bytes: grad_x = g8 @ w8 and grad_w = g8^T @ x8, each
+    scaled by RN32(sg * s_operand), against the exact rational triple loop.  The operands are
+    transposed here with numpy, not through the oracle's layout handling."""
+    rng = np.random.default_rng(31)
+    for m, k, n in ((2, 3, 4), (5, 7, 3), (16, 8, 12)):
+        g = _bits(rng.standard_normal((m, n)) * 1e-3)
+        x8 = _rand_codes(rng, (m, k), "e4m3")
+        w8 = _rand_codes(rng, (n, k), "e4m3")
+        sx, sw = np.float32(0.0625), np.float32(1.5e-4)
+        out = L.backward_mixed(g, x8, w8, "e5m2", "e4m3", "e4m3", sx, sw)
+        g8 = out["g8"]
+        exact_dx = _brute(g8, w8, "e5m2", "e4m3", out["sg"], sw, None)
+        exact_dw = _brute(np.ascontiguousarray(g8.T), x8, "e5m2", "e4m3", out["sg"], sx, None)
+        for ref, abs_, sc, exact in ((out["dx"], out["dx_abs"], out["dx_sc"], exact_dx),
+                                     (out["dw"], out["dw_abs"], out["dw_sc"], exact_dw)):
+            for i in range(ref.shape[0]):
+                for j in range(ref.shape[1]):
+                    tol = Fraction(2) ** -45 * Fraction(float(abs_[i, j])) * Fraction(float(sc))
+                    assert abs(Fraction(ref[i, j]) - exact[i, j]) <= tol
+
+
+def test_backward_mixed_with_one_format_is_the_backward():
+    """With every operand in the backward's format and x8 / w8 quantized at the forward's
+    steps, reusing the bytes gives exactly the backward that re-quantizes x and w
+    transposed: same g8, step, ring fold, grad_x, grad_w and grad_b."""
+    rng = np.random.default_rng(6)
+    m, k, n = 48, 32, 40
+    g = _bits(rng.standard_normal((m, n)) * 1e-3)
+    x = _bits(rng.standard_normal((m, k)))
+    w = _bits(rng.standard_normal((n, k)) * 0.02)
+    sx, sw = np.float32(3.0e-3), np.float32(1.1e-4)
+    x8, _ = Q.quantize(C.bf16_bits_to_f64(x).astype(np.float32), sx, "e5m2")
+    w8, _ = Q.quantize(C.bf16_bits_to_f64(w).astype(np.float32), sw, "e5m2")
+    r1, r2 = S.Ring(4, "e5m2"), S.Ring(4, "e5m2")
+    gv = C.bf16_bits_to_f64(g).astype(np.float32)
+    r1.seed(gv)
+    r2.seed(gv)
+    ref = L.backward(g, x, w, "e5m2", sx, sw, r1)
+    mix = L.backward_mixed(g, x8, w8, "e5m2", "e5m2", "e5m2", sx, sw, r2)
+    assert np.array_equal(ref["g8"], mix["g8"]) and ref["sg"] == mix["sg"]
+    assert np.array_equal(r1.state.view(np.uint32), r2.state.view(np.uint32))
+    for key in ("dx", "dw", "dx_abs", "dw_abs"):
+        assert np.array_equal(ref[key], mix[key]), key
+    assert np.array_equal(ref["grad_b"], mix["grad_b"])
