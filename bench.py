@@ -53,6 +53,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sweeps", action="store_true")
+    p.add_argument("--no-variants", action="store_true", help="skip the mixed-format backward variant")
     p.add_argument("--kernel", default=None, choices=["gemm", "quantize"],
                    help="time one kernel on one shape instead of the step (small cases for ncu)")
     p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS")
@@ -188,6 +189,32 @@ class Linear:
                               self.steps[0:1], self.steps[1:2], self.rg, 1.0, self.steps[2:3], self.bws,
                               self.bws_n, self.gx, self.gw, self.gb)
 
+    def fwd_keep(self):
+        """Forward that keeps x8 / w8 for the mixed-format backward."""
+        F = self.F
+        if not hasattr(self, "x8k"):
+            import torch
+            self.x8k = torch.empty((self.m, self.k), dtype=torch.uint8, device=self.x.device)
+            self.w8k = torch.empty((self.n, self.k), dtype=torch.uint8, device=self.x.device)
+            self.mws_n = F.linear_backward_fp8_mixed_workspace_size(self.m, self.k, self.n)
+            self.mws = torch.empty(self.mws_n, dtype=torch.uint8, device=self.x.device)
+        F.linear_forward_fp8_keep(self.x, self.w, 0, None, self.b, None, self.m, self.k, self.n, F.FP8_E4M3, self.rx,
+                                  self.rw, 1.0, self.steps[0:1], self.steps[1:2], self.x8k, self.w8k, self.fws,
+                                  self.fws_n, self.y)
+
+    def bwd_mixed(self):
+        """Backward that quantizes only g (E5M2) and reuses the forward's E4M3 x8 / w8."""
+        F = self.F
+        F.linear_backward_fp8_mixed(self.g, self.x8k, self.w8k, self.m, self.k, self.n, F.FP8_E5M2, F.FP8_E4M3,
+                                    F.FP8_E4M3, 1, 1, 1, self.steps[0:1], self.steps[1:2], self.rg, 1.0,
+                                    self.steps[2:3], self.mws, self.mws_n, self.gx, self.gw, self.gb)
+
+    @property
+    def quant_bytes_mixed(self):
+        m, k, n = self.m, self.k, self.n
+        # fwd: x, w row-major (2 B in, 1 B out); bwd: g row-major (2 B in, 1 B out)
+        return 3 * (m * k + n * k) + 3 * m * n
+
     @property
     def gemm_flops(self):
         return 3 * 2.0 * self.m * self.k * self.n
@@ -207,13 +234,15 @@ def build_workload(F, W, torch, dev, seed_base):
     return lins
 
 
-def run_step(lins, slot):
+def run_step(lins, slot, mixed=False):
+    """One training step: every linear's forward, then every backward in reverse order.
+    mixed=True: the forward keeps x8 / w8 and the backward reuses them (E5M2 g only)."""
     for lin in lins:
         lin.set_slot(slot)
     for lin in lins:
-        lin.fwd()
+        lin.fwd_keep() if mixed else lin.fwd()
     for lin in reversed(lins):
-        lin.bwd()
+        lin.bwd_mixed() if mixed else lin.bwd()
 
 
 # ---------------------------------------------------------------------------------------
@@ -504,6 +533,46 @@ def main():
     ms_max = float(ms_t.item())
     status = F.fp8_get_device_status()
 
+    # the mixed-format variant of the step (forward keeps x8 / w8, backward quantizes only g):
+    # its own graphs, warm-up and timed replays, reported beside the headline step
+    mixed = None
+    if not args.no_variants:
+        run_step(lins, counter[0] % HIST, mixed=True)
+        counter[0] += 1
+        torch.cuda.synchronize()
+        mgraphs = []
+        for slot in range(HIST):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                run_step(lins, slot, mixed=True)
+            mgraphs.append(g)
+        torch.cuda.synchronize()
+        for t in range(args.warmup):
+            mgraphs[counter[0] % HIST].replay()
+            counter[0] += 1
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        msteps = max(3, args.steps // 2)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for t in range(msteps):
+            mgraphs[counter[0] % HIST].replay()
+            counter[0] += 1
+        s1.record()
+        torch.cuda.synchronize()
+        mt = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(mt, op=dist.ReduceOp.MAX)
+        mms = float(mt.item())
+        mixed = {"ms_per_step": mms / msteps, "value": flops_step * msteps * world / (mms * 1e-3) / 1e12,
+                 "unit": UNIT, "steps": msteps,
+                 "quantize_bytes_per_step": sum(l.quant_bytes_mixed for l in lins),
+                 "device_status": F.fp8_get_device_status(),
+                 "what": "forward keeps its E4M3 x8 / w8; backward quantizes only g (E5M2, row-major + column "
+                         "sums) and reads x8 / w8 in place (mixed-format GEMMs); not the pages' HYBRID numerics"}
+        del mgraphs
+
     # per-kernel durations: the same step captured again with the library's profiler on
     # (an event-record node on each side of every kernel), each of the 16 slot graphs
     # replayed once, then every event pair read back
@@ -599,6 +668,8 @@ def main():
     }
     if clocks:
         line["clocks"] = clocks
+    if mixed is not None:
+        line["variants"] = {"mixed_backward": mixed}
     if e2e:
         line["e2e"] = e2e
     if world == 1 and not args.no_sweeps:

@@ -53,6 +53,13 @@ _SIGNATURES = {
     "linear_backward_fp8_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_backward_fp8": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, _P, _P,
                                     POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P, _P]),
+    "linear_forward_fp8_keep": (c_int, [_P, _P, c_int, _P, _P, _P, c_int64, c_int64, c_int64, c_int,
+                                        POINTER(fp8_ring_t), POINTER(fp8_ring_t), c_float, _P, _P, _P, _P, _P,
+                                        c_size_t, _P, _P]),
+    "linear_backward_fp8_mixed_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
+    "linear_backward_fp8_mixed": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int,
+                                          c_int, _P, _P, POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P,
+                                          _P]),
     "fp8_get_device_status": (c_int, [_P, POINTER(c_int)]),
     "fp8_set_wait_timeout_ns": (c_int, [c_uint64]),
     "fp8_debug_stalled_wait": (c_int, [_P]),
@@ -223,6 +230,30 @@ def linear_backward_fp8(g, x, w, m, k, n, fmt, need_grad_x, need_grad_w, need_gr
         _ptr(g), _ptr(x), _ptr(w), int(m), int(k), int(n), int(fmt), int(bool(need_grad_x)), int(bool(need_grad_w)),
         int(bool(need_grad_b)), _ptr(sx_fwd), _ptr(sw_fwd), _ring(g_ring), float(pow2_margin), _ptr(sg_used),
         _ptr(workspace), int(workspace_bytes), _ptr(grad_x), _ptr(grad_w), _ptr(grad_b), _stream(stream)))
+
+
+def linear_forward_fp8_keep(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
+                            sx_used, sw_used, x8_out, w8_out, workspace, workspace_bytes, y, stream=None):
+    """linear_forward_fp8 that also leaves the quantized operands in x8_out / w8_out (for
+    linear_backward_fp8_mixed)."""
+    return _check("linear_forward_fp8_keep", lib().linear_forward_fp8_keep(
+        _ptr(x), _ptr(w), int(bool(w_is_fp8)), _ptr(w_step), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n),
+        int(fmt), _ring(x_ring), _ring(w_ring), float(pow2_margin), _ptr(sx_used), _ptr(sw_used), _ptr(x8_out),
+        _ptr(w8_out), _ptr(workspace), int(workspace_bytes), _ptr(y), _stream(stream)))
+
+
+def linear_backward_fp8_mixed_workspace_size(m, k, n) -> int:
+    return int(lib().linear_backward_fp8_mixed_workspace_size(int(m), int(k), int(n)))
+
+
+def linear_backward_fp8_mixed(g, x8, w8, m, k, n, fmt_g, fmt_x, fmt_w, need_grad_x, need_grad_w, need_grad_b, sx,
+                              sw, g_ring, pow2_margin, sg_used, workspace, workspace_bytes, grad_x, grad_w, grad_b,
+                              stream=None):
+    return _check("linear_backward_fp8_mixed", lib().linear_backward_fp8_mixed(
+        _ptr(g), _ptr(x8), _ptr(w8), int(m), int(k), int(n), int(fmt_g), int(fmt_x), int(fmt_w),
+        int(bool(need_grad_x)), int(bool(need_grad_w)), int(bool(need_grad_b)), _ptr(sx), _ptr(sw), _ring(g_ring),
+        float(pow2_margin), _ptr(sg_used), _ptr(workspace), int(workspace_bytes), _ptr(grad_x), _ptr(grad_w),
+        _ptr(grad_b), _stream(stream)))
 
 
 def fp8_get_device_status(stream=None) -> int:

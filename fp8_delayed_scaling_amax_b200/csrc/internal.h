@@ -175,13 +175,14 @@ int gemm_set_split_mode(int mode);
 // Workspace bytes of linear_forward_fp8 without the optional split-K region.
 size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n);
 
-// linear_forward_fp8 with a choice: allow_split = false needs only the base workspace and
+// linear_forward_fp8 with choices: x8_keep / w8_keep (may be null) receive the quantized
+// operands instead of the workspace; allow_split = false needs only the base workspace and
 // runs the GEMM without split-K.
 int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
                         const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
                         const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
-                        float* sw_used, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
-                        cudaStream_t stream);
+                        float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, void* workspace,
+                        size_t workspace_bytes, bool allow_split, void* y, cudaStream_t stream);
 
 // The GEMM entry with arguments already validated (used by the linear compositions).
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn_major,

@@ -85,6 +85,31 @@ BwdLayout bwd_layout(int64_t m, int64_t k, int64_t n) {
     return L;
 }
 
+struct MixLayout {
+    size_t g8, colsum, scratch, base, counters, partial, total;
+    int64_t counter_words;
+};
+
+MixLayout mix_layout(int64_t m, int64_t k, int64_t n) {
+    MixLayout L;
+    size_t off = 0;
+    L.g8 = off;
+    off = align_up(off + static_cast<size_t>(m) * n, kAlign);
+    L.colsum = off;
+    off = align_up(off + sizeof(float) * static_cast<size_t>((m + 127) / 128) * n, kAlign);
+    L.scratch = off;
+    off = align_up(off + kScratchBytes, kAlign);
+    L.base = off;
+    const int64_t om[2] = {m, n}, on[2] = {k, k};  // grad_x [m][k], grad_w [n][k]
+    L.counter_words = splitk_counter_words(om, on, 2);
+    L.counters = off;
+    off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(L.counter_words), kAlign);
+    L.partial = off;
+    off = align_up(off + splitk_partial_bytes(om, on, 2), kAlign);
+    L.total = off;
+    return L;
+}
+
 int check_ring_arg(const fp8_ring_t* r, const char* name) {
     if (r == nullptr) return FP8DSA_OK;
     if (r->state == nullptr || r->hist_len < 1 || r->hist_idx < 0 || r->hist_idx >= r->hist_len ||
@@ -111,7 +136,19 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
                        const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                        float* sw_used, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
     return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
-                               sx_used, sw_used, workspace, workspace_bytes, true, y, stream);
+                               sx_used, sw_used, nullptr, nullptr, workspace, workspace_bytes, true, y, stream);
+}
+
+int linear_forward_fp8_keep(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
+                            const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                            const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                            float* sw_used, uint8_t* x8_out, uint8_t* w8_out, void* workspace,
+                            size_t workspace_bytes, void* y, cudaStream_t stream) {
+    clear_error();
+    if ((x8_out == nullptr && m > 0 && k > 0) || (!w_is_fp8 && w8_out == nullptr && n > 0 && k > 0))
+        return fail(FP8DSA_ERR_INVALID_ARG, "x8_out (and w8_out unless w_is_fp8) are required");
+    return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
+                               sx_used, sw_used, x8_out, w8_out, workspace, workspace_bytes, true, y, stream);
 }
 
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
@@ -131,8 +168,8 @@ size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n) {
 int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
                         const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
                         const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
-                        float* sw_used, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
-                        cudaStream_t stream) {
+                        float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, void* workspace,
+                        size_t workspace_bytes, bool allow_split, void* y, cudaStream_t stream) {
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
@@ -156,12 +193,14 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     if (workspace_bytes < need)
         return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) + " bytes");
     if (w_is_fp8 && !aligned16(w)) return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 w must be 16-byte aligned");
+    if ((x8_keep != nullptr && !aligned16(x8_keep)) || (!w_is_fp8 && w8_keep != nullptr && !aligned16(w8_keep)))
+        return fail(FP8DSA_ERR_UNSUPPORTED, "x8_out / w8_out must be 16-byte aligned");
     rc = check_device();
     if (rc) return rc;
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    uint8_t* x8 = ws + L.x8;
-    uint8_t* w8 = w_is_fp8 ? static_cast<uint8_t*>(const_cast<void*>(w)) : ws + L.w8;
+    uint8_t* x8 = x8_keep != nullptr ? x8_keep : ws + L.x8;
+    uint8_t* w8 = w_is_fp8 ? static_cast<uint8_t*>(const_cast<void*>(w)) : (w8_keep != nullptr ? w8_keep : ws + L.w8);
     uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
     float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
     float* sx = sx_used ? sx_used : internal;
@@ -379,6 +418,95 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
                            need_grad_b ? grad_b : nullptr, &split, stream);
     if (rc) return rc;
     return FP8DSA_OK;
+}
+
+size_t linear_backward_fp8_mixed_workspace_size(int64_t m, int64_t k, int64_t n) {
+    if (m < 0 || k < 0 || n < 0) return 0;
+    return mix_layout(m, k, n).total;
+}
+
+int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w8, int64_t m, int64_t k, int64_t n,
+                              fp8_fmt_t fmt_g, fp8_fmt_t fmt_x, fp8_fmt_t fmt_w, int need_grad_x, int need_grad_w,
+                              int need_grad_b, const float* sx, const float* sw, const fp8_ring_t* g_ring,
+                              float pow2_margin, float* sg_used, void* workspace, size_t workspace_bytes,
+                              void* grad_x, void* grad_w, void* grad_b, cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt_g) || !valid_fmt(fmt_x) || !valid_fmt(fmt_w))
+        return fail(FP8DSA_ERR_INVALID_ARG, "formats must be FP8_E4M3 or FP8_E5M2");
+    if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (w8 == nullptr || sw == nullptr || grad_x == nullptr))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w8, sw and grad_x");
+    if (need_grad_w && (x8 == nullptr || sx == nullptr || grad_w == nullptr))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x8, sx and grad_w");
+    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
+    if ((need_grad_w && !aligned16(x8)) || (need_grad_x && !aligned16(w8)))
+        return fail(FP8DSA_ERR_UNSUPPORTED, "x8 and w8 must be 16-byte aligned");
+    const bool dynamic = g_ring == nullptr;
+    if (dynamic && !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "pow2_margin must be > 0");
+    int rc = check_ring_arg(g_ring, "g_ring");
+    if (rc) return rc;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    const MixLayout L = mix_layout(m, k, n);
+    if (workspace_bytes < L.total)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    rc = check_device();
+    if (rc) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* g8 = ws + L.g8;
+    float* colsum = reinterpret_cast<float*>(ws + L.colsum);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
+    float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
+    float* sg = sg_used ? sg_used : internal;
+
+    if (dynamic) {
+        cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset scratch: ") + cudaGetErrorString(e));
+        AmaxJob job;
+        job.x = g;
+        job.numel = m * n;
+        job.fp8_max = fmt_max(fmt_g);
+        job.pow2_margin = pow2_margin;
+        job.scale_out = sg;
+        rc = launch_amax_jobs(&job, 1, scratch, stream);
+        if (rc) return rc;
+    }
+    // g only: row-major bytes, its ring fold and (for grad_b) the per-tile column sums
+    QuantJob qg;
+    qg.x = g;
+    qg.rows = m;
+    qg.cols = n;
+    qg.fmt = fmt_g;
+    qg.out = g8;
+    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    if (dynamic) {
+        qg.scale = sg;
+    } else {
+        qg.scale = g_ring->state + g_ring->hist_len;
+        qg.ring = g_ring;
+        qg.scale_used_out = sg;
+    }
+    SplitWorkspace split;
+    split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+    split.counter_words = L.counter_words;
+    split.partial = reinterpret_cast<float*>(ws + L.partial);
+    split.partial_bytes = L.total - L.partial;
+    rc = launch_quantize_batch(&qg, 1, stream, split.counters, split.counter_words);
+    if (rc) return rc;
+    // the forward's bytes are read in place: w8 [n][k] is B = [K][N] of grad_x (MN-major);
+    // g8 [m][n] is A = [K][M] and x8 [m][k] is B = [K][N] of grad_w (both MN-major)
+    GemmDesc gd[2];
+    int ng = 0;
+    if (need_grad_x)  // grad_x [m][k] = g8 [m][n] . w8 [n][k]
+        gd[ng++] = GemmDesc{g8, w8, fmt_g, fmt_w, 0, 1, m, k, n, n, k, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x};
+    if (need_grad_w)  // grad_w [n][k] = g8^T [n][m] . x8 [m][k]
+        gd[ng++] = GemmDesc{g8, x8, fmt_g, fmt_x, 1, 1, n, k, m, n, k, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
+    const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
+    return gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
+                             need_grad_b ? grad_b : nullptr, &split, stream);
 }
 
 }  // extern "C"

@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         const int jb = tile_job(batch, tl);
         const QArgs& a = batch.job[jb];
         const bool row_out = a.out != nullptr;
+        const bool col_out = a.out_t != nullptr;  // transposed output (else row-major + column sums only)
         const bool colsum = a.colsum != nullptr;
         const float mult = __frcp_rn(__ldg(a.scale));
         const auto* x = static_cast<const E*>(a.x);
@@ -469,8 +470,10 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
                         dst[e] = static_cast<uint8_t>(qq[e >> 2] >> (8 * (e & 3)));
                 }
             }
-            const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
-            *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = q;
+            if (col_out) {
+                const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
+                *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = q;
+            }
         }
         tamax = fmaxf(tamax, In::acc_value(acc));
         if (jb == 0)
@@ -505,7 +508,9 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
             a.colsum[static_cast<int64_t>(tile_y) * cols + c0 + t] = sum;
         }
 
-        // Phase 2: warp w owns tile columns 16w .. 16w+15; lane -> (column group of 4, 16 rows).
+        // Phase 2 (transposed output only): warp w owns tile columns 16w .. 16w+15; lane ->
+        // (column group of 4, 16 rows).
+        if (col_out) {
         uint32_t W[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) W[i] = tile[(16 * rg + i) * 32 + ((w ^ rg) << 2) + cgl];
@@ -533,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
                 for (int b = 0; b < 16 && gr0 + b < rows; ++b)
                     dst[b] = static_cast<uint8_t>(O[jj][b >> 2] >> (8 * (b & 3)));
             }
+        }
         }
         __syncthreads();  // the byte tile and the column sums are free
     }
@@ -746,9 +752,11 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     if (njobs < 1 || njobs > kMaxJobs) return fail(FP8DSA_ERR_INVALID_ARG, "quantize batch of 1..3 tensors");
     const fp8_fmt_t fmt = jobs[0].fmt;
     const fp8_in_t in_type = jobs[0].in_type;
-    const bool tiled = jobs[0].out_t != nullptr;
+    // the tiled kernel serves transposed / dual outputs and anything that needs column sums
+    auto wants_tiles = [](const QuantJob& j) { return j.out_t != nullptr || j.colsum_partial != nullptr; };
+    const bool tiled = wants_tiles(jobs[0]);
     for (int i = 1; i < njobs; ++i)
-        if (jobs[i].fmt != fmt || jobs[i].in_type != in_type || (jobs[i].out_t != nullptr) != tiled)
+        if (jobs[i].fmt != fmt || jobs[i].in_type != in_type || wants_tiles(jobs[i]) != tiled)
             return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares format, input type and orientation");
     QBatch b{};
     b.njobs = njobs;

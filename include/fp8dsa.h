@@ -210,6 +210,51 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
                         void* workspace, size_t workspace_bytes, void* grad_x, void* grad_w,
                         void* grad_b, cudaStream_t stream);
 
+/* linear_forward_fp8 that also keeps its quantized operands for linear_backward_fp8_mixed:
+ *   x8_out: dev [m][k] bytes in `fmt` (16-byte aligned) receives x8;
+ *   w8_out: dev [n][k] bytes in `fmt` (16-byte aligned) receives w8 (ignored when w_is_fp8:
+ *      the caller's w already holds those bytes).
+ * Everything else, including the workspace, is as for linear_forward_fp8; the bytes are the
+ * ones the forward GEMM reads.  Not a separate step on the pages: their backward binding
+ * accepts operands the forward already quantized [compare: the linear backward binding in
+ * an earlier state, pre-quantized g / x / w skip their quantize kernels]. */
+int linear_forward_fp8_keep(const void* x, const void* w, int w_is_fp8, const float* w_step,
+                            const void* bias, const float* bias_scale, int64_t m, int64_t k,
+                            int64_t n, fp8_fmt_t fmt, const fp8_ring_t* x_ring,
+                            const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
+                            float* sw_used, uint8_t* x8_out, uint8_t* w8_out, void* workspace,
+                            size_t workspace_bytes, void* y, cudaStream_t stream);
+
+/* Workspace bytes linear_backward_fp8_mixed needs for (m, k, n): g8, the per-tile column sums,
+ * scale scratch and the GEMM's split-K region. */
+size_t linear_backward_fp8_mixed_workspace_size(int64_t m, int64_t k, int64_t n);
+
+/* Mixed-format backward that reuses the forward's quantized operands as they are (a reading of
+ * the pages' reuse of pre-quantized operands, with each operand keeping its own format: the
+ * tensor core takes the A and B formats separately) [compare: the linear backward binding in
+ * an earlier state]:
+ *   g: dev bf16 [m][n], quantized once row-major in fmt_g (folding g_ring, or at the dynamic
+ *      step when g_ring == NULL: max(amax / fp8_max(fmt_g) / pow2_margin, 1e-12));
+ *   x8: dev [m][k] bytes in fmt_x with step *sx; w8: dev [n][k] bytes in fmt_w with step *sw
+ *      (e.g. from linear_forward_fp8_keep; sx / sw are its sx_used / sw_used); 16-byte aligned.
+ *       grad_x [m][k] = g8 . w8 * RN32(sg * sw)      (w8 read in place as B = [K][N])
+ *       grad_w [n][k] = g8^T . x8 * RN32(sg * sx)    (g8 and x8 read in place)
+ *       grad_b [n]    = RN_bf16(sum over rows of g)
+ *   One quantize launch (g) and one GEMM launch (grad_x and grad_w); x and w are not
+ *   re-quantized.  The numbers differ from linear_backward_fp8 under HYBRID (there x and w are
+ *   re-quantized to E5M2); with fmt_g == fmt_x == fmt_w and x8 / w8 quantized at sx / sw they
+ *   are the same.
+ *   need_grad_x / need_grad_w / need_grad_b select the outputs (the others may be NULL).
+ *   workspace: dev, >= linear_backward_fp8_mixed_workspace_size(m, k, n) bytes, 256-byte
+ *      aligned, no initial contents needed.  k and n must be multiples of 16. */
+int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w8, int64_t m,
+                              int64_t k, int64_t n, fp8_fmt_t fmt_g, fp8_fmt_t fmt_x,
+                              fp8_fmt_t fmt_w, int need_grad_x, int need_grad_w, int need_grad_b,
+                              const float* sx, const float* sw, const fp8_ring_t* g_ring,
+                              float pow2_margin, float* sg_used, void* workspace,
+                              size_t workspace_bytes, void* grad_x, void* grad_w, void* grad_b,
+                              cudaStream_t stream);
+
 /* Device status word of the current device: 0, or a nonzero code a kernel set when a bounded
  * wait ran out (a pipeline stall instead of a hang).  Synchronises `stream`, reads the word
  * into *status (host) and clears it.  Not on the pages: added so no kernel can hang a GPU. */

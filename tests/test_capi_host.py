@@ -109,6 +109,43 @@ def test_linear_argument_checks():
              4096, 4096, 4096, None) == INVALID
 
 
+def test_keep_forward_and_mixed_backward_argument_checks():
+    lib = F.lib()
+    ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
+    kf = lib.linear_forward_fp8_keep
+    # x8_out is required
+    assert kf(256, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, None, 4096, 1024, ws,
+              4096, None) == INVALID
+    # w8_out is required unless w is already fp8
+    assert kf(256, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 4096, None, 1024, ws,
+              4096, None) == INVALID
+    # kept buffers must be 16-byte aligned (TMA reads them)
+    assert kf(256, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 4104, 8192, 1024, ws,
+              4096, None) == UNSUPPORTED
+    mb = lib.linear_backward_fp8_mixed
+    wsm = F.linear_backward_fp8_mixed_workspace_size(64, 64, 64)
+    assert wsm >= 64 * 64 + 4 * 64 and wsm % 256 == 0
+    assert F.linear_backward_fp8_mixed_workspace_size(-1, 1, 1) == 0
+    args = dict(g=256, x8=4096, w8=8192, m=64, k=64, n=64, fg=1, fx=0, fw=0, gx=1, gw=1, gb=1, sx=512, sw=768,
+                ring=None, margin=1.0, sg=None, ws=1024, wsb=wsm, dx=16384, dw=32768, db=65536)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return mb(a["g"], a["x8"], a["w8"], a["m"], a["k"], a["n"], a["fg"], a["fx"], a["fw"], a["gx"], a["gw"],
+                  a["gb"], a["sx"], a["sw"], a["ring"], a["margin"], a["sg"], a["ws"], a["wsb"], a["dx"], a["dw"],
+                  a["db"], None)
+    assert call(fg=5) == INVALID
+    assert call(fx=-1) == INVALID
+    assert call(w8=None) == INVALID          # grad_x without w8
+    assert call(sx=None) == INVALID          # grad_w without x8's step
+    assert call(db=None) == INVALID
+    assert call(k=40) == UNSUPPORTED
+    assert call(x8=4100) == UNSUPPORTED      # x8 not 16-byte aligned
+    assert call(ws=1040) == UNSUPPORTED      # workspace not 256-byte aligned
+    assert call(wsb=wsm - 256) == WORKSPACE
+    assert call(margin=0.0) == INVALID       # dynamic scaling needs a positive margin
+
+
 def test_misc_argument_checks():
     lib = F.lib()
     assert lib.fp8_set_wait_timeout_ns(0) == INVALID
