@@ -420,6 +420,23 @@ __device__ __forceinline__ void add2_rn(float& a, float& b, float c, float d) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
 }
 
+// History-ring fold done after the quantize kernel that measured the amax (one thread; the
+// quantize blocks only left their maxima in the amax slot).  Ring layout [hist n | scale |
+// scale_used | amax | done]: scale_used = the step the quantize used (the current scale),
+// hist[idx] = amax, scale = max(RN32(RN32(peak / fp8_max) / pow2_margin), 1e-12) over the
+// window, amax slot re-zeroed -- the same state the in-kernel fold leaves.
+__device__ __forceinline__ void ring_fold_deferred(float* st, int n, int idx, float fp8_max, float pow2_margin) {
+    const float step = __ldcg(st + n);
+    const float am = __ldcg(st + n + 2);
+    float peak = am;
+    for (int i = 0; i < n; ++i)
+        if (i != idx) peak = fmaxf(peak, __ldcg(st + i));
+    st[n + 1] = step;
+    st[idx] = am;
+    st[n] = fmaxf(__fdiv_rn(__fdiv_rn(peak, fp8_max), pow2_margin), 1e-12f);
+    st[n + 2] = 0.0f;
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
     return __uint_as_float(b << 16);
 }

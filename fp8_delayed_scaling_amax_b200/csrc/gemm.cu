@@ -104,8 +104,18 @@ struct ColsumJob {
     uint16_t* out;
 };
 
+// A history ring whose quantize launch left its fold to this launch.
+constexpr int kMaxFolds = 3;
+struct RingFold {
+    float* state;
+    int hist_len, hist_idx;
+    float fp8_max, pow2_margin;
+};
+
 struct GemmArgs {
     GemmProblem p[kMaxProblems];
+    RingFold folds[kMaxFolds];
+    int nfolds;
     int nprob;
     int num_tiles;
     int num_units, contrib_units;  // work units (tile, K range); the first contrib_units are split-K contributors
@@ -444,6 +454,12 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
         const int cbase = (ew >> 2) * C::kEpiCols;
         uint8_t* my_stage = sOut + ew * 2 * kOutStageBytes;
 
+        // side job: the deferred ring folds of the quantize launch before (one thread)
+        if (g.nfolds > 0 && blockIdx.x == 0 && ew == 0 && lane == 0) {
+            for (int f = 0; f < g.nfolds; ++f)
+                ring_fold_deferred(g.folds[f].state, g.folds[f].hist_len, g.folds[f].hist_idx, g.folds[f].fp8_max,
+                                   g.folds[f].pow2_margin);
+        }
         // side job: the bias gradient from the per-tile column sums (before the first tile)
         if (g.colsum.tiles > 0) {
             const int et = ew * 32 + lane;
@@ -642,6 +658,16 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
         else
             tmem_dealloc(tmem_base, 2 * BN);
     }
+}
+
+// The deferred ring folds, when no GEMM kernel runs to do them.
+__global__ void ring_fold_kernel(const __grid_constant__ GemmArgs g) {
+    pdl_trigger();
+    pdl_wait();
+    if (threadIdx.x == 0)
+        for (int f = 0; f < g.nfolds; ++f)
+            ring_fold_deferred(g.folds[f].state, g.folds[f].hist_len, g.folds[f].hist_idx, g.folds[f].fp8_max,
+                               g.folds[f].pow2_margin);
 }
 
 // k == 0: the product is empty; out = bias (or 0), rounded to bf16.
@@ -937,8 +963,23 @@ int64_t splitk_counter_words(const int64_t* m, const int64_t* n, int nprob) {
     return total;
 }
 
+// Launch the one-thread fold kernel for `g.nfolds` rings.
+int launch_fold_only(const GemmArgs& g, cudaStream_t stream) {
+    launch_begin(kKindOther, stream);
+    launch_ex(ring_fold_kernel, dim3(1), dim3(32), 0, stream, 1, g);
+    launch_end(kKindOther, stream, 0.0);
+    return check_launch("ring fold kernel");
+}
+
 int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
-                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, cudaStream_t stream) {
+                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, const fp8_ring_t* folds,
+                      int nfolds, cudaStream_t stream) {
+    if (nfolds < 0 || nfolds > kMaxFolds) return fail(FP8DSA_ERR_INVALID_ARG, "at most 3 deferred ring folds");
+    GemmArgs fold_args{};
+    fold_args.nfolds = nfolds;
+    for (int i = 0; i < nfolds; ++i)
+        fold_args.folds[i] = RingFold{folds[i].state, folds[i].hist_len, folds[i].hist_idx, folds[i].fp8_max,
+                                      folds[i].pow2_margin};
     // problems with an empty product write their bias (or zeros) without the tensor cores
     GemmDesc work[kMaxProblems];
     int nwork = 0;
@@ -962,19 +1003,21 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
     }
     const bool colsum = colsum_tiles > 0 && colsum_cols > 0;
     if (nwork == 0) {
-        if (colsum) return launch_colsum_finalize(colsum_partial, colsum_tiles, colsum_cols, colsum_out, stream);
-        if (colsum_cols > 0 && colsum_out != nullptr) {  // no rows: the bias gradient is zero
+        if (colsum) {
+            const int rc = launch_colsum_finalize(colsum_partial, colsum_tiles, colsum_cols, colsum_out, stream);
+            if (rc) return rc;
+        } else if (colsum_cols > 0 && colsum_out != nullptr) {  // no rows: the bias gradient is zero
             cudaError_t e = cudaMemsetAsync(colsum_out, 0, sizeof(uint16_t) * colsum_cols, stream);
             if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset grad_b: ") + cudaGetErrorString(e));
         }
-        return FP8DSA_OK;
+        return nfolds > 0 ? launch_fold_only(fold_args, stream) : FP8DSA_OK;
     }
     if (colsum_cols > 0x7FFFFFFF || colsum_tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "bias gradient too wide");
     const TileChoice tc = choose_tiles(work, nwork);
     const int b_rows = tc.pair ? tc.bn / 2 : tc.bn;  // rows of B each CTA loads
 
     CUtensorMap maps[6];
-    GemmArgs g{};
+    GemmArgs g = fold_args;
     int64_t batch[kMaxProblems] = {1, 1};
     const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
     for (int i = 0; i < nwork; ++i) {
@@ -1062,7 +1105,7 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
                 int bias_kind, const float* bias_scale, void* out, cudaStream_t stream) {
     GemmDesc d{a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
                scale_a, scale_b, bias, bias_kind, bias_scale, out};
-    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, nullptr, stream);
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, stream);
 }
 
 }  // namespace fp8dsa

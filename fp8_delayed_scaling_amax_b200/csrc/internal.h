@@ -121,6 +121,7 @@ struct QuantJob {
     const fp8_ring_t* ring = nullptr;
     float* scale_used_out = nullptr;  // the step used, written once (may be nullptr)
     float* colsum_partial = nullptr;  // [ceil(rows/128)][cols] fp32 column sums (tiled only)
+    bool defer_fold = false;          // ring: only leave the amax; a later kernel folds the ring
 };
 int launch_quantize(const QuantJob& job, cudaStream_t stream);
 // Up to three tensors in one launch (same format, input type and orientation); each tensor
@@ -166,8 +167,12 @@ int64_t splitk_counter_words(const int64_t* m, const int64_t* n, int nprob);
 // the epilogue warps first write colsum_out[c] = RN_bf16(sum_t colsum_partial[t][c]).  With
 // `split` (may be null) the launch may cut tiles' K ranges across CTAs where that shortens
 // the schedule; the result differs from the unsplit one only in fp32 summation order.
+// `folds` (up to 3, may be empty): rings whose quantize launch deferred its fold; the GEMM
+// launch folds them (one thread, after its dependency wait), or a one-thread kernel does
+// when no GEMM kernel runs.
 int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_partial, int64_t colsum_tiles,
-                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, cudaStream_t stream);
+                      int64_t colsum_cols, void* colsum_out, const SplitWorkspace* split, const fp8_ring_t* folds,
+                      int nfolds, cudaStream_t stream);
 
 // Split-K mode of later GEMM launches (0 automatic, 1 never, 2..4 forced); rejects others.
 int gemm_set_split_mode(int mode);

@@ -8,12 +8,15 @@
 // grad_w = g8T . x8T^T, both NT; grad_b = column sum of g).
 //
 // Launches per call (delayed scaling):
-//   forward : one quantize launch for x and w (each folds its own ring) + GEMM           = 2
-//   backward: one quantize launch for g (both orientations, ring fold, per-tile column
-//             sums), x^T and w^T + one GEMM launch for dX and dW whose epilogue warps
-//             also reduce the column sums into grad_b                                 = 2
-// The snapshot of each step is written by the folding kernel itself (no clone launches), so
-// the GEMM dequantizes with exactly the step the bytes were quantized with.
+//   forward : one quantize launch for x and w + GEMM                                    = 2
+//   backward: one quantize launch for g (both orientations, per-tile column sums), x^T
+//             and w^T + one GEMM launch for dX and dW whose epilogue warps also reduce
+//             the column sums into grad_b                                             = 2
+// The quantize launch reads each ring's step, writes the snapshot (the step used) from its
+// first block and leaves the measured amax in the ring's amax slot; the GEMM launch that
+// follows folds the rings (one epilogue thread, after its dependency wait), so the quantize
+// launch ends without a last-block tail.  The GEMM dequantizes with exactly the step the
+// bytes were quantized with.
 #include <cuda_runtime.h>
 
 #include <string>
@@ -244,6 +247,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
         qx.scale = x_ring->state + x_ring->hist_len;
         qx.ring = x_ring;
         qx.scale_used_out = sx;
+        qx.defer_fold = true;  // folded by the GEMM launch below
     }
     QuantJob fwd_jobs[2];
     int nfj = 0;
@@ -261,6 +265,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
             qw.scale = w_ring->state + w_ring->hist_len;
             qw.ring = w_ring;
             qw.scale_used_out = sw;
+            qw.defer_fold = true;
         }
         fwd_jobs[nfj++] = qw;
     }
@@ -278,7 +283,13 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     int bias_kind = 0;
     if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt == FP8_E4M3 ? 2 : 3);
     const GemmDesc d{x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y};
-    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, allow_split ? &split : nullptr, stream);
+    fp8_ring_t folds[2];
+    int nfolds = 0;
+    if (!dynamic) {
+        folds[nfolds++] = *x_ring;
+        if (!w_is_fp8) folds[nfolds++] = *w_ring;
+    }
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, allow_split ? &split : nullptr, folds, nfolds, stream);
 }
 
 }  // namespace fp8dsa
@@ -374,6 +385,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         qg.scale = g_ring->state + g_ring->hist_len;
         qg.ring = g_ring;
         qg.scale_used_out = sg;
+        qg.defer_fold = true;  // folded by the GEMM launch below
     }
     // g (both orientations), x^T and w^T in one launch
     QuantJob bwd_jobs[3];
@@ -415,7 +427,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         gd[ng++] = GemmDesc{g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
     const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
     rc = gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
-                           need_grad_b ? grad_b : nullptr, &split, stream);
+                           need_grad_b ? grad_b : nullptr, &split, g_ring, dynamic ? 0 : 1, stream);
     if (rc) return rc;
     return FP8DSA_OK;
 }
@@ -488,6 +500,7 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
         qg.scale = g_ring->state + g_ring->hist_len;
         qg.ring = g_ring;
         qg.scale_used_out = sg;
+        qg.defer_fold = true;  // folded by the GEMM launch below
     }
     SplitWorkspace split;
     split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
@@ -506,7 +519,7 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
         gd[ng++] = GemmDesc{g8, x8, fmt_g, fmt_x, 1, 1, n, k, m, n, k, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
     const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
     return gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
-                             need_grad_b ? grad_b : nullptr, &split, stream);
+                             need_grad_b ? grad_b : nullptr, &split, g_ring, dynamic ? 0 : 1, stream);
 }
 
 }  // extern "C"

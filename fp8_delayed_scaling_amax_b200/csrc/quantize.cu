@@ -136,6 +136,7 @@ struct QArgs {
     int hist_len, hist_idx;
     float fp8_max, pow2_margin;
     float* scale_used_out;     // receives the step used, or null
+    int defer_fold;            // ring: leave the amax in its slot; the next kernel folds it
     float* colsum;             // [row tiles][cols] per-tile column sums (tiled kernel), or null
     int vec_in, vec_out, vec_out_t;
     int tma;                   // tiled kernel: input tiles arrive by TMA through map[job]
@@ -200,6 +201,11 @@ __device__ __forceinline__ void ring_prefetch(const QArgs& a, float* hist) {
 __device__ __forceinline__ void job_finish(const QArgs& a, float m, float step, bool first_block,
                                            const float* hist) {
     if (a.amax_accum != nullptr) atomicMax(reinterpret_cast<unsigned*>(a.amax_accum), __float_as_uint(m));
+    if (a.ring_state != nullptr && a.defer_fold) {
+        // the fold runs in the kernel that follows (no ticket: the launch ends with no tail)
+        if (first_block && a.scale_used_out != nullptr) *a.scale_used_out = step;
+        return;
+    }
     if (a.ring_state != nullptr) {
         float* st = a.ring_state;
         const int n = a.hist_len;
@@ -778,6 +784,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         a.out_t = job.out_t;
         a.scale_used_out = job.scale_used_out;
         a.colsum = job.colsum_partial;
+        a.defer_fold = job.ring != nullptr && job.defer_fold ? 1 : 0;
         if (job.ring != nullptr) {
             const int n = job.ring->hist_len;
             a.ring_state = job.ring->state;

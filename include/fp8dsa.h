@@ -143,9 +143,11 @@ size_t linear_forward_fp8_workspace_size(int64_t m, int64_t k, int64_t n);
  *   x: dev bf16 [m][k]; w: dev bf16 [n][k], or fp8 bytes in `fmt` when w_is_fp8 (then
  *      w_step, dev fp32, is the step those bytes were quantized with, and w_ring is unused).
  *   bias: NULL, dev bf16[n], or dev fp8[n] in `fmt` with bias_scale (dev fp32).
- *   Delayed scaling: x_ring and w_ring given.  Each quantize reads its ring's step, folds the
- *      fresh amax in its last block and publishes the next step; the GEMM dequantizes with
- *      the steps used (the snapshot) [ext-log: snapshot sx/sw before the finalize].
+ *   Delayed scaling: x_ring and w_ring given.  Each quantize reads its ring's step and
+ *      measures the fresh amax; the fold (hist[idx] = amax, next step published, snapshot of
+ *      the step used) runs in the GEMM launch that follows, so the GEMM dequantizes with the
+ *      steps used (the snapshot) [ext-log: snapshot sx/sw before the finalize].  The ring
+ *      states after the call are the same as with the quantize entry's in-kernel fold.
  *   Dynamic scaling: x_ring == NULL (and w_ring == NULL): the steps are measured from x and
  *      w first (max(amax / fp8_max / pow2_margin, 1e-12)), with fp8_max of `fmt` and
  *      pow2_margin given here.
