@@ -255,7 +255,11 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     pdl_trigger();
     pdl_wait();
     zero_side_job(batch);
-    const QArgs& a = batch.job[blockIdx.y];  // one grid row of blocks per tensor
+    // each tensor owns a contiguous range of blocks, sized to its share of the elements
+    int jb = 0;
+    while (jb + 1 < batch.njobs && static_cast<int>(blockIdx.x) >= batch.job[jb + 1].tile_begin) ++jb;
+    const QArgs& a = batch.job[jb];
+    const int64_t lb = static_cast<int64_t>(blockIdx.x) - a.tile_begin;  // block within the tensor
     __shared__ float s_hist[kHistPrefetch];
     ring_prefetch(a, s_hist);
     const float step = __ldg(a.scale);
@@ -263,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     const auto* x = static_cast<const typename In::E*>(a.x);
     float amax = 0.0f;
     typename In::Acc acc = In::acc_zero();  // running max of |x| over the vector chunks
-    const int64_t gstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t gstride = static_cast<int64_t>(a.nblocks) * blockDim.x;
+    const int64_t tid = lb * blockDim.x + threadIdx.x;
     const int64_t n16 = a.vec_in ? a.numel / 16 : 0;
     for (int64_t g = tid; g < n16; g += 2 * gstride) {
         const int64_t g1 = g + gstride;
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
         amax = fmaxf(amax, fabsf(v));
         a.out[i] = convert1<kFmt>(v, mult);
     }
-    block_finish(a, amax, step, blockIdx.x == 0, s_hist);
+    block_finish(a, amax, step, lb == 0, s_hist);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -684,6 +688,14 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
     out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
 }
 
+#ifndef FLAT_WAVES
+#define FLAT_WAVES 1
+#endif
+constexpr int kFlatWaves = FLAT_WAVES;
+
+// Resident 256-thread blocks per SM of the row-major kernel (its launch bounds ask for 4).
+int flat_blocks_per_sm() { return 4; }
+
 template <int kFmt, class In>
 void launch_flat(const QBatch& b, dim3 grid, cudaStream_t stream) {
     launch_ex(quant_flat_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
@@ -770,7 +782,6 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     b.zero_words = zero != nullptr ? zero_words : 0;
     const int eb = in_type_bytes(in_type);
     double bytes = 0.0;
-    int64_t max_groups = 0;
     int64_t tiles_total = 0;
     for (int i = 0; i < njobs; ++i) {
         const QuantJob& job = jobs[i];
@@ -826,8 +837,6 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
             a.tile_begin = static_cast<int>(tiles_total);
             tiles_total += tx * ty;
             if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
-        } else {
-            max_groups = std::max(max_groups, (a.numel + 15) / 16);
         }
     }
     dim3 grid;
@@ -837,10 +846,24 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         const int rc = wait_ctl(&ctl);
         if (rc) return rc;
     } else {
-        const int64_t want = std::max<int64_t>(1, (max_groups + kThreads - 1) / kThreads);
-        const int per_job = static_cast<int>(std::min<int64_t>(want, std::max<int64_t>(1, static_cast<int64_t>(sm_count()) * 8 / njobs)));
-        for (int i = 0; i < njobs; ++i) b.job[i].nblocks = static_cast<unsigned>(per_job);
-        grid = dim3(static_cast<unsigned>(per_job), static_cast<unsigned>(njobs));
+        // one wave: the resident blocks are shared out in proportion to the tensors' sizes
+        // (every tensor gets at least one block; none more than one thread per 16 elements)
+        const int64_t budget = static_cast<int64_t>(sm_count()) * flat_blocks_per_sm() * kFlatWaves;
+        int64_t groups[kMaxJobs], total_groups = 0;
+        for (int i = 0; i < njobs; ++i) {
+            groups[i] = std::max<int64_t>(1, (b.job[i].numel + 15) / 16);
+            total_groups += groups[i];
+        }
+        int64_t begin = 0;
+        for (int i = 0; i < njobs; ++i) {
+            const int64_t want = (groups[i] + kThreads - 1) / kThreads;
+            const int64_t share = std::max<int64_t>(1, budget * groups[i] / total_groups);
+            const int64_t nb = std::max<int64_t>(1, std::min(want, share));
+            b.job[i].nblocks = static_cast<unsigned>(nb);
+            b.job[i].tile_begin = static_cast<int>(begin);
+            begin += nb;
+        }
+        grid = dim3(static_cast<unsigned>(begin));
     }
     launch_begin(kKindQuantize, stream);
     int rc;
