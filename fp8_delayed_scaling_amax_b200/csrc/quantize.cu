@@ -446,6 +446,29 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
 #pragma unroll
             for (int i = 0; i < 8; ++i) raw[i] = In::load_raw(x + (r0 + rr + 16 * i) * cols + gc);
         }
+        // a full tile with vector-aligned outputs: no per-row checks, addresses stepped (in the
+        // one-tile-per-CTA kernel, which is issue-bound on small batches; the persistent one keeps
+        // its register budget)
+        const bool full = !kPersist && (from_smem || interior) && r0 + kTile <= rows && c0 + kTile <= cols &&
+                          (!row_out || a.vec_out);
+        if (full) {
+            uint8_t* orow = row_out ? a.out + (r0 + rr) * cols + gc : nullptr;
+            const int64_t ostep = 16 * cols;
+            uint32_t* trow = tile + rr * 32 + (j & 1) * 2;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float f[8];
+                In::acc_max(acc, raw[i]);
+                In::unpack(raw[i], f);
+                if (colsum) {
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
+                }
+                const uint2 q = quant8<kFmt>(f, mult);
+                if (row_out) *reinterpret_cast<uint2*>(orow + i * ostep) = q;
+                if (col_out) *reinterpret_cast<uint2*>(trow + i * 512 + (((j >> 1) ^ i) << 2)) = q;
+            }
+        } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int r = rr + 16 * i;
@@ -484,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
                 const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
                 *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = q;
             }
+        }
         }
         tamax = fmaxf(tamax, In::acc_value(acc));
         if (jb == 0)
