@@ -142,6 +142,8 @@ struct QArgs {
     int tma;                   // tiled kernel: input tiles arrive by TMA through map[job]
     unsigned nblocks;          // blocks working on this tensor (the ticket count of its fold)
     int tile_begin, tiles_x;   // tiled kernel: first tile of this tensor, column tiles
+    int tiles_y;               // tiled kernel: row tiles
+    int tile_group;            // tiled kernel: tile rows per group of the traversal order
 };
 
 // Up to three tensors quantized by one launch; each keeps its own amax, ticket and fold.
@@ -331,6 +333,26 @@ struct TiledCfg {
     static constexpr int kMinBlocks = kPersist ? (kF32 ? 1 : 2) : (kF32 ? 2 : 3);
 };
 
+// Tile `local` of a tensor -> (tile row, tile column): groups of a.tile_group tile rows,
+// walked column by column within a group.  Row order (group 1) keeps the tiles in flight on
+// the same input rows; groups of 4 put four neighbouring 128-byte pieces of each transposed
+// output row in flight together, which the dual quantize of very tall tensors prefers.
+__device__ __forceinline__ void tile_coords(const QArgs& a, int local, int& ty, int& tx) {
+    const int G = a.tile_group;
+    if (G <= 1) {
+        ty = local / a.tiles_x;
+        tx = local % a.tiles_x;
+        return;
+    }
+    const int per_group = G * a.tiles_x;
+    const int grp = local / per_group;
+    const int first = grp * G;
+    const int gh = min(a.tiles_y - first, G);
+    const int within = local - grp * per_group;
+    ty = first + within % gh;
+    tx = within / gh;
+}
+
 __device__ __forceinline__ int tile_job(const QBatch& b, int tl) {
     int jb = 0;
     while (jb + 1 < b.njobs && tl >= b.job[jb + 1].tile_begin) ++jb;
@@ -383,8 +405,9 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         if (!kPersist || !a.tma) return;
         const int local = tl - a.tile_begin;
         mbar_arrive_expect_tx(&bar[s], C::kRawBytes);
-        tma_load_3d(smem + s * C::kRawBytes, &batch.map[jb], &bar[s], (local % a.tiles_x) * kTile,
-                    (local / a.tiles_x) * kTile, 0);
+        int ty, tx;
+        tile_coords(a, local, ty, tx);
+        tma_load_3d(smem + s * C::kRawBytes, &batch.map[jb], &bar[s], tx * kTile, ty * kTile, 0);
         pending |= 1u << s;
     };
     if (t == 0) {
@@ -413,9 +436,10 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         const auto* x = static_cast<const E*>(a.x);
         const int64_t rows = a.rows, cols = a.cols;
         const int local = tl - a.tile_begin;
-        const int tile_y = local / a.tiles_x;
+        int tile_y, tile_x;
+        tile_coords(a, local, tile_y, tile_x);
         const int64_t r0 = static_cast<int64_t>(tile_y) * kTile;
-        const int64_t c0 = static_cast<int64_t>(local % a.tiles_x) * kTile;
+        const int64_t c0 = static_cast<int64_t>(tile_x) * kTile;
         const int64_t gc = c0 + 8 * j;
         const bool from_smem = kPersist && a.tma != 0;
         const bool interior = !from_smem && a.vec_in && r0 + kTile <= rows && c0 + kTile <= cols;
@@ -858,6 +882,10 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
             const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);
             const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
             a.tiles_x = static_cast<int>(tx);
+            a.tiles_y = static_cast<int>(ty);
+            // measured (persistent kernel, B200): groups of 4 tile rows pay off only for the dual
+            // quantize with transposed rows at least 16 KB apart; row order everywhere else
+            a.tile_group = (job.out != nullptr && job.out_t != nullptr && job.rows >= 16384) ? 4 : 1;
             a.tile_begin = static_cast<int>(tiles_total);
             tiles_total += tx * ty;
             if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
