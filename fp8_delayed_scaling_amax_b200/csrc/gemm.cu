@@ -197,6 +197,13 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& g) {
     return r;
 }
 
+// The unit a CTA (or pair) `unit` of `units` takes in round r: rounds alternate direction
+// (boustrophedon), so a CTA that drew a long unit in one round draws a short one in the next
+// when the units are ordered longest first.  Each CTA's units still increase with r.
+__device__ __forceinline__ int snake_unit(int r, int unit, int units) {
+    return r * units + ((r & 1) ? units - 1 - unit : unit);
+}
+
 // Contributor unit index of split s (>= 1) of tile `tile` of problem P.
 __device__ __forceinline__ int contrib_slot(const GemmProblem& P, int tile, int s) {
     return P.contrib_begin + (s - 1) * P.tiles + (tile - P.tile_begin);
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;  // per-stage: ever issued, parity of the last issue
             bool ok = true;
-            for (int u = unit; u < g.num_units && ok; u += units) {
+            for (int r = 0, u = unit; u < g.num_units && ok; u = snake_unit(++r, unit, units)) {
                 const Unit w = decode_unit<kSplit>(u, g);
                 int pi, b, tm, tn;
                 decode_tile(w.tile, g, pi, b, tm, tn);
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             constexpr uint32_t kLboB = 128 * kBK;  // distance between 128-wide MN blocks of B
-            for (int u = unit; u < g.num_units && ok; u += units) {
+            for (int r = 0, u = unit; u < g.num_units && ok; u = snake_unit(++r, unit, units)) {
                 const Unit w = decode_unit<kSplit>(u, g);
                 const GemmProblem& P = g.p[w.pi];
                 const bool got = kPair ? mbar_wait_bounded_cluster(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
@@ -499,7 +506,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
         uint32_t acc_phase = 0;
         constexpr int kCtas = kPair ? 2 : 1;
         const int row_in = q * 32 + lane;  // this thread's row within the CTA's 128 rows
-        for (int u = unit; u < g.num_units; u += units) {
+        for (int r = 0, u = unit; u < g.num_units; u = snake_unit(++r, unit, units)) {
             const Unit w = decode_unit<kSplit>(u, g);
             int pi, b, tm, tn;
             decode_tile(w.tile, g, pi, b, tm, tn);
@@ -1001,6 +1008,9 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
         work[nwork++] = d;
         flops += 2.0 * static_cast<double>(d.m) * d.n * d.k * d.batch;
     }
+    // the problem with the longer K (the longer tiles) first: with the alternating rounds of
+    // the tile schedule this spreads long and short tiles evenly over the CTAs
+    if (nwork == 2 && work[1].k > work[0].k) std::swap(work[0], work[1]);
     const bool colsum = colsum_tiles > 0 && colsum_cols > 0;
     if (nwork == 0) {
         if (colsum) {
