@@ -54,6 +54,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sweeps", action="store_true")
     p.add_argument("--no-variants", action="store_true", help="skip the mixed-format backward variant")
+    p.add_argument("--dp-fold", action="store_true",
+                   help="fold the rings once per step after an amax all-reduce (always on with several GPUs)")
     p.add_argument("--kernel", default=None, choices=["gemm", "quantize"],
                    help="time one kernel on one shape instead of the step (small cases for ncu)")
     p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS")
@@ -490,8 +492,26 @@ def main():
     flops_step = sum(l.gemm_flops for l in lins)
     qbytes_step = sum(l.quant_bytes for l in lins)
 
+    # Data parallel over several GPUs: the linears leave each ring's amax in its slot and, after
+    # every step, the ranks reduce all rings' amax (one all-reduce MAX) and fold them, so every
+    # rank keeps the same rings.  One GPU folds inside the calls.
+    dp_rings, dp_buf = [], None
+    use_dp = world > 1 or args.dp_fold
+    if use_dp:
+        from fp8_delayed_scaling_amax_b200 import dp as DP
+        F.fp8_set_ring_fold_mode(1)
+        dp_rings = [r for l in lins for r in (l.rx, l.rw, l.rg)]
+        dp_buf = torch.zeros(len(dp_rings), dtype=torch.float32, device=dev)
+
+    def end_of_step(slot):
+        if use_dp:
+            for l in lins:
+                l.set_slot(slot)
+            DP.fold_rings_data_parallel(dp_rings, dp_buf)
+
     # eager warm step (module load, attributes), then one graph per ring slot
     run_step(lins, 0)
+    end_of_step(0)
     torch.cuda.synchronize()
     assert F.fp8_get_device_status() == 0
     cap = torch.cuda.Stream()
@@ -506,7 +526,9 @@ def main():
     counter = [1]  # the eager warm step used slot 0
 
     def replay():
-        graphs[counter[0] % HIST].replay()
+        slot = counter[0] % HIST
+        graphs[slot].replay()
+        end_of_step(slot)
         counter[0] += 1
 
     for t in range(args.warmup):
@@ -538,6 +560,7 @@ def main():
     mixed = None
     if not args.no_variants:
         run_step(lins, counter[0] % HIST, mixed=True)
+        end_of_step(counter[0] % HIST)
         counter[0] += 1
         torch.cuda.synchronize()
         mgraphs = []
@@ -549,6 +572,7 @@ def main():
         torch.cuda.synchronize()
         for t in range(args.warmup):
             mgraphs[counter[0] % HIST].replay()
+            end_of_step(counter[0] % HIST)
             counter[0] += 1
         torch.cuda.synchronize()
         if world > 1:
@@ -558,6 +582,7 @@ def main():
         s0.record()
         for t in range(msteps):
             mgraphs[counter[0] % HIST].replay()
+            end_of_step(counter[0] % HIST)
             counter[0] += 1
         s1.record()
         torch.cuda.synchronize()
@@ -587,6 +612,7 @@ def main():
     F.fp8_profiler_enable(False)
     for t in range(HIST):
         timed_graphs[counter[0] % HIST].replay()
+        end_of_step(counter[0] % HIST)
         counter[0] += 1
     torch.cuda.synchronize()
     n_instr = HIST
@@ -652,7 +678,8 @@ def main():
                    "linears_kn": [list(kn) for kn in W.TRAINING_LINEARS],
                    "l2": "inputs larger than L2: every layer has its own x, w, g (about 3 GB working set)",
                    "graphs": f"one CUDA graph per history slot ({HIST})",
-                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+                   "parallelism": (f"data parallel over {world} GPU(s): each rank its own batch, one all-reduce "
+                                   f"(MAX) of every ring's amax per step" if use_dp else "single GPU")},
         "gemm_flops_per_step": flops_step, "quantize_bytes_per_step": qbytes_step,
         "kernels": {"gemm_tflops": gemm_tflops, "gemm_ms_per_step": g_ms / n_instr,
                     "quantize_gbs": quant_gbs, "quantize_ms_per_step": q_ms / n_instr,

@@ -66,6 +66,9 @@ _SIGNATURES = {
     "fp8_set_pdl": (c_int, [c_int]),
     "fp8_set_tiled_persist_threshold": (c_int, [c_int64]),
     "fp8_set_gemm_split_k": (c_int, [c_int]),
+    "fp8_set_ring_fold_mode": (c_int, [c_int]),
+    "fp8_scale_ring_collect_amax": (c_int, [POINTER(fp8_ring_t), c_int, _P, _P]),
+    "fp8_scale_ring_fold": (c_int, [POINTER(fp8_ring_t), c_int, _P, _P]),
     "fp8_profiler_enable": (c_int, [c_int]),
     "fp8_profiler_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double)]),
     "fp8_last_error": (c_char_p, []),
@@ -268,6 +271,29 @@ def fp8_set_wait_timeout_ns(ns: int):
 
 def fp8_set_pdl(enabled: bool = True):
     return _check("fp8_set_pdl", lib().fp8_set_pdl(int(bool(enabled))))
+
+
+def _ring_array(rings):
+    arr = (fp8_ring_t * max(1, len(rings)))()
+    for i, r in enumerate(rings):
+        arr[i] = r.as_c() if isinstance(r, Ring) else r
+    return arr
+
+
+def fp8_scale_ring_collect_amax(rings, amax_out, stream=None):
+    """amax_out[i] = ring i's amax slot (dev fp32 tensor of len(rings))."""
+    return _check("fp8_scale_ring_collect_amax", lib().fp8_scale_ring_collect_amax(
+        _ring_array(rings), len(rings), _ptr(amax_out), _stream(stream)))
+
+
+def fp8_scale_ring_fold(rings, amax=None, stream=None):
+    """Fold every ring with amax[i] (or its own amax slot when amax is None)."""
+    return _check("fp8_scale_ring_fold", lib().fp8_scale_ring_fold(
+        _ring_array(rings), len(rings), _ptr(amax), _stream(stream)))
+
+
+def fp8_set_ring_fold_mode(mode: int = 0):
+    return _check("fp8_set_ring_fold_mode", lib().fp8_set_ring_fold_mode(int(mode)))
 
 
 def fp8_set_gemm_split_k(splits: int = 1):

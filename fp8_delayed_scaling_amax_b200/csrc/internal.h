@@ -44,6 +44,10 @@ int encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* b
 // After a launch: map a launch failure to FP8DSA_ERR_CUDA.
 int check_launch(const char* what);
 
+// Whether the linear entries fold their rings within the call (default) or leave the measured
+// amax in each ring's amax slot for fp8_scale_ring_fold (data-parallel training).
+bool ring_fold_in_call();
+
 // Whether library kernels are launched with programmatic dependent launch (default on).
 bool pdl_enabled();
 

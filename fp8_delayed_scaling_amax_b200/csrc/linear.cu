@@ -285,7 +285,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     const GemmDesc d{x8, w8, fmt, fmt, 0, 0, m, n, k, k, k, n, 1, 0, 0, 0, sx, sw, bias, bias_kind, bias_scale, y};
     fp8_ring_t folds[2];
     int nfolds = 0;
-    if (!dynamic) {
+    if (!dynamic && ring_fold_in_call()) {
         folds[nfolds++] = *x_ring;
         if (!w_is_fp8) folds[nfolds++] = *w_ring;
     }
@@ -427,7 +427,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
         gd[ng++] = GemmDesc{g8t, x8t, fmt, fmt, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
     const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
     rc = gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
-                           need_grad_b ? grad_b : nullptr, &split, g_ring, dynamic ? 0 : 1, stream);
+                           need_grad_b ? grad_b : nullptr, &split, g_ring, (dynamic || !ring_fold_in_call()) ? 0 : 1, stream);
     if (rc) return rc;
     return FP8DSA_OK;
 }
@@ -519,7 +519,7 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
         gd[ng++] = GemmDesc{g8, x8, fmt_g, fmt_x, 1, 1, n, k, m, n, k, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
     const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
     return gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
-                             need_grad_b ? grad_b : nullptr, &split, g_ring, dynamic ? 0 : 1, stream);
+                             need_grad_b ? grad_b : nullptr, &split, g_ring, (dynamic || !ring_fold_in_call()) ? 0 : 1, stream);
 }
 
 }  // extern "C"

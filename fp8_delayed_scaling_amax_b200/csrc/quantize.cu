@@ -713,6 +713,33 @@ __global__ void __launch_bounds__(kThreads) amax_jobs_kernel(AmaxArgs a) {
     atomicExch(scr + 1, 0u);
 }
 
+// Ring lists for the data-parallel fold (up to kRingChunk rings per launch, by value).
+constexpr int kRingChunk = 128;  // 3 KB of kernel parameters
+struct RingList {
+    fp8_ring_t ring[kRingChunk];
+    int n;
+};
+
+// out[i] = ring i's amax slot (the maxima its quantize launches left there).
+__global__ void ring_collect_kernel(const __grid_constant__ RingList L, float* out) {
+    pdl_trigger();
+    pdl_wait();
+    const int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+    if (i < L.n) out[i] = __ldcg(L.ring[i].state + L.ring[i].hist_len + 2);
+}
+
+// Fold ring i (one thread each): with `amax` given, that value replaces the slot's (the
+// maximum over all ranks), then the same fold the linear entries do after their quantize.
+__global__ void ring_fold_list_kernel(const __grid_constant__ RingList L, const float* amax) {
+    pdl_trigger();
+    pdl_wait();
+    const int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= L.n) return;
+    const fp8_ring_t& r = L.ring[i];
+    if (amax != nullptr) r.state[r.hist_len + 2] = __ldcg(amax + i);
+    ring_fold_deferred(r.state, r.hist_len, r.hist_idx, r.fp8_max, r.pow2_margin);
+}
+
 __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* partial, int64_t tiles,
                                                                     int64_t cols, uint16_t* out) {
     pdl_trigger();
@@ -1081,6 +1108,45 @@ int fp8_set_tiled_persist_threshold(int64_t min_tiles) {
     if (min_tiles < 0) return fail(FP8DSA_ERR_INVALID_ARG, "min_tiles must be >= 0");
     g_persist_min_tiles.store(min_tiles);
     return FP8DSA_OK;
+}
+
+static int ring_list_call(const fp8_ring_t* rings, int n, float* collect_out, const float* fold_amax, bool fold,
+                          cudaStream_t stream) {
+    if (n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "n must be >= 0");
+    if (n > 0 && rings == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "rings is NULL");
+    for (int i = 0; i < n; ++i) {
+        int rc = check_ring(&rings[i]);
+        if (rc) return fail(rc, "ring " + std::to_string(i) + ": " + fp8_last_error());
+    }
+    if (n == 0) return FP8DSA_OK;
+    int rc = check_device();
+    if (rc) return rc;
+    for (int base = 0; base < n; base += kRingChunk) {
+        RingList L{};
+        L.n = std::min(kRingChunk, n - base);
+        for (int i = 0; i < L.n; ++i) L.ring[i] = rings[base + i];
+        launch_begin(kKindOther, stream);
+        if (fold)
+            launch_ex(ring_fold_list_kernel, dim3(1), dim3(kRingChunk), 0, stream, 1, L,
+                      fold_amax != nullptr ? fold_amax + base : nullptr);
+        else
+            launch_ex(ring_collect_kernel, dim3(1), dim3(kRingChunk), 0, stream, 1, L, collect_out + base);
+        launch_end(kKindOther, stream, 0.0);
+        rc = check_launch(fold ? "ring fold kernel" : "ring collect kernel");
+        if (rc) return rc;
+    }
+    return FP8DSA_OK;
+}
+
+int fp8_scale_ring_collect_amax(const fp8_ring_t* rings, int n, float* amax_out, cudaStream_t stream) {
+    clear_error();
+    if (n > 0 && amax_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "amax_out is NULL");
+    return ring_list_call(rings, n, amax_out, nullptr, false, stream);
+}
+
+int fp8_scale_ring_fold(const fp8_ring_t* rings, int n, const float* amax, cudaStream_t stream) {
+    clear_error();
+    return ring_list_call(rings, n, nullptr, amax, true, stream);
 }
 
 int fp8_quantize_dual(const void* x, fp8_in_t in_type, int64_t rows, int64_t cols, const float* scale,

@@ -57,6 +57,9 @@ __device__ int g_status;
 
 bool pdl_enabled() { return g_pdl.load() != 0; }
 
+std::atomic<int> g_fold_in_call{1};
+bool ring_fold_in_call() { return g_fold_in_call.load() != 0; }
+
 int fail(int code, const std::string& msg) {
     t_last_error = msg;
     return code;
@@ -233,6 +236,13 @@ int fp8_debug_stalled_wait(cudaStream_t stream) {
     if (rc) return rc;
     stalled_wait_kernel<<<1, 32, 0, stream>>>(ctl);
     return check_launch("stalled_wait_kernel");
+}
+
+int fp8_set_ring_fold_mode(int mode) {
+    clear_error();
+    if (mode != 0 && mode != 1) return fail(FP8DSA_ERR_INVALID_ARG, "mode must be 0 (fold in the call) or 1 (defer)");
+    g_fold_in_call.store(mode == 0 ? 1 : 0);
+    return FP8DSA_OK;
 }
 
 int fp8_set_gemm_split_k(int splits) {

@@ -80,6 +80,25 @@ int fp8_scale_ring_init(float* state, int hist_len, cudaStream_t stream);
 int fp8_scale_ring_seed(const fp8_ring_t* ring, const void* x, fp8_in_t in_type, int64_t numel,
                         cudaStream_t stream);
 
+/* Data-parallel scaling (the pages measure one GPU; this is the standard extension where every
+ * rank's rings must agree): with fp8_set_ring_fold_mode(1) the linear entries leave each ring's
+ * measured amax in its amax slot instead of folding it.  At the end of a step the caller
+ *   1. gathers the slots: fp8_scale_ring_collect_amax(rings, n, amax) -- amax: dev fp32 [n];
+ *   2. reduces amax over the ranks with MAX (e.g. an NCCL all-reduce);
+ *   3. folds every ring with the reduced values: fp8_scale_ring_fold(rings, n, amax) --
+ *      hist[hist_idx] = amax[i], scale_used = the current scale, scale = the formula over the
+ *      window, amax slot zeroed (amax == NULL folds each ring's own slot).
+ * rings: host array of n descriptors (hist_idx = the slot the step's quantize used); n >= 0.
+ * Both run one launch per 128 rings. */
+int fp8_scale_ring_collect_amax(const fp8_ring_t* rings, int n, float* amax_out, cudaStream_t stream);
+int fp8_scale_ring_fold(const fp8_ring_t* rings, int n, const float* amax, cudaStream_t stream);
+
+/* 0 (default): linear_forward_fp8 / _keep / _noalloc, linear_backward_fp8 and _mixed fold the
+ * rings they quantize with, inside the call.  1: they leave the measured amax in each ring's
+ * amax slot for fp8_scale_ring_fold (data-parallel training, see above).  Other values:
+ * FP8DSA_ERR_INVALID_ARG.  Applies to later calls.  Not on the pages. */
+int fp8_set_ring_fold_mode(int mode);
+
 /* Dynamic (current-amax) step [compare: astrai/extension/fp8.py, _dynamic_scale]:
  * *scale_out = max(RN32(max|x| / fp8_max) / pow2_margin, 1e-12) and, if amax_out is not
  * NULL, *amax_out = max|x|.  scratch: dev, 16 bytes, 16-byte aligned, all zero before the

@@ -159,6 +159,13 @@ def test_misc_argument_checks():
     assert lib.fp8_set_gemm_split_k(-1) == INVALID
     assert lib.fp8_set_gemm_split_k(5) == INVALID
     assert lib.fp8_set_gemm_split_k(0) == 0
+    assert lib.fp8_set_ring_fold_mode(2) == INVALID
+    assert lib.fp8_set_ring_fold_mode(0) == 0
+    bad = (F.fp8_ring_t * 2)(F.fp8_ring_t(256, 16, 0, 448.0, 1.0), F.fp8_ring_t(256, 0, 0, 448.0, 1.0))
+    assert lib.fp8_scale_ring_fold(bad, 2, None, None) == INVALID          # second ring: hist_len 0
+    assert lib.fp8_scale_ring_collect_amax(bad, 1, None, None) == INVALID  # no output
+    assert lib.fp8_scale_ring_fold(None, 3, None, None) == INVALID
+    assert lib.fp8_scale_ring_fold(None, 0, None, None) == 0               # nothing to fold
     assert lib.fp8_set_gemm_split_k(1) == 0
     ring = F.Ring(None, 4)
     for _ in range(5):
