@@ -115,3 +115,19 @@ def gemm_entry(a_stored, b_stored, layout, fmt_a, fmt_b, sa, sb, bias, bias_scal
     if bv is not None:
         ref += float(bv[j])
     return ref, float(np.sum(np.abs(prod))), sc
+
+
+def gemm_fp8_out(a_stored, b_stored, layout="NT", fmt_a="e4m3", fmt_b="e4m3", sa=1.0, sb=1.0,
+                 bias=None, bias_scale=None, out8_fmt="e4m3", out8_step=1.0):
+    """The GEMM whose epilogue also quantizes its output (the FP8-output GEMM of an earlier
+    state of the pages' epilogue, read as "quantize the bf16 output"): ``y = RN_bf16(ref)``
+    as in :func:`gemm_bf16`, then ``out8 = q(RN32(y * RN32(1/out8_step)))`` and
+    ``amax = max |y|`` -- the same bytes and amax the quantize gives for ``y``.
+
+    Returns ``(ref64, s_abs, sc, y_bits, out8_codes, amax)``."""
+    from .fp8_codec import f64_to_bf16_bits, bf16_bits_to_f64
+    from .quantize import amax as amax_of, quantize_values
+    ref, s_abs, sc = gemm_ref(a_stored, b_stored, layout, fmt_a, fmt_b, sa, sb, bias, bias_scale)
+    y_bits = f64_to_bf16_bits(ref)
+    y = bf16_bits_to_f64(y_bits).astype(np.float32)
+    return ref, s_abs, sc, y_bits, quantize_values(y, out8_step, out8_fmt), amax_of(y)

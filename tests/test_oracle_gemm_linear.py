@@ -251,3 +251,39 @@ def test_backward_mixed_with_one_format_is_the_backward():
     for key in ("dx", "dw", "dx_abs", "dw_abs"):
         assert np.array_equal(ref[key], mix[key]), key
     assert np.array_equal(ref["grad_b"], mix["grad_b"])
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_fp8_output_gemm_one_hot_returns_the_codes(fmt):
+    """A one-hot A with unit scales copies rows of B into the output: every output is an fp8
+    value of B's format, exactly representable in bf16, so quantizing it with step 1 in the
+    same format must give back B's codes (signed zeros included) and the amax of those rows."""
+    rng = np.random.default_rng(12)
+    m, k, n = 9, 16, 24
+    b = _rand_codes(rng, (k, n), fmt)
+    pick = rng.integers(0, k, size=m)
+    a = np.full((m, k), 0x00, np.uint8)  # +0
+    one = 0x38 if fmt == "e4m3" else 0x3C  # the code of 1.0
+    a[np.arange(m), pick] = one
+    ref, s_abs, sc, y_bits, out8, am = G.gemm_fp8_out(a, b, "NN", fmt, fmt, 1.0, 1.0, None, None, fmt, 1.0)
+    want = b[pick]
+    assert np.array_equal(out8, want)
+    assert np.float32(am) == np.float32(np.max(np.abs(C.decode(want, fmt))))
+    assert np.array_equal(C.bf16_bits_to_f64(y_bits), C.decode(want, fmt))
+
+
+def test_fp8_output_gemm_is_the_quantized_bf16_output():
+    """The fp8 output is the quantize of the bf16 output at out8_step (any scales, bias)."""
+    rng = np.random.default_rng(13)
+    a = _rand_codes(rng, (20, 48), "e4m3")
+    b = _rand_codes(rng, (48, 32), "e4m3")
+    bias = C.f64_to_bf16_bits(rng.standard_normal(32))
+    ref, s_abs, sc, y_bits, out8, am = G.gemm_fp8_out(a, b, "NN", "e4m3", "e4m3", 0.02, 0.5, bias, None, "e5m2", 0.37)
+    y = C.bf16_bits_to_f64(y_bits)
+    assert np.array_equal(y, C.round_to_bf16(ref))
+    mult = Q.reciprocal_f32(0.37)
+    for i in (0, 7, 19):
+        for j in (0, 5, 31):
+            prod = np.float32(np.float32(y[i, j]) * mult)
+            assert out8[i, j] == C.encode(np.array([prod], np.float64), "e5m2")[0]
+    assert np.float32(am) == np.float32(np.max(np.abs(y)))
