@@ -45,6 +45,8 @@ _SIGNATURES = {
     "fp8_quantize_dual": (c_int, [_P, c_int, c_int64, c_int64, _P, c_int, _P, _P, _P, POINTER(fp8_ring_t), _P]),
     "fp8_gemm": (c_int, [_P, _P, c_int, c_int, c_int, c_int64, c_int64, c_int64, c_int64, c_int64, c_int64,
                          c_int64, c_int64, c_int64, c_int64, _P, _P, _P, _P, _P, _P]),
+    "fp8_gemm_fp8out": (c_int, [_P, _P, c_int, c_int, c_int, c_int64, c_int64, c_int64, c_int64, c_int64, c_int64,
+                                c_int64, c_int64, c_int64, c_int64, _P, _P, _P, _P, _P, c_int, _P, _P, _P, _P, _P]),
     "linear_forward_fp8_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_forward_fp8": (c_int, [_P, _P, c_int, _P, _P, _P, c_int64, c_int64, c_int64, c_int,
                                    POINTER(fp8_ring_t), POINTER(fp8_ring_t), c_float, _P, _P, _P, c_size_t, _P, _P]),
@@ -196,6 +198,16 @@ def fp8_gemm(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a
                                              int(k), int(lda), int(ldb), int(ldo), int(batch), int(stride_a),
                                              int(stride_b), int(stride_o), _ptr(scale_a), _ptr(scale_b), _ptr(bias),
                                              _ptr(bias_scale), _ptr(out), _stream(stream)))
+
+
+def fp8_gemm_fp8out(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
+                    scale_a, scale_b, bias, bias_scale, out, out8_fmt, out8_step, out8, out8_amax=None,
+                    out8_step_used=None, stream=None):
+    return _check("fp8_gemm_fp8out", lib().fp8_gemm_fp8out(
+        _ptr(a), _ptr(b), int(fmt_a), int(fmt_b), int(layout), int(m), int(n), int(k), int(lda), int(ldb), int(ldo),
+        int(batch), int(stride_a), int(stride_b), int(stride_o), _ptr(scale_a), _ptr(scale_b), _ptr(bias),
+        _ptr(bias_scale), _ptr(out), int(out8_fmt), _ptr(out8_step), _ptr(out8), _ptr(out8_amax),
+        _ptr(out8_step_used), _stream(stream)))
 
 
 def linear_forward_fp8_workspace_size(m, k, n) -> int:

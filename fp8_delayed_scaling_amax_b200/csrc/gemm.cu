@@ -94,6 +94,13 @@ struct GemmProblem {
     const float* bias_scale;
     const float* scale_a;
     const float* scale_b;
+    // fp8 output (see GemmDesc): null = none
+    uint8_t* out8;
+    int out8_fmt;
+    int out8_vec;  // out8, ldo and stride_o allow 16-byte stores
+    const float* out8_step;
+    float* out8_amax;
+    float* out8_step_used;
 };
 
 // Optional side job of the epilogue warps, done before their first tile: the bias gradient
@@ -235,7 +242,7 @@ __device__ __forceinline__ float bias_value(const GemmProblem& P, int col, float
     return __fmul_rn(P.bias_kind == 2 ? fp8_to_float<0>(v) : fp8_to_float<1>(v), bsc);
 }
 
-template <int BN, bool kPair, bool kSplit>
+template <int BN, bool kPair, bool kSplit, bool kOut8>
 __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a0, const __grid_constant__ CUtensorMap tma_b0,
                     const __grid_constant__ CUtensorMap tma_o0, const __grid_constant__ CUtensorMap tma_a1,
@@ -501,7 +508,20 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 bsc[i] = g.p[i].bias_kind >= 2 ? __ldg(g.p[i].bias_scale) : 0.0f;
             }
         }
+        // fp8 output: the multiplier RN32(1 / step) per problem, and the step snapshot
+        float mult8[kMaxProblems];
+#pragma unroll
+        for (int i = 0; i < kMaxProblems; ++i) {
+            mult8[i] = 0.0f;
+            if (kOut8 && i < g.nprob && g.p[i].out8 != nullptr) {
+                const float step8 = __ldg(g.p[i].out8_step);
+                mult8[i] = __frcp_rn(step8);
+                if (g.p[i].out8_step_used != nullptr && blockIdx.x == 0 && ew == 0 && lane == 0)
+                    *g.p[i].out8_step_used = step8;
+            }
+        }
         const uint32_t acc_empty_leader0 = kPair ? mapa_shared(smem_addr(acc_empty), 0) : 0u;
+        uint32_t am8 = 0u;  // running |max| of this thread's fp8-output values (bf16x2)
         int acc = 0, buf = 0;
         uint32_t acc_phase = 0;
         constexpr int kCtas = kPair ? 2 : 1;
@@ -615,7 +635,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                         bulk_commit_group();
                     }
                     buf ^= 1;
-                } else if (row < P.m && colg < P.n) {
+                } else if (P.out != nullptr && row < P.m && colg < P.n) {
                     uint16_t* orow = P.out + static_cast<int64_t>(b) * P.stride_o + row * P.ldo;
                     if (P.vec_out && colg + kOutBox <= P.n) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + colg);
@@ -628,6 +648,55 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                             if (colg + e < P.n) orow[colg + e] = static_cast<uint16_t>(packed[e >> 1] >> (16 * (e & 1)));
                     }
                 }
+                if (kOut8 && P.out8 != nullptr && row < P.m && colg < P.n) {
+                    // the same bf16 values, quantized: q(RN32(v * mult8)); amax over the valid ones
+                    const float m8 = pi ? mult8[1] : mult8[0];
+                    uint32_t q8[16];
+#pragma unroll
+                    for (int qd = 0; qd < 8; ++qd) {
+                        uint32_t wv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            wv[e] = packed[4 * qd + e];
+                            // columns past n hold no output: keep them out of the amax
+                            const int col = colg + 8 * qd + 2 * e;
+                            if (col >= P.n) wv[e] = 0u;
+                            else if (col + 1 >= P.n) wv[e] &= 0xFFFFu;
+                        }
+                        am8 = max_abs_bf16x2(max_abs_bf16x2(am8, wv[0]), max_abs_bf16x2(wv[1], max_abs_bf16x2(wv[2], wv[3])));
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            f[2 * e] = __uint_as_float(packed[4 * qd + e] << 16);
+                            f[2 * e + 1] = __uint_as_float(packed[4 * qd + e] & 0xFFFF0000u);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) mul2_rn(f[e], f[e + 1], m8);
+                        if (P.out8_fmt == 0) {
+                            q8[2 * qd] = cvt_fp8x4<0>(f[0], f[1], f[2], f[3]);
+                            q8[2 * qd + 1] = cvt_fp8x4<0>(f[4], f[5], f[6], f[7]);
+                        } else {
+                            q8[2 * qd] = cvt_fp8x4<1>(f[0], f[1], f[2], f[3]);
+                            q8[2 * qd + 1] = cvt_fp8x4<1>(f[4], f[5], f[6], f[7]);
+                        }
+                    }
+                    uint8_t* orow8 = P.out8 + static_cast<int64_t>(b) * P.stride_o + row * P.ldo;
+                    if (P.out8_vec && colg + kOutBox <= P.n) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow8 + colg);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(q8[4 * v], q8[4 * v + 1], q8[4 * v + 2], q8[4 * v + 3]);
+                    } else {
+                        for (int e = 0; e < kOutBox && colg + e < P.n; ++e)
+                            orow8[colg + e] = static_cast<uint8_t>(q8[e >> 2] >> (8 * (e & 3)));
+                    }
+                }
+            }
+            if (kOut8 && P.out8 != nullptr && P.out8_amax != nullptr) {
+                // this warp's share of the tile's amax: one atomic per warp and tile
+                float v = fmaxf(fabsf(__uint_as_float(am8 << 16)), fabsf(__uint_as_float(am8 & 0xFFFF0000u)));
+                v = warp_max(v);
+                if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(P.out8_amax), __float_as_uint(v));
+                am8 = 0u;
             }
             tc_fence_before_sync();
             if constexpr (kPair) {
@@ -821,14 +890,14 @@ void plan_units(GemmArgs& g, int units, int64_t max_contrib, int64_t counter_wor
 
 // One-time set-up of a kernel instance: its shared-memory limit and (pairs) how many
 // 2-CTA clusters fit on the device at once.
-template <int BN, bool kPair, bool kSplit>
+template <int BN, bool kPair, bool kSplit, bool kOut8>
 cudaError_t kernel_setup(int* max_units_out) {
     using C = Cfg<BN, kPair>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     static int max_units = 0;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, kSplit, kOut8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::kSmem);
         if (attr_err != cudaSuccess) return;
         if (kPair) {
@@ -845,7 +914,7 @@ cudaError_t kernel_setup(int* max_units_out) {
             cfg.attrs = at;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, kPair, kSplit>, &cfg) == cudaSuccess && n > 0)
+            if (cudaOccupancyMaxActiveClusters(&n, fp8_gemm_kernel<BN, kPair, kSplit, kOut8>, &cfg) == cudaSuccess && n > 0)
                 max_units = n;
             cudaGetLastError();
         }
@@ -859,7 +928,7 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
                cudaStream_t stream) {
     using C = Cfg<BN, kPair>;
     int max_units = 0;
-    const cudaError_t attr_err = kernel_setup<BN, kPair, false>(&max_units);
+    const cudaError_t attr_err = kernel_setup<BN, kPair, false, false>(&max_units);
     if (attr_err != cudaSuccess)
         return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(attr_err));
     int64_t tiles = 0;
@@ -884,10 +953,24 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
     } else {
         plan_units(g, units, 0, 0);
     }
-    auto kernel = fp8_gemm_kernel<BN, kPair, false>;
-    if (g.splitk) {
+    bool out8 = false;
+    for (int i = 0; i < g.nprob; ++i) out8 = out8 || g.p[i].out8 != nullptr;
+    if (out8 && g.splitk) {  // the fp8-output instance has no split-K: one range per tile
+        g.partial = nullptr;
+        g.counters = nullptr;
+        plan_units(g, units, 0, 0);
+    }
+    auto kernel = fp8_gemm_kernel<BN, kPair, false, false>;
+    if (out8) {
+        int o8_units = 0;
+        const cudaError_t oe = kernel_setup<BN, kPair, false, true>(&o8_units);
+        if (oe != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(oe));
+        if (kPair && o8_units > 0 && o8_units < units)
+            return fail(FP8DSA_ERR_CUDA, "fp8-output GEMM instance fits fewer clusters than the plan");
+        kernel = fp8_gemm_kernel<BN, kPair, false, true>;
+    } else if (g.splitk) {
         int split_units = 0;
-        const cudaError_t se = kernel_setup<BN, kPair, true>(&split_units);
+        const cudaError_t se = kernel_setup<BN, kPair, true, false>(&split_units);
         if (se != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(se));
         // both instances must have every cluster of the plan resident at once
         if (kPair && split_units > 0 && split_units < units) {
@@ -895,7 +978,7 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
             g.counters = nullptr;
             plan_units(g, units, 0, 0);
         } else {
-            kernel = fp8_gemm_kernel<BN, kPair, true>;
+            kernel = fp8_gemm_kernel<BN, kPair, true, false>;
         }
     }
     const int grid_units = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g.num_units, units)));
@@ -1050,7 +1133,8 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
             rc = make_map(&mb, u8, d.b, d.n, d.k, b_bat ? d.batch : 1, d.ldb, b_bat ? d.stride_b : d.ldb * d.k, 128, kBK);
         if (rc) return rc;
         // TMA stores need 16-byte aligned rows and batches of the output
-        const bool tma_out = aligned16(d.out) && d.ldo % 8 == 0 && (d.batch == 1 || d.stride_o % 8 == 0);
+        const bool tma_out = d.out != nullptr && aligned16(d.out) && d.ldo % 8 == 0 &&
+                             (d.batch == 1 || d.stride_o % 8 == 0);
         if (tma_out) {
             rc = make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d.out, d.n, d.m, d.batch, d.ldo * 2,
                           d.batch > 1 ? d.stride_o * 2 : d.ldo * 2 * d.m, kOutBox, 32);
@@ -1078,6 +1162,12 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
         P.bias_scale = d.bias_scale;
         P.scale_a = d.scale_a;
         P.scale_b = d.scale_b;
+        P.out8 = d.out8;
+        P.out8_fmt = d.out8_fmt;
+        P.out8_vec = d.out8 != nullptr && aligned16(d.out8) && d.ldo % 16 == 0 && (d.batch == 1 || d.stride_o % 16 == 0);
+        P.out8_step = d.out8_step;
+        P.out8_amax = d.out8_amax;
+        P.out8_step_used = d.out8_step_used;
         batch[i] = d.batch;
     }
     for (int i = nwork; i < kMaxProblems; ++i) maps[3 * i] = maps[3 * i + 1] = maps[3 * i + 2] = maps[0];
@@ -1122,24 +1212,32 @@ int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_
 
 using namespace fp8dsa;
 
-extern "C" int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b, fp8_layout_t layout,
-                        int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch,
-                        int64_t stride_a, int64_t stride_b, int64_t stride_o, const float* scale_a,
-                        const float* scale_b, const void* bias, const float* bias_scale, void* out,
-                        cudaStream_t stream) {
-    clear_error();
+namespace {
+
+// fp8_gemm / fp8_gemm_fp8out: argument checks, then one GEMM launch.  out8 == null: bf16 only.
+int gemm_entry(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b, fp8_layout_t layout, int64_t m,
+               int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch, int64_t stride_a,
+               int64_t stride_b, int64_t stride_o, const float* scale_a, const float* scale_b, const void* bias,
+               const float* bias_scale, void* out, fp8_fmt_t out8_fmt, const float* out8_step, uint8_t* out8,
+               float* out8_amax, float* out8_step_used, cudaStream_t stream) {
     if (!valid_fmt(fmt_a) || !valid_fmt(fmt_b)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (layout < FP8_LAYOUT_NT || layout > FP8_LAYOUT_TT) return fail(FP8DSA_ERR_INVALID_ARG, "bad layout");
     if (m < 0 || n < 0 || k < 0 || batch < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
     if (m > 0x7FFFFFFF || n > 0x7FFFFFFF || k > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "sizes must be < 2^31");
     if (batch > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "batch must be < 2^31");
-    if (out == nullptr || scale_a == nullptr || scale_b == nullptr)
-        return fail(FP8DSA_ERR_INVALID_ARG, "out, scale_a and scale_b are required");
+    if ((out == nullptr && out8 == nullptr) || scale_a == nullptr || scale_b == nullptr)
+        return fail(FP8DSA_ERR_INVALID_ARG, "an output, scale_a and scale_b are required");
     if (bias == nullptr && bias_scale != nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "bias_scale without bias");
     if (ldo < n) return fail(FP8DSA_ERR_INVALID_ARG, "ldo must be >= n");
     if (batch > 1 && stride_o < ldo * m && stride_o != 0 && m > 1)
         return fail(FP8DSA_ERR_INVALID_ARG, "stride_o overlaps batches");
     if (batch > 1 && stride_o == 0 && m > 0 && n > 0) return fail(FP8DSA_ERR_INVALID_ARG, "stride_o must be non-zero when batch > 1");
+    if (out8 != nullptr) {
+        if (!valid_fmt(out8_fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "out8_fmt must be FP8_E4M3 or FP8_E5M2");
+        if (out8_step == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out8 needs out8_step");
+        if (k == 0 && m > 0 && n > 0 && batch > 0)
+            return fail(FP8DSA_ERR_UNSUPPORTED, "the fp8 output needs k > 0");
+    }
     const int a_mn = (layout == FP8_LAYOUT_TN || layout == FP8_LAYOUT_TT) ? 1 : 0;
     const int b_mn = (layout == FP8_LAYOUT_NN || layout == FP8_LAYOUT_TN) ? 1 : 0;
     if (m > 0 && n > 0 && batch > 0 && k > 0) {
@@ -1157,6 +1255,37 @@ extern "C" int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8
     if (rc) return rc;
     int bias_kind = 0;
     if (bias != nullptr) bias_kind = bias_scale == nullptr ? 1 : (fmt_a == FP8_E4M3 ? 2 : 3);
-    return gemm_launch(a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
-                       scale_a, scale_b, bias, bias_kind, bias_scale, out, stream);
+    GemmDesc d{a, b, fmt_a, fmt_b, a_mn, b_mn, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o,
+               scale_a, scale_b, bias, bias_kind, bias_scale, out};
+    d.out8 = out8;
+    d.out8_fmt = out8_fmt;
+    d.out8_step = out8_step;
+    d.out8_amax = out8_amax;
+    d.out8_step_used = out8_step_used;
+    return gemm_launch_group(&d, 1, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, stream);
+}
+
+}  // namespace
+
+extern "C" int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b, fp8_layout_t layout,
+                        int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb, int64_t ldo, int64_t batch,
+                        int64_t stride_a, int64_t stride_b, int64_t stride_o, const float* scale_a,
+                        const float* scale_b, const void* bias, const float* bias_scale, void* out,
+                        cudaStream_t stream) {
+    clear_error();
+    if (out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out, scale_a and scale_b are required");
+    return gemm_entry(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o, scale_a,
+                      scale_b, bias, bias_scale, out, FP8_E4M3, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+extern "C" int fp8_gemm_fp8out(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b,
+                               fp8_layout_t layout, int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb,
+                               int64_t ldo, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_o,
+                               const float* scale_a, const float* scale_b, const void* bias,
+                               const float* bias_scale, void* out, fp8_fmt_t out8_fmt, const float* out8_step,
+                               uint8_t* out8, float* out8_amax, float* out8_step_used, cudaStream_t stream) {
+    clear_error();
+    if (out8 == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out8 is required");
+    return gemm_entry(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o, scale_a,
+                      scale_b, bias, bias_scale, out, out8_fmt, out8_step, out8, out8_amax, out8_step_used, stream);
 }

@@ -150,7 +150,15 @@ struct GemmDesc {
     const void* bias;
     int bias_kind;
     const float* bias_scale;
-    void* out;
+    void* out;  // bf16 output, or null when only out8 is wanted
+    // optional fp8 output of the same values: out8 = q(RN32(RN_bf16(v) * RN32(1 / *out8_step))),
+    // same element strides as out; |RN_bf16(v)| atomically maxed into *out8_amax (if not null);
+    // *out8_step written to *out8_step_used (if not null)
+    uint8_t* out8 = nullptr;
+    int out8_fmt = 0;
+    const float* out8_step = nullptr;
+    float* out8_amax = nullptr;
+    float* out8_step_used = nullptr;
 };
 
 // Split-K scratch a GEMM launch may use (see gemm_launch_group): fp32 partial tiles and one

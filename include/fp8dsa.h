@@ -153,6 +153,26 @@ int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_
              const float* scale_a, const float* scale_b, const void* bias,
              const float* bias_scale, void* out, cudaStream_t stream);
 
+/* fp8_gemm whose epilogue also quantizes its output for the next consumer (the quantize fused
+ * into the producer; the pages' FP8-output GEMM, which their final state dropped, is the
+ * closest counterpart) [compare: csrc/kernels/fp8/gemm/epilogue.cuh, out_dtype / out_scale in
+ * an earlier state]:
+ *   every output element v = acc * RN32(sa*sb) + bias is rounded to bf16 as in fp8_gemm, then
+ *       out8 = q_{out8_fmt}(RN32(RN_bf16(v) * RN32(1 / *out8_step)))   (RN, saturating)
+ *   i.e. exactly the bytes fp8_quantize gives for the bf16 output; |RN_bf16(v)| over the valid
+ *   elements is atomically maxed into *out8_amax (dev fp32; not zeroed here -- pass a zeroed
+ *   value, or a ring's amax slot and fold later with fp8_scale_ring_fold); *out8_step is
+ *   copied to *out8_step_used (may be NULL) for the consumer's dequantization.
+ *   out: bf16 output as in fp8_gemm, or NULL to write only out8.  out8: dev bytes with the
+ *   same element strides as out (ldo, stride_o).  out8_step: dev fp32 (e.g. a ring's step).
+ *   k must be > 0.  Not on the pages in their final state. */
+int fp8_gemm_fp8out(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fmt_b,
+                    fp8_layout_t layout, int64_t m, int64_t n, int64_t k, int64_t lda, int64_t ldb,
+                    int64_t ldo, int64_t batch, int64_t stride_a, int64_t stride_b, int64_t stride_o,
+                    const float* scale_a, const float* scale_b, const void* bias,
+                    const float* bias_scale, void* out, fp8_fmt_t out8_fmt, const float* out8_step,
+                    uint8_t* out8, float* out8_amax, float* out8_step_used, cudaStream_t stream);
+
 /* Workspace bytes linear_forward_fp8 needs for (m, k, n): x8, w8 and scale scratch, then the
  * GEMM's split-K region (arrival counters and fp32 partial tiles for up to 4 K ranges per
  * output tile; used only where splitting shortens the schedule). */
