@@ -389,6 +389,40 @@ def time_gemm(F, W, torch, dev, m, n, k, iters=20, warmup=5, batch=1, bcast_b=Fa
     return {"ms": ms, "tflops": 2.0 * batch * m * n * k / (ms * 1e-3) / 1e12, "sets": nsets}
 
 
+def time_fp8_output(F, W, torch, dev, m, n, k, fused, iters=20, warmup=5):
+    """The producer-side quantize of a GEMM output: fused (fp8_gemm_fp8out writing only the fp8
+    bytes, amax into a ring slot) or as two launches (fp8_gemm to bf16, then fp8_quantize of that
+    output folding a ring)."""
+    per_set = m * k + n * k + m * n * 3
+    nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
+    sets = []
+    for i in range(nsets):
+        a = W.fp8_bytes((m, k), seed=131 + i, device=dev)
+        b = W.fp8_bytes((n, k), seed=157 + i, device=dev)
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        out8 = torch.empty((m, n), dtype=torch.uint8, device=dev)
+        st = torch.zeros(HIST + 4, dtype=torch.float32, device=dev)
+        F.fp8_scale_ring_init(st, HIST)
+        st[HIST] = 1.0 / 64
+        sets.append((a, b, out, out8, st, F.Ring(st, HIST, F.FP8_E4M3)))
+    sa = torch.tensor([0.75], device=dev)
+    sb = torch.tensor([1.5], device=dev)
+    bias = W.normal_bf16((n,), 0.1, seed=5, device=dev)
+    used = torch.zeros(1, device=dev)
+
+    def launch(i):
+        a, b, out, out8, st, ring = sets[i % nsets]
+        if fused:
+            F.fp8_gemm_fp8out(a, b, 0, 0, F.FP8_LAYOUT_NT, m, n, k, k, k, n, 1, 0, 0, 0, sa, sb, bias, None, None,
+                              F.FP8_E4M3, st[HIST:HIST + 1], out8, st[HIST + 2:HIST + 3], used)
+        else:
+            F.fp8_gemm(a, b, 0, 0, F.FP8_LAYOUT_NT, m, n, k, k, k, n, 1, 0, 0, 0, sa, sb, bias, None, out)
+            F.fp8_quantize(out, F.FP8_IN_BF16, m, n, st[HIST:HIST + 1], F.FP8_E4M3, 0, out8, None, ring)
+
+    ms = _graph_time(torch, launch, iters, warmup)
+    return {"ms": ms, "tflops": 2.0 * m * n * k / (ms * 1e-3) / 1e12}
+
+
 def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5):
     per_set = rows * cols * (2 + (2 if mode == "dual" else 1))
     nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
@@ -447,7 +481,7 @@ def run_sweeps(F, W, torch, dev):
     quantize bandwidth sweep, each timed alone with operands rotated through HBM."""
     peaks = measured_peaks()
     burst_fp8 = 2.0 * peaks["bf16_tflops"]
-    out = {"gemm_square": {}, "gemm_skinny_batched": {}, "quantize": {}}
+    out = {"gemm_square": {}, "gemm_skinny_batched": {}, "quantize": {}, "gemm_fp8_output": {}}
     for s in W.SQUARE_SIZES:
         r = time_gemm(F, W, torch, dev, s, s, s, iters=20 if s < 8192 else 10)
         out["gemm_square"][str(s)] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
@@ -463,6 +497,12 @@ def run_sweeps(F, W, torch, dev):
             r = time_quantize(F, W, torch, dev, rows, cols, mode)
             out["quantize"][f"{mode}_{rows}x{cols}"] = {"gbs": round(r["gbs"], 1), "us": round(r["ms"] * 1e3, 2),
                                                        "frac": round(r["gbs"] / peaks["hbm_gbs"], 4)}
+    for m, n, k in ((2048, 3072, 1024), (2048, 4096, 1024), (4096, 4096, 4096)):
+        fused = time_fp8_output(F, W, torch, dev, m, n, k, True)
+        split = time_fp8_output(F, W, torch, dev, m, n, k, False)
+        out["gemm_fp8_output"][f"{m}x{n}x{k}"] = {"fused_us": round(fused["ms"] * 1e3, 2),
+                                                  "gemm_then_quantize_us": round(split["ms"] * 1e3, 2),
+                                                  "fused_tflops": round(fused["tflops"], 1)}
     out["peaks"] = {"fp8_tflops_burst": burst_fp8, "hbm_gbs": peaks["hbm_gbs"], "source": peaks["source"]}
     return out
 

@@ -146,6 +146,23 @@ def test_keep_forward_and_mixed_backward_argument_checks():
     assert call(margin=0.0) == INVALID       # dynamic scaling needs a positive margin
 
 
+def test_fp8_output_gemm_argument_checks():
+    lib = F.lib()
+    g8 = lib.fp8_gemm_fp8out
+    # out8 required; out8_step required; bad out8 format; k = 0 with an fp8 output
+    assert g8(16, 16, 0, 0, 0, 64, 64, 64, 64, 64, 64, 1, 0, 0, 0, 256, 256, None, None, 1024, 0, 512, None, None,
+              None, None) == INVALID
+    assert g8(16, 16, 0, 0, 0, 64, 64, 64, 64, 64, 64, 1, 0, 0, 0, 256, 256, None, None, 1024, 0, None, 2048, None,
+              None, None) == INVALID
+    assert g8(16, 16, 0, 0, 0, 64, 64, 64, 64, 64, 64, 1, 0, 0, 0, 256, 256, None, None, 1024, 7, 512, 2048, None,
+              None, None) == INVALID
+    assert g8(16, 16, 0, 0, 0, 64, 64, 0, 64, 64, 64, 1, 0, 0, 0, 256, 256, None, None, None, 0, 512, 2048, None,
+              None, None) == UNSUPPORTED
+    # fp8_gemm itself still requires its bf16 output
+    assert lib.fp8_gemm(16, 16, 0, 0, 0, 64, 64, 64, 64, 64, 64, 1, 0, 0, 0, 256, 256, None, None, None,
+                        None) == INVALID
+
+
 def test_misc_argument_checks():
     lib = F.lib()
     assert lib.fp8_set_wait_timeout_ns(0) == INVALID
