@@ -188,12 +188,21 @@ __device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
 
 constexpr int kHistPrefetch = 64;
 
-// Called at kernel start: copy the ring's history window (it does not change during the
-// kernel; only the last block writes it, at the very end) into shared memory, so the fold
-// does not pay one dependent L2 round trip per slot.  Visible after the next barrier.
-__device__ __forceinline__ void ring_prefetch(const QArgs& a, float* hist) {
-    if (a.ring_state != nullptr && a.hist_len <= kHistPrefetch && static_cast<int>(threadIdx.x) < a.hist_len)
-        hist[threadIdx.x] = __ldcg(a.ring_state + threadIdx.x);
+// The fold needs the ring's history window, which does not change during the kernel (only
+// the last block writes it, at the very end).  ring_peek, called after the PDL wait, starts the
+// load of slot threadIdx.x into a register; ring_stash puts it in shared memory just before the
+// final barrier, so the load's latency hides behind the kernel's work instead of stalling the
+// first warp, and the fold pays no dependent L2 round trip per slot.  A deferred fold (done by
+// the kernel that follows) needs no window.
+__device__ __forceinline__ bool ring_window_wanted(const QArgs& a) {
+    return a.ring_state != nullptr && !a.defer_fold && a.hist_len <= kHistPrefetch &&
+           static_cast<int>(threadIdx.x) < a.hist_len;
+}
+__device__ __forceinline__ float ring_peek(const QArgs& a) {
+    return ring_window_wanted(a) ? __ldcg(a.ring_state + threadIdx.x) : 0.0f;
+}
+__device__ __forceinline__ void ring_stash(const QArgs& a, float v, float* hist) {
+    if (ring_window_wanted(a)) hist[threadIdx.x] = v;
 }
 
 // One thread per block and tensor, with the block's amax `m`: one atomicMax, then (with a
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     const QArgs& a = batch.job[jb];
     const int64_t lb = static_cast<int64_t>(blockIdx.x) - a.tile_begin;  // block within the tensor
     __shared__ float s_hist[kHistPrefetch];
-    ring_prefetch(a, s_hist);
+    const float hist_v = ring_peek(a);
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
@@ -306,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
         amax = fmaxf(amax, fabsf(v));
         a.out[i] = convert1<kFmt>(v, mult);
     }
+    ring_stash(a, hist_v, s_hist);
     block_finish(a, amax, step, lb == 0, s_hist);
 }
 
@@ -388,11 +398,15 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
     pdl_trigger();
     pdl_wait();
     zero_side_job(batch);
+    // the window of each tensor this CTA may fold (one tile per CTA: only its own tensor)
+    float hist_v[kMaxJobs] = {0.0f, 0.0f, 0.0f};
+    const int own_job = kPersist ? 0 : tile_job(batch, static_cast<int>(blockIdx.x));
     if constexpr (kPersist) {
-        for (int jb = 0; jb < njobs; ++jb) ring_prefetch(batch.job[jb], s_hist[jb]);
+#pragma unroll
+        for (int jb = 0; jb < kMaxJobs; ++jb)
+            if (jb < njobs) hist_v[jb] = ring_peek(batch.job[jb]);
     } else {
-        const int jb = tile_job(batch, static_cast<int>(blockIdx.x));
-        ring_prefetch(batch.job[jb], s_hist[jb]);
+        hist_v[0] = ring_peek(batch.job[own_job]);
     }
 
     const int total = batch.tiles_total;
@@ -626,9 +640,16 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         am0 = warp_max(fmaxf(am0, fmaxf(am1, am2)));
         if (lane == 0) s_red[0][w] = am0;
     }
+    if constexpr (kPersist) {
+#pragma unroll
+        for (int jb = 0; jb < kMaxJobs; ++jb)
+            if (jb < njobs) ring_stash(batch.job[jb], hist_v[jb], s_hist[jb]);
+    } else {
+        ring_stash(batch.job[own_job], hist_v[0], s_hist[own_job]);
+    }
     __syncthreads();
     // Persistent: every CTA finishes every tensor.  One tile per CTA: only its own tensor.
-    if (t < njobs && (kPersist || t == tile_job(batch, static_cast<int>(blockIdx.x)))) {
+    if (t < njobs && (kPersist || t == own_job)) {
         const int row = kPersist ? t : 0;
         float m = s_red[row][0];
 #pragma unroll
