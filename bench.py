@@ -57,7 +57,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sweeps", action="store_true")
-    p.add_argument("--no-variants", action="store_true", help="skip the mixed-format backward variant")
+    p.add_argument("--no-variants", action="store_true", help="skip the variant steps")
+    p.add_argument("--path", default=STEP_PATH[0], choices=PATHS,
+                   help="headline step: x^T / w^T saved by the forward's quantize launch, or re-quantized "
+                        "by the backward's (identical numbers)")
     p.add_argument("--dp-fold", action="store_true",
                    help="fold the rings once per step after an amax all-reduce (always on with several GPUs)")
     p.add_argument("--kernel", default=None, choices=["gemm", "quantize"],
@@ -215,6 +218,32 @@ class Linear:
                                     F.FP8_E4M3, 1, 1, 1, self.steps[0:1], self.steps[1:2], self.rg, 1.0,
                                     self.steps[2:3], self.mws, self.mws_n, self.gx, self.gw, self.gb)
 
+    def fwd_save(self):
+        """Forward whose quantize launch also writes x^T / w^T (E5M2, the forward's steps)."""
+        F = self.F
+        if not hasattr(self, "x8t"):
+            import torch
+            self.x8t = torch.empty((self.k, self.m), dtype=torch.uint8, device=self.x.device)
+            self.w8t = torch.empty((self.k, self.n), dtype=torch.uint8, device=self.x.device)
+            self.sws_n = F.linear_backward_fp8_saved_t_workspace_size(self.m, self.k, self.n)
+            self.sws = torch.empty(self.sws_n, dtype=torch.uint8, device=self.x.device)
+        F.linear_forward_fp8_save_t(self.x, self.w, self.b, None, self.m, self.k, self.n, F.FP8_E4M3, F.FP8_E5M2,
+                                    self.rx, self.rw, self.steps[0:1], self.steps[1:2], self.x8t, self.w8t, self.fws,
+                                    self.fws_n, self.y)
+
+    def bwd_saved(self):
+        """Backward that quantizes only g and reads the forward's saved x^T / w^T."""
+        F = self.F
+        F.linear_backward_fp8_saved_t(self.g, self.x8t, self.w8t, self.m, self.k, self.n, F.FP8_E5M2, F.FP8_E5M2,
+                                      1, 1, 1, self.steps[0:1], self.steps[1:2], self.rg, 1.0, self.steps[2:3],
+                                      self.sws, self.sws_n, self.gx, self.gw, self.gb)
+
+    @property
+    def quant_bytes_saved(self):
+        m, k, n = self.m, self.k, self.n
+        # fwd: x, w in both orientations (2 B in, 1 + 1 B out); bwd: g dual (2 + 1 + 1)
+        return 4 * (m * k + n * k) + 4 * m * n
+
     @property
     def quant_bytes_mixed(self):
         m, k, n = self.m, self.k, self.n
@@ -240,15 +269,37 @@ def build_workload(F, W, torch, dev, seed_base):
     return lins
 
 
-def run_step(lins, slot, mixed=False):
+PATHS = ("saved", "requant")
+PATH_WHAT = {
+    "saved": "x^T / w^T (E5M2, the forward's steps) written by the forward's quantize launch; the backward "
+             "quantizes only g",
+    "requant": "the backward's quantize launch re-quantizes x^T / w^T (E5M2, the forward's steps) beside g",
+}
+STEP_PATH = ["saved"]  # the headline step's composition (--path)
+
+
+def run_step(lins, slot, mixed=False, path=None):
     """One training step: every linear's forward, then every backward in reverse order.
+    path "saved": the forward's quantize launch also writes x^T / w^T for the backward (same
+    bytes as re-quantizing them there); "requant": the backward re-quantizes x^T / w^T.
     mixed=True: the forward keeps x8 / w8 and the backward reuses them (E5M2 g only)."""
+    path = path or STEP_PATH[0]
     for lin in lins:
         lin.set_slot(slot)
     for lin in lins:
-        lin.fwd_keep() if mixed else lin.fwd()
+        if mixed:
+            lin.fwd_keep()
+        elif path == "saved":
+            lin.fwd_save()
+        else:
+            lin.fwd()
     for lin in reversed(lins):
-        lin.bwd_mixed() if mixed else lin.bwd()
+        if mixed:
+            lin.bwd_mixed()
+        elif path == "saved":
+            lin.bwd_saved()
+        else:
+            lin.bwd()
 
 
 # ---------------------------------------------------------------------------------------
@@ -532,9 +583,10 @@ def main():
     if args.gemm_split_k is not None:
         F.fp8_set_gemm_split_k(args.gemm_split_k)
 
+    STEP_PATH[0] = args.path
     lins = build_workload(F, W, torch, dev, seed_base=100000 * rank)
     flops_step = sum(l.gemm_flops for l in lins)
-    qbytes_step = sum(l.quant_bytes for l in lins)
+    qbytes_step = sum(l.quant_bytes_saved if args.path == "saved" else l.quant_bytes for l in lins)
 
     # Data parallel over several GPUs: the linears leave each ring's amax in its slot and, after
     # every step, the ranks reduce all rings' amax (one all-reduce MAX) and fold them, so every
@@ -599,48 +651,56 @@ def main():
     ms_max = float(ms_t.item())
     status = F.fp8_get_device_status()
 
-    # the mixed-format variant of the step (forward keeps x8 / w8, backward quantizes only g):
-    # its own graphs, warm-up and timed replays, reported beside the headline step
-    mixed = None
-    if not args.no_variants:
-        run_step(lins, counter[0] % HIST, mixed=True)
+    # variants of the step, each with its own graphs, warm-up and timed replays, reported beside
+    # the headline: the other composition of the same numbers, and the mixed-format backward
+    def time_variant(mixed_v, path_v):
+        run_step(lins, counter[0] % HIST, mixed=mixed_v, path=path_v)
         end_of_step(counter[0] % HIST)
         counter[0] += 1
         torch.cuda.synchronize()
-        mgraphs = []
+        vgraphs = []
         for slot in range(HIST):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap):
-                run_step(lins, slot, mixed=True)
-            mgraphs.append(g)
+                run_step(lins, slot, mixed=mixed_v, path=path_v)
+            vgraphs.append(g)
         torch.cuda.synchronize()
         for t in range(args.warmup):
-            mgraphs[counter[0] % HIST].replay()
+            vgraphs[counter[0] % HIST].replay()
             end_of_step(counter[0] % HIST)
             counter[0] += 1
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        msteps = max(3, args.steps // 2)
+        vsteps = max(3, args.steps // 2)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record()
-        for t in range(msteps):
-            mgraphs[counter[0] % HIST].replay()
+        for t in range(vsteps):
+            vgraphs[counter[0] % HIST].replay()
             end_of_step(counter[0] % HIST)
             counter[0] += 1
         s1.record()
         torch.cuda.synchronize()
-        mt = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        vt = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
         if world > 1:
-            dist.all_reduce(mt, op=dist.ReduceOp.MAX)
-        mms = float(mt.item())
-        mixed = {"ms_per_step": mms / msteps, "value": flops_step * msteps * world / (mms * 1e-3) / 1e12,
-                 "unit": UNIT, "steps": msteps,
-                 "quantize_bytes_per_step": sum(l.quant_bytes_mixed for l in lins),
-                 "device_status": F.fp8_get_device_status(),
-                 "what": "forward keeps its E4M3 x8 / w8; backward quantizes only g (E5M2, row-major + column "
-                         "sums) and reads x8 / w8 in place (mixed-format GEMMs); not the pages' HYBRID numerics"}
-        del mgraphs
+            dist.all_reduce(vt, op=dist.ReduceOp.MAX)
+        vms = float(vt.item())
+        del vgraphs
+        return {"ms_per_step": vms / vsteps, "value": flops_step * vsteps * world / (vms * 1e-3) / 1e12,
+                "unit": UNIT, "steps": vsteps, "device_status": F.fp8_get_device_status()}
+
+    variants = {}
+    if not args.no_variants:
+        other = "requant" if args.path == "saved" else "saved"
+        v = time_variant(False, other)
+        v["quantize_bytes_per_step"] = sum(l.quant_bytes if other == "requant" else l.quant_bytes_saved for l in lins)
+        v["what"] = PATH_WHAT[other] + " (the same numbers as the headline step)"
+        variants[f"path_{other}"] = v
+        v = time_variant(True, None)
+        v["quantize_bytes_per_step"] = sum(l.quant_bytes_mixed for l in lins)
+        v["what"] = ("forward keeps its E4M3 x8 / w8; backward quantizes only g (E5M2, row-major + column sums) "
+                     "and reads x8 / w8 in place (mixed-format GEMMs); not the pages' HYBRID numerics")
+        variants["mixed_backward"] = v
 
     # per-kernel durations: the same step captured again with the library's profiler on
     # (an event-record node on each side of every kernel), each of the 16 slot graphs
@@ -722,6 +782,7 @@ def main():
                    "linears_kn": [list(kn) for kn in W.TRAINING_LINEARS],
                    "l2": "inputs larger than L2: every layer has its own x, w, g (about 3 GB working set)",
                    "graphs": f"one CUDA graph per history slot ({HIST})",
+                   "path": PATH_WHAT[args.path],
                    "parallelism": (f"data parallel over {world} GPU(s): each rank its own batch, one all-reduce "
                                    f"(MAX) of every ring's amax per step" if use_dp else "single GPU")},
         "gemm_flops_per_step": flops_step, "quantize_bytes_per_step": qbytes_step,
@@ -739,8 +800,8 @@ def main():
     }
     if clocks:
         line["clocks"] = clocks
-    if mixed is not None:
-        line["variants"] = {"mixed_backward": mixed}
+    if variants:
+        line["variants"] = variants
     if e2e:
         line["e2e"] = e2e
     if world == 1 and not args.no_sweeps:

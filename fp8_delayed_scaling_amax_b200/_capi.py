@@ -62,6 +62,13 @@ _SIGNATURES = {
     "linear_backward_fp8_mixed": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int,
                                           c_int, _P, _P, POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P,
                                           _P]),
+    "linear_forward_fp8_save_t": (c_int, [_P, _P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int,
+                                          POINTER(fp8_ring_t), POINTER(fp8_ring_t), _P, _P, _P, _P, _P, c_size_t,
+                                          _P, _P]),
+    "linear_backward_fp8_saved_t_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
+    "linear_backward_fp8_saved_t": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int,
+                                            _P, _P, POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P,
+                                            _P]),
     "fp8_get_device_status": (c_int, [_P, POINTER(c_int)]),
     "fp8_set_wait_timeout_ns": (c_int, [c_uint64]),
     "fp8_debug_stalled_wait": (c_int, [_P]),
@@ -269,6 +276,30 @@ def linear_backward_fp8_mixed(g, x8, w8, m, k, n, fmt_g, fmt_x, fmt_w, need_grad
         int(bool(need_grad_x)), int(bool(need_grad_w)), int(bool(need_grad_b)), _ptr(sx), _ptr(sw), _ring(g_ring),
         float(pow2_margin), _ptr(sg_used), _ptr(workspace), int(workspace_bytes), _ptr(grad_x), _ptr(grad_w),
         _ptr(grad_b), _stream(stream)))
+
+
+def linear_forward_fp8_save_t(x, w, bias, bias_scale, m, k, n, fmt, fmt_t, x_ring, w_ring, sx_used, sw_used, x8t_out,
+                              w8t_out, workspace, workspace_bytes, y, stream=None):
+    """Delayed-scaling forward that also writes x^T / w^T in fmt_t (for
+    linear_backward_fp8_saved_t)."""
+    return _check("linear_forward_fp8_save_t", lib().linear_forward_fp8_save_t(
+        _ptr(x), _ptr(w), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n), int(fmt), int(fmt_t), _ring(x_ring),
+        _ring(w_ring), _ptr(sx_used), _ptr(sw_used), _ptr(x8t_out), _ptr(w8t_out), _ptr(workspace),
+        int(workspace_bytes), _ptr(y), _stream(stream)))
+
+
+def linear_backward_fp8_saved_t_workspace_size(m, k, n) -> int:
+    return int(lib().linear_backward_fp8_saved_t_workspace_size(int(m), int(k), int(n)))
+
+
+def linear_backward_fp8_saved_t(g, x8t, w8t, m, k, n, fmt, fmt_t, need_grad_x, need_grad_w, need_grad_b, sx, sw,
+                                g_ring, pow2_margin, sg_used, workspace, workspace_bytes, grad_x, grad_w, grad_b,
+                                stream=None):
+    return _check("linear_backward_fp8_saved_t", lib().linear_backward_fp8_saved_t(
+        _ptr(g), _ptr(x8t), _ptr(w8t), int(m), int(k), int(n), int(fmt), int(fmt_t), int(bool(need_grad_x)),
+        int(bool(need_grad_w)), int(bool(need_grad_b)), _ptr(sx), _ptr(sw), _ring(g_ring), float(pow2_margin),
+        _ptr(sg_used), _ptr(workspace), int(workspace_bytes), _ptr(grad_x), _ptr(grad_w), _ptr(grad_b),
+        _stream(stream)))
 
 
 def fp8_get_device_status(stream=None) -> int:

@@ -7,6 +7,11 @@
 // re-quantized transposed with the forward's steps and no ring; grad_x = g8 . w8T^T and
 // grad_w = g8T . x8T^T, both NT; grad_b = column sum of g).
 //
+// linear_forward_fp8_save_t / linear_backward_fp8_saved_t split the same work differently:
+// the forward's quantize launch also writes x^T and w^T in the backward's format from the
+// products it already forms (the backward's delayed-scaling rule quantizes them with the
+// forward's steps), so the backward quantizes only g and x and w are read once per step.
+//
 // Launches per call (delayed scaling):
 //   forward : one quantize launch for x and w + GEMM                                    = 2
 //   backward: one quantize launch for g (both orientations, per-tile column sums), x^T
@@ -113,6 +118,36 @@ MixLayout mix_layout(int64_t m, int64_t k, int64_t n) {
     return L;
 }
 
+// Backward from transposed copies the forward saved: only g's bytes, its column sums and the
+// scratch, then the split-K region.
+struct SavedLayout {
+    size_t g8, g8t, colsum, scratch, base, counters, partial, total;
+    int64_t counter_words;
+};
+
+SavedLayout saved_layout(int64_t m, int64_t k, int64_t n) {
+    SavedLayout L;
+    size_t off = 0;
+    const size_t mn = static_cast<size_t>(m) * n;
+    L.g8 = off;
+    off = align_up(off + mn, kAlign);
+    L.g8t = off;
+    off = align_up(off + mn, kAlign);
+    L.colsum = off;
+    off = align_up(off + sizeof(float) * static_cast<size_t>((m + 127) / 128) * n, kAlign);
+    L.scratch = off;
+    off = align_up(off + kScratchBytes, kAlign);
+    L.base = off;
+    const int64_t om[2] = {m, n}, on[2] = {k, k};  // grad_x [m][k], grad_w [n][k]
+    L.counter_words = splitk_counter_words(om, on, 2);
+    L.counters = off;
+    off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(L.counter_words), kAlign);
+    L.partial = off;
+    off = align_up(off + splitk_partial_bytes(om, on, 2), kAlign);
+    L.total = off;
+    return L;
+}
+
 int check_ring_arg(const fp8_ring_t* r, const char* name) {
     if (r == nullptr) return FP8DSA_OK;
     if (r->state == nullptr || r->hist_len < 1 || r->hist_idx < 0 || r->hist_idx >= r->hist_len ||
@@ -139,7 +174,8 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
                        const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                        float* sw_used, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
     return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
-                               sx_used, sw_used, nullptr, nullptr, workspace, workspace_bytes, true, y, stream);
+                               sx_used, sw_used, nullptr, nullptr, nullptr, nullptr, fmt, workspace, workspace_bytes,
+                               true, y, stream);
 }
 
 int linear_forward_fp8_keep(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
@@ -151,7 +187,19 @@ int linear_forward_fp8_keep(const void* x, const void* w, int w_is_fp8, const fl
     if ((x8_out == nullptr && m > 0 && k > 0) || (!w_is_fp8 && w8_out == nullptr && n > 0 && k > 0))
         return fail(FP8DSA_ERR_INVALID_ARG, "x8_out (and w8_out unless w_is_fp8) are required");
     return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
-                               sx_used, sw_used, x8_out, w8_out, workspace, workspace_bytes, true, y, stream);
+                               sx_used, sw_used, x8_out, w8_out, nullptr, nullptr, fmt, workspace, workspace_bytes,
+                               true, y, stream);
+}
+
+int linear_forward_fp8_save_t(const void* x, const void* w, const void* bias, const float* bias_scale, int64_t m,
+                              int64_t k, int64_t n, fp8_fmt_t fmt, fp8_fmt_t fmt_t, const fp8_ring_t* x_ring,
+                              const fp8_ring_t* w_ring, float* sx_used, float* sw_used, uint8_t* x8t_out,
+                              uint8_t* w8t_out, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
+    clear_error();
+    if (x8t_out == nullptr || w8t_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x8t_out and w8t_out are required");
+    return linear_forward_impl(x, w, 0, nullptr, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, 1.0f, sx_used,
+                               sw_used, nullptr, nullptr, x8t_out, w8t_out, fmt_t, workspace, workspace_bytes, true, y,
+                               stream);
 }
 
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
@@ -171,8 +219,9 @@ size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n) {
 int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
                         const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
                         const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
-                        float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, void* workspace,
-                        size_t workspace_bytes, bool allow_split, void* y, cudaStream_t stream) {
+                        float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, uint8_t* x8t_keep, uint8_t* w8t_keep,
+                        fp8_fmt_t fmt_t, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
+                        cudaStream_t stream) {
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
@@ -198,6 +247,15 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     if (w_is_fp8 && !aligned16(w)) return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 w must be 16-byte aligned");
     if ((x8_keep != nullptr && !aligned16(x8_keep)) || (!w_is_fp8 && w8_keep != nullptr && !aligned16(w8_keep)))
         return fail(FP8DSA_ERR_UNSUPPORTED, "x8_out / w8_out must be 16-byte aligned");
+    const bool save_t = x8t_keep != nullptr;
+    if (save_t) {
+        if (!valid_fmt(fmt_t)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt_t must be FP8_E4M3 or FP8_E5M2");
+        if (dynamic || w_is_fp8 || w8t_keep == nullptr)
+            return fail(FP8DSA_ERR_INVALID_ARG, "transposed copies need x_ring, w_ring, a bf16 w and both outputs");
+        if (!aligned16(x8t_keep) || !aligned16(w8t_keep))
+            return fail(FP8DSA_ERR_UNSUPPORTED, "x8t_out / w8t_out must be 16-byte aligned");
+        if (m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for x8t_out");
+    }
     rc = check_device();
     if (rc) return rc;
 
@@ -241,6 +299,10 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     qx.cols = k;
     qx.fmt = fmt;
     qx.out = x8;
+    if (save_t) {  // the backward's x^T from the same products, in its own format
+        qx.out_t = x8t_keep;
+        qx.fmt_t = fmt_t;
+    }
     if (dynamic) {
         qx.scale = sx;
     } else {
@@ -259,6 +321,10 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
         qw.cols = k;
         qw.fmt = fmt;
         qw.out = w8;
+        if (save_t) {
+            qw.out_t = w8t_keep;
+            qw.fmt_t = fmt_t;
+        }
         if (dynamic) {
             qw.scale = sw;
         } else {
@@ -430,6 +496,97 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
                            need_grad_b ? grad_b : nullptr, &split, g_ring, (dynamic || !ring_fold_in_call()) ? 0 : 1, stream);
     if (rc) return rc;
     return FP8DSA_OK;
+}
+
+size_t linear_backward_fp8_saved_t_workspace_size(int64_t m, int64_t k, int64_t n) {
+    if (m < 0 || k < 0 || n < 0) return 0;
+    return saved_layout(m, k, n).total;
+}
+
+int linear_backward_fp8_saved_t(const void* g, const uint8_t* x8t, const uint8_t* w8t, int64_t m, int64_t k, int64_t n,
+                                fp8_fmt_t fmt, fp8_fmt_t fmt_t, int need_grad_x, int need_grad_w, int need_grad_b,
+                                const float* sx, const float* sw, const fp8_ring_t* g_ring, float pow2_margin,
+                                float* sg_used, void* workspace, size_t workspace_bytes, void* grad_x, void* grad_w,
+                                void* grad_b, cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt) || !valid_fmt(fmt_t)) return fail(FP8DSA_ERR_INVALID_ARG, "formats must be FP8_E4M3 or FP8_E5M2");
+    if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (w8t == nullptr || sw == nullptr || grad_x == nullptr))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w8t, sw and grad_x");
+    if (need_grad_w && (x8t == nullptr || sx == nullptr || grad_w == nullptr))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x8t, sx and grad_w");
+    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
+    if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
+    if ((need_grad_w && !aligned16(x8t)) || (need_grad_x && !aligned16(w8t)))
+        return fail(FP8DSA_ERR_UNSUPPORTED, "x8t and w8t must be 16-byte aligned");
+    const bool dynamic = g_ring == nullptr;
+    if (dynamic && !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "pow2_margin must be > 0");
+    int rc = check_ring_arg(g_ring, "g_ring");
+    if (rc) return rc;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    const SavedLayout L = saved_layout(m, k, n);
+    if (workspace_bytes < L.total)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    rc = check_device();
+    if (rc) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* g8 = ws + L.g8;
+    uint8_t* g8t = ws + L.g8t;
+    float* colsum = reinterpret_cast<float*>(ws + L.colsum);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
+    float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
+    float* sg = sg_used ? sg_used : internal;
+
+    if (dynamic) {
+        cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset scratch: ") + cudaGetErrorString(e));
+        AmaxJob job;
+        job.x = g;
+        job.numel = m * n;
+        job.fp8_max = fmt_max(fmt);
+        job.pow2_margin = pow2_margin;
+        job.scale_out = sg;
+        rc = launch_amax_jobs(&job, 1, scratch, stream);
+        if (rc) return rc;
+    }
+    // g only: both orientations, its ring fold and (for grad_b) the per-tile column sums
+    QuantJob qg;
+    qg.x = g;
+    qg.rows = m;
+    qg.cols = n;
+    qg.fmt = fmt;
+    qg.out = g8;
+    qg.out_t = g8t;
+    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    if (dynamic) {
+        qg.scale = sg;
+    } else {
+        qg.scale = g_ring->state + g_ring->hist_len;
+        qg.ring = g_ring;
+        qg.scale_used_out = sg;
+        qg.defer_fold = true;  // folded by the GEMM launch below
+    }
+    SplitWorkspace split;
+    split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+    split.counter_words = L.counter_words;
+    split.partial = reinterpret_cast<float*>(ws + L.partial);
+    split.partial_bytes = L.total - L.partial;
+    rc = launch_quantize_batch(&qg, 1, stream, split.counters, split.counter_words);
+    if (rc) return rc;
+    // the same two NT GEMMs as linear_backward_fp8, on the saved transposes
+    GemmDesc gd[2];
+    int ng = 0;
+    if (need_grad_x)  // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T
+        gd[ng++] = GemmDesc{g8, w8t, fmt, fmt_t, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0, nullptr, grad_x};
+    if (need_grad_w)  // grad_w [n][k] = g8t [n][m] . (x8t [k][m])^T
+        gd[ng++] = GemmDesc{g8t, x8t, fmt, fmt_t, 0, 0, n, k, m, m, m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
+    const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
+    return gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
+                             need_grad_b ? grad_b : nullptr, &split, g_ring, (dynamic || !ring_fold_in_call()) ? 0 : 1, stream);
 }
 
 size_t linear_backward_fp8_mixed_workspace_size(int64_t m, int64_t k, int64_t n) {

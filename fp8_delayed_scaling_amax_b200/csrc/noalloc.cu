@@ -75,6 +75,6 @@ extern "C" int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is
     if (rc) return rc;
     // the GEMM runs without split-K: the built-in array holds only the operand buffers
     return linear_forward_impl(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,
-                               sx_used, sw_used, nullptr, nullptr, ws,
+                               sx_used, sw_used, nullptr, nullptr, nullptr, nullptr, fmt, ws,
                                static_cast<size_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES), false, y, stream);
 }

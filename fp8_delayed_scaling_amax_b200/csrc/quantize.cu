@@ -173,6 +173,16 @@ __device__ __forceinline__ uint2 quant8(float (&f)[8], float mult) {
     return make_uint2(cvt_fp8x4<kFmt>(f[0], f[1], f[2], f[3]), cvt_fp8x4<kFmt>(f[4], f[5], f[6], f[7]));
 }
 
+// The transposed bytes in format kFmtT of the products that quant8<kFmt> left in f (one
+// product per element, one conversion per format); `q` are quant8's own bytes.
+template <int kFmt, int kFmtT>
+__device__ __forceinline__ uint2 second_format(const float (&f)[8], uint2 q) {
+    if constexpr (kFmtT == kFmt)
+        return q;
+    else
+        return make_uint2(cvt_fp8x4<kFmtT>(f[0], f[1], f[2], f[3]), cvt_fp8x4<kFmtT>(f[4], f[5], f[6], f[7]));
+}
+
 template <int kFmt>
 __device__ __forceinline__ uint8_t convert1(float v, float mult) {
     return static_cast<uint8_t>(cvt_fp8x2<kFmt>(__fmul_rn(v, mult), 0.0f) & 0xFFu);
@@ -369,7 +379,7 @@ __device__ __forceinline__ int tile_job(const QBatch& b, int tl) {
     return jb;
 }
 
-template <class In, int kFmt, bool kPersist>
+template <class In, int kFmt, int kFmtT, bool kPersist>
 __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
     quant_tiled_kernel(const __grid_constant__ QBatch batch, const WaitCtl ctl) {
     using C = TiledCfg<In, kPersist>;
@@ -502,9 +512,10 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
                 }
-                const uint2 q = quant8<kFmt>(f, mult);
+                const uint2 q = quant8<kFmt>(f, mult);  // leaves the products in f
                 if (row_out) *reinterpret_cast<uint2*>(orow + i * ostep) = q;
-                if (col_out) *reinterpret_cast<uint2*>(trow + i * 512 + (((j >> 1) ^ i) << 2)) = q;
+                if (col_out)
+                    *reinterpret_cast<uint2*>(trow + i * 512 + (((j >> 1) ^ i) << 2)) = second_format<kFmt, kFmtT>(f, q);
             }
         } else {
 #pragma unroll
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
             }
-            const uint2 q = quant8<kFmt>(f, mult);
+            const uint2 q = quant8<kFmt>(f, mult);  // leaves the products in f
             if (row_out && gr < rows) {
                 uint8_t* dst = a.out + gr * cols + gc;
                 if (a.vec_out && gc + 8 <= cols) {
@@ -543,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
             }
             if (col_out) {
                 const int chunk = (j >> 1) ^ i;  // (r >> 4) & 7 == i
-                *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = q;
+                *reinterpret_cast<uint2*>(&tile[r * 32 + chunk * 4 + (j & 1) * 2]) = second_format<kFmt, kFmtT>(f, q);
             }
         }
         }
@@ -804,10 +815,10 @@ int64_t persist_min_tiles() { return g_persist_min_tiles.load(); }
 // Tiled launch.  Persistent: grid = min(tiles, resident CTAs) and every CTA draws one ticket
 // per tensor, so each tensor's fold counts gridDim.x blocks.  One tile per CTA: grid = tiles,
 // inputs not read by TMA, and each tensor's fold counts that tensor's tiles.
-template <int kFmt, class In, bool kPersist>
+template <int kFmt, int kFmtT, class In, bool kPersist>
 int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
     using C = TiledCfg<In, kPersist>;
-    auto kernel = quant_tiled_kernel<In, kFmt, kPersist>;
+    auto kernel = quant_tiled_kernel<In, kFmt, kFmtT, kPersist>;
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     static int per_sm = 0;
@@ -833,14 +844,27 @@ int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
     return FP8DSA_OK;
 }
 
-template <int kFmt, class In>
+// kFmtT: format of the transposed bytes (the tiled kernel only; the flat kernel writes one
+// orientation, so its launches always have kFmtT == kFmt).
+template <int kFmt, int kFmtT, class In>
 int launch_quant(QBatch& b, bool tiled, dim3 grid, const WaitCtl& ctl, cudaStream_t stream) {
     if (tiled) {
-        if (b.tiles_total > persist_min_tiles()) return launch_tiled<kFmt, In, true>(b, ctl, stream);
-        return launch_tiled<kFmt, In, false>(b, ctl, stream);
+        if (b.tiles_total > persist_min_tiles()) return launch_tiled<kFmt, kFmtT, In, true>(b, ctl, stream);
+        return launch_tiled<kFmt, kFmtT, In, false>(b, ctl, stream);
     }
-    launch_flat<kFmt, In>(b, grid, stream);
-    return FP8DSA_OK;
+    if constexpr (kFmtT == kFmt) {
+        launch_flat<kFmt, In>(b, grid, stream);
+        return FP8DSA_OK;
+    } else {
+        return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output");
+    }
+}
+
+template <int kFmt, int kFmtT>
+int launch_quant_in(fp8_in_t in_type, QBatch& b, bool tiled, dim3 grid, const WaitCtl& ctl, cudaStream_t stream) {
+    if (in_type == FP8_IN_BF16) return launch_quant<kFmt, kFmtT, Bf16In>(b, tiled, grid, ctl, stream);
+    if (in_type == FP8_IN_F16) return launch_quant<kFmt, kFmtT, F16In>(b, tiled, grid, ctl, stream);
+    return launch_quant<kFmt, kFmtT, F32In>(b, tiled, grid, ctl, stream);
 }
 
 CUtensorMapDataType map_type(fp8_in_t t) {
@@ -865,13 +889,16 @@ int check_ring(const fp8_ring_t* ring) {
 int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, uint32_t* zero, int64_t zero_words) {
     if (njobs < 1 || njobs > kMaxJobs) return fail(FP8DSA_ERR_INVALID_ARG, "quantize batch of 1..3 tensors");
     const fp8_fmt_t fmt = jobs[0].fmt;
+    const fp8_fmt_t fmt_t = jobs[0].fmt_t < 0 ? fmt : static_cast<fp8_fmt_t>(jobs[0].fmt_t);
     const fp8_in_t in_type = jobs[0].in_type;
     // the tiled kernel serves transposed / dual outputs and anything that needs column sums
     auto wants_tiles = [](const QuantJob& j) { return j.out_t != nullptr || j.colsum_partial != nullptr; };
     const bool tiled = wants_tiles(jobs[0]);
     for (int i = 1; i < njobs; ++i)
-        if (jobs[i].fmt != fmt || jobs[i].in_type != in_type || wants_tiles(jobs[i]) != tiled)
-            return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares format, input type and orientation");
+        if (jobs[i].fmt != fmt || (jobs[i].fmt_t < 0 ? fmt : static_cast<fp8_fmt_t>(jobs[i].fmt_t)) != fmt_t ||
+            jobs[i].in_type != in_type || wants_tiles(jobs[i]) != tiled)
+            return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares formats, input type and orientation");
+    if (fmt_t != fmt && !tiled) return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output");
     QBatch b{};
     b.njobs = njobs;
     b.zero = zero;
@@ -967,15 +994,12 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     }
     launch_begin(kKindQuantize, stream);
     int rc;
-    if (fmt == FP8_E4M3) {
-        if (in_type == FP8_IN_BF16) rc = launch_quant<0, Bf16In>(b, tiled, grid, ctl, stream);
-        else if (in_type == FP8_IN_F16) rc = launch_quant<0, F16In>(b, tiled, grid, ctl, stream);
-        else rc = launch_quant<0, F32In>(b, tiled, grid, ctl, stream);
-    } else {
-        if (in_type == FP8_IN_BF16) rc = launch_quant<1, Bf16In>(b, tiled, grid, ctl, stream);
-        else if (in_type == FP8_IN_F16) rc = launch_quant<1, F16In>(b, tiled, grid, ctl, stream);
-        else rc = launch_quant<1, F32In>(b, tiled, grid, ctl, stream);
-    }
+    if (fmt == FP8_E4M3)
+        rc = fmt_t == FP8_E4M3 ? launch_quant_in<0, 0>(in_type, b, tiled, grid, ctl, stream)
+                               : launch_quant_in<0, 1>(in_type, b, tiled, grid, ctl, stream);
+    else
+        rc = fmt_t == FP8_E4M3 ? launch_quant_in<1, 0>(in_type, b, tiled, grid, ctl, stream)
+                               : launch_quant_in<1, 1>(in_type, b, tiled, grid, ctl, stream);
     launch_end(kKindQuantize, stream, bytes);
     if (rc) return rc;
     return check_launch("fp8 quantize kernel");

@@ -296,6 +296,50 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
                               size_t workspace_bytes, void* grad_x, void* grad_w, void* grad_b,
                               cudaStream_t stream);
 
+/* Delayed-scaling forward that also saves the backward's transposed operands (the pages'
+ * backward quantizes x^T and w^T with the forward's steps [AstrAI compare view,
+ * astrai/extension/fp8.py, _LinearFp8.backward]; this entry forms them in the forward's
+ * quantize launch, from the same products, so x and w are read once per step):
+ *   everything as linear_forward_fp8 with w bf16 (no w_is_fp8) and both rings given, plus
+ *   x8t_out: dev [k][m] bytes = q_{fmt_t}(RN32(x[r][c] * RN32(1 / sx_used)))  at [c][r];
+ *   w8t_out: dev [k][n] bytes = q_{fmt_t}(RN32(w[r][c] * RN32(1 / sw_used)))  at [c][r];
+ *   both required, 16-byte aligned; m a multiple of 16.  The bytes equal those
+ *   linear_backward_fp8 quantizes for the same steps, so linear_backward_fp8_saved_t gives
+ *   exactly its results.  Workspace as linear_forward_fp8 (linear_forward_fp8_workspace_size).
+ *   One quantize launch (x and w, both orientations) and one GEMM launch.
+ *   FP8DSA_ERR_INVALID_ARG without both rings or outputs, or with a bad fmt_t. */
+int linear_forward_fp8_save_t(const void* x, const void* w, const void* bias,
+                              const float* bias_scale, int64_t m, int64_t k, int64_t n,
+                              fp8_fmt_t fmt, fp8_fmt_t fmt_t, const fp8_ring_t* x_ring,
+                              const fp8_ring_t* w_ring, float* sx_used, float* sw_used,
+                              uint8_t* x8t_out, uint8_t* w8t_out, void* workspace,
+                              size_t workspace_bytes, void* y, cudaStream_t stream);
+
+/* Workspace bytes linear_backward_fp8_saved_t needs for (m, k, n): g8, g8t, the per-tile
+ * column sums, scale scratch and the GEMM's split-K region. */
+size_t linear_backward_fp8_saved_t_workspace_size(int64_t m, int64_t k, int64_t n);
+
+/* linear_backward_fp8 on the transposes the forward saved (linear_forward_fp8_save_t):
+ *   g: dev bf16 [m][n], quantized once in both orientations in fmt (folding g_ring, or at the
+ *      dynamic step when g_ring == NULL), with the per-tile column sums for grad_b;
+ *   x8t: dev [k][m] bytes in fmt_t with step *sx; w8t: dev [k][n] bytes in fmt_t with step *sw
+ *      (the forward's x8t_out / w8t_out and sx_used / sw_used); 16-byte aligned.
+ *       grad_x [m][k] = g8 . w8t^T * RN32(sg * sw)    (NT)
+ *       grad_w [n][k] = g8t . x8t^T * RN32(sg * sx)   (NT)
+ *       grad_b [n]    = RN_bf16(sum over rows of g)
+ *   One quantize launch (g only) and one GEMM launch (grad_x and grad_w).  With fmt_t == fmt
+ *   the results are bit-identical to linear_backward_fp8 with the same steps.
+ *   need_grad_x / need_grad_w / need_grad_b select the outputs (the others may be NULL).
+ *   workspace: dev, >= linear_backward_fp8_saved_t_workspace_size(m, k, n) bytes, 256-byte
+ *      aligned, no initial contents needed.  k and n multiples of 16; m too for grad_w. */
+int linear_backward_fp8_saved_t(const void* g, const uint8_t* x8t, const uint8_t* w8t,
+                                int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt, fp8_fmt_t fmt_t,
+                                int need_grad_x, int need_grad_w, int need_grad_b,
+                                const float* sx, const float* sw, const fp8_ring_t* g_ring,
+                                float pow2_margin, float* sg_used, void* workspace,
+                                size_t workspace_bytes, void* grad_x, void* grad_w, void* grad_b,
+                                cudaStream_t stream);
+
 /* Device status word of the current device: 0, or a nonzero code a kernel set when a bounded
  * wait ran out (a pipeline stall instead of a hang).  Synchronises `stream`, reads the word
  * into *status (host) and clears it.  Not on the pages: added so no kernel can hang a GPU. */

@@ -146,6 +146,53 @@ def test_keep_forward_and_mixed_backward_argument_checks():
     assert call(margin=0.0) == INVALID       # dynamic scaling needs a positive margin
 
 
+def test_saved_transpose_forward_and_backward_argument_checks():
+    lib = F.lib()
+    ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
+    rx = F.fp8_ring_t(256, 16, 0, 448.0, 1.0)
+    rw = F.fp8_ring_t(512, 16, 0, 448.0, 1.0)
+    fa = dict(x=256, w=256, b=None, bs=None, m=64, k=64, n=64, f=0, ft=1, rx=ctypes.byref(rx), rw=ctypes.byref(rw),
+              sx=None, sw=None, xt=4096, wt=8192, ws=1024, wsb=ws, y=2048)
+
+    def fwd(**kw):
+        a = dict(fa, **kw)
+        return lib.linear_forward_fp8_save_t(a["x"], a["w"], a["b"], a["bs"], a["m"], a["k"], a["n"], a["f"], a["ft"],
+                                             a["rx"], a["rw"], a["sx"], a["sw"], a["xt"], a["wt"], a["ws"], a["wsb"],
+                                             a["y"], None)
+    assert fwd(xt=None) == INVALID            # both transposed outputs are required
+    assert fwd(wt=None) == INVALID
+    assert fwd(ft=7) == INVALID               # bad second format
+    assert fwd(rx=None, rw=None) == INVALID   # dynamic scaling: the backward's steps differ
+    assert fwd(rw=None) == INVALID
+    assert fwd(xt=4100) == UNSUPPORTED        # not 16-byte aligned
+    assert fwd(m=72, wsb=F.linear_forward_fp8_workspace_size(72, 64, 64)) == UNSUPPORTED  # x8t rows: 16-B multiples
+    assert fwd(wsb=ws - 256) == WORKSPACE
+    sb = lib.linear_backward_fp8_saved_t
+    wss = F.linear_backward_fp8_saved_t_workspace_size(64, 64, 64)
+    assert wss >= 2 * 64 * 64 + 4 * 64 and wss % 256 == 0
+    assert F.linear_backward_fp8_saved_t_workspace_size(-1, 1, 1) == 0
+    assert wss < F.linear_backward_fp8_workspace_size(64, 64, 64)  # no x^T / w^T inside
+    ba = dict(g=256, xt=4096, wt=8192, m=64, k=64, n=64, f=1, ft=1, gx=1, gw=1, gb=1, sx=512, sw=768, ring=None,
+              margin=1.0, sg=None, ws=1024, wsb=wss, dx=16384, dw=32768, db=65536)
+
+    def bwd(**kw):
+        a = dict(ba, **kw)
+        return sb(a["g"], a["xt"], a["wt"], a["m"], a["k"], a["n"], a["f"], a["ft"], a["gx"], a["gw"], a["gb"],
+                  a["sx"], a["sw"], a["ring"], a["margin"], a["sg"], a["ws"], a["wsb"], a["dx"], a["dw"], a["db"],
+                  None)
+    assert bwd(f=3) == INVALID
+    assert bwd(ft=-1) == INVALID
+    assert bwd(wt=None) == INVALID           # grad_x without w8t
+    assert bwd(sx=None) == INVALID           # grad_w without x8t's step
+    assert bwd(db=None) == INVALID
+    assert bwd(n=40) == UNSUPPORTED
+    assert bwd(m=40) == UNSUPPORTED          # grad_w reads x8t rows of m bytes
+    assert bwd(xt=4100) == UNSUPPORTED
+    assert bwd(ws=1040) == UNSUPPORTED
+    assert bwd(wsb=wss - 256) == WORKSPACE
+    assert bwd(margin=0.0) == INVALID
+
+
 def test_fp8_output_gemm_argument_checks():
     lib = F.lib()
     g8 = lib.fp8_gemm_fp8out
