@@ -5,18 +5,22 @@ One *step* is the whole hot path over one batch: the forward and backward (dX, d
 gradient) of every linear of a 12-layer, dim-1024 transformer trained at batch 4 x 512
 tokens (M = 2048 rows); per layer the (K, N) = (1024, 3072), (1024, 1024), (1024, 4096),
 (4096, 1024) projections.  HYBRID formats (E4M3 forward, E5M2 backward), delayed scaling with
-history 16 and margin 0, bias fused into the forward GEMM.  Per linear and step: one quantize
-launch (x, w) + one GEMM launch forward (the GEMM also folds the two rings), one quantize
-launch (g in both orientations with per-tile column sums, x^T, w^T) + one GEMM launch (dX and
-dW, grad_b reduced by its epilogue warps, the g ring folded) backward.
+history 16 and margin 0, bias fused into the forward GEMM.  Per linear and step (default
+``--path saved``): one quantize launch (x and w, each written row-major in E4M3 and transposed
+in E5M2 with the forward's steps) + one GEMM launch forward (the GEMM also folds the two
+rings), one quantize launch (g in both orientations with per-tile column sums) + one GEMM
+launch (dX and dW, grad_b reduced by its epilogue warps, the g ring folded) backward.
+``--path requant`` runs the pages' own split of the same work (the forward quantizes x, w
+row-major; the backward re-quantizes x^T, w^T beside g); both give identical numbers, and the
+line reports the other one as a variant.
 
 Timing: every layer has its own weights, activations and gradients (about 3 GB, far above
 the 126 MB L2).  The step is captured as CUDA graphs (one per history-ring slot, since the
 slot index is a host-side argument) and replayed; device time from CUDA events with a
 synchronize on both sides, max over ranks.  Per-kernel durations for the roofline come from
 the library's own CUDA-event profiler over instrumented replays of the same step.  Beside the
-headline the line reports the same step with the mixed-format backward (variants) and the
-sweeps of single GEMMs and quantizes.
+headline the line reports the other composition and the mixed-format backward (variants), and
+the sweeps of single GEMMs and quantizes.
 
 ``--impl reference`` times the CPU oracle (the plain restatement of the method, on the host
 cores) on a bounded sample of the same workload: one training linear per step.
