@@ -67,9 +67,9 @@ def parse_args():
                         "by the backward's (identical numbers)")
     p.add_argument("--dp-fold", action="store_true",
                    help="fold the rings once per step after an amax all-reduce (always on with several GPUs)")
-    p.add_argument("--kernel", default=None, choices=["gemm", "quantize"],
+    p.add_argument("--kernel", default=None, choices=["gemm", "quantize", "linear"],
                    help="time one kernel on one shape instead of the step (small cases for ncu)")
-    p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS")
+    p.add_argument("--shape", default="4096,4096,4096", help="gemm: M,N,K; quantize: ROWS,COLS; linear: M,K,N")
     p.add_argument("--qmode", default="dual", choices=["row", "t", "dual"])
     p.add_argument("--gemm-split-k", type=int, default=None,
                    help="GEMM split-K mode: 0 automatic, 1 never, 2..4 forced (library default if omitted)")
@@ -522,6 +522,19 @@ def run_kernel_mode(args):
         m, n, k = dims
         r = time_gemm(F, W, torch, dev, m, n, k, iters=args.steps, warmup=args.warmup)
         r.update(kernel="fp8_gemm", shape=[m, n, k], frac=r["tflops"] / (2 * peaks["bf16_tflops"]))
+    elif args.kernel == "linear":
+        # one training linear, forward + backward, in the step's composition (--path), in a
+        # CUDA graph: 4 launches per iteration
+        m, k, n = dims
+        STEP_PATH[0] = args.path
+        lin = Linear(F, W, torch, m, k, n, 7, dev)
+
+        def launch(i):
+            run_step([lin], i % HIST)
+
+        ms = _graph_time(torch, launch, args.steps, args.warmup)
+        r = {"ms": ms, "tflops": lin.gemm_flops / (ms * 1e-3) / 1e12, "kernel": f"linear_{args.path}",
+             "shape": [m, k, n]}
     else:
         rows, cols = dims
         r = time_quantize(F, W, torch, dev, rows, cols, args.qmode, iters=args.steps, warmup=args.warmup)
