@@ -9,7 +9,9 @@
 // extension commit log (bias_scale: fp8 bias dequantized after the operand scaling).
 //
 // B200 design (the pages' sm_89 mma.sync / cp.async / ldmatrix design is not used):
-//  * persistent grid, one CTA per SM, grouped-raster static tile schedule;
+//  * persistent grid, one CTA (or CTA pair) per SM, static schedule: tiles in grouped-raster
+//    order, dealt to the CTAs boustrophedon-wise (odd rounds in reverse), the problem with the
+//    longer K first when a launch carries two;
 //  * warp 0 = TMA producer: 3-D tensor maps (K-major or MN-major), 128-byte swizzle, into a
 //    ring of shared-memory stages guarded by full / empty mbarriers;
 //  * warp 1 = MMA issuer: one thread issues tcgen05.mma (M = 128, N = BN, K = 32) into a
@@ -24,6 +26,10 @@
 //    each SM holding 128 rows of A and half of B; pair loads complete on the leader's barriers;
 //  * one launch may carry two GEMMs over one tile space (the backward's dX and dW), and its
 //    epilogue warps can first reduce the bias-gradient column sums (a side job, no launch).
+//  * separate instances for split-K (an output tile's K range cut across CTAs: contributors
+//    leave fp32 partials, the owner adds them after a bounded acquire wait; opt-in) and for
+//    the fp8-output epilogue (the bf16 values also quantized at a given step, with their
+//    amax), so the plain instance carries neither;
 //  * every wait is bounded (globaltimer); on expiry the CTA records a status code, drains its
 //    in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>

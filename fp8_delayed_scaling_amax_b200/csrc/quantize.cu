@@ -8,15 +8,18 @@
 //
 // B200 design:
 //  * Row-major quantize is a flat grid-stride kernel: 16 elements per thread-iteration
-//    (two or four 128-bit loads, one 128-bit store of packed fp8x4 words), two iterations
-//    in flight, grid = 8 resident 256-thread blocks per SM.
-//  * Transposed / dual quantize is tiled 128 x 128 and persistent (two CTAs per SM walk all
-//    tiles of the batch): each 128 x 128 input tile arrives by one TMA bulk-tensor copy into
-//    a two-stage shared-memory ring, so the next tile loads while this one is converted;
+//    (two 128-bit loads, one 128-bit store of packed fp8x4 words), two iterations in flight;
+//    one wave of 4 resident 256-thread blocks per SM, shared out to the tensors of the launch
+//    in proportion to their sizes.
+//  * Transposed / dual quantize is tiled 128 x 128.  Large batches run persistent (two CTAs
+//    per SM walk all tiles of the batch): each input tile arrives by one TMA bulk-tensor copy
+//    into a two-stage shared-memory ring, so the next tile loads while this one is converted.
+//    Small batches run one tile per CTA (three per SM), loaded straight into registers.  The
 //    fp8 bytes are staged in a 16 KB shared tile whose 16-byte chunks are XOR-swizzled by row
 //    group, then a register 4x4 byte transpose (PRMT) and 128-byte coalesced stores of each
-//    output row.  The dual mode also writes the row-major bytes straight from registers, and
-//    can emit per-tile fp32 column sums (the bias gradient) from the values it already holds.
+//    output row.  The dual mode also writes the row-major bytes straight from registers (the
+//    transposed bytes may take a second format: the same products rounded twice), and can
+//    emit per-tile fp32 column sums (the bias gradient) from the values it already holds.
 //  * Each block reduces amax with warp shuffles, one atomicMax per block and tensor; with a
 //    ring, an acq_rel ticket elects the last block, which folds the amax into the window and
 //    publishes the next step.  The fold itself never waits; the tiled kernel's only wait (for
@@ -795,10 +798,9 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
     out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
 }
 
-#ifndef FLAT_WAVES
-#define FLAT_WAVES 1
-#endif
-constexpr int kFlatWaves = FLAT_WAVES;
+// Waves of resident blocks a row-major launch is sized to (measured on B200: one wave, each
+// block looping over its share, beats several waves of shorter blocks).
+constexpr int kFlatWaves = 1;
 
 // Resident 256-thread blocks per SM of the row-major kernel (its launch bounds ask for 4).
 int flat_blocks_per_sm() { return 4; }
