@@ -156,6 +156,7 @@ struct QBatch {
     QArgs job[kMaxJobs];
     int njobs;
     int tiles_total;            // tiled kernel: tiles of all jobs, concatenated
+    int row_out_any;            // tiled kernel: some job also writes row-major bytes
     uint32_t* zero;             // side job of the launch's first block: zero[0 .. zero_words)
     int64_t zero_words;
 };
@@ -349,9 +350,12 @@ struct TiledCfg {
     static constexpr bool kF32 = sizeof(typename In::E) == 4;
     static constexpr int kStages = kPersist ? 2 : 0;
     static constexpr int kRawBytes = kTile * kTile * static_cast<int>(sizeof(typename In::E));
-    static constexpr int kOffTile = kStages * kRawBytes;       // 128 x 128 fp8 byte tile
-    static constexpr int kOffCsum = kOffTile + kTile * kTile;  // 8 x 128 fp32 column sums
-    static constexpr int kOffBar = kOffCsum + 8 * kTile * 4;   // one mbarrier per stage
+    // persistent: byte tile and column sums double-buffered, so a tile's transposed stores
+    // need no barrier before the next tile's conversion
+    static constexpr int kBufs = kPersist ? 2 : 1;
+    static constexpr int kOffTile = kStages * kRawBytes;               // 128 x 128 fp8 byte tile(s)
+    static constexpr int kOffCsum = kOffTile + kBufs * kTile * kTile;  // 8 x 128 fp32 column sums
+    static constexpr int kOffBar = kOffCsum + kBufs * 8 * kTile * 4;   // one mbarrier per stage
     static constexpr int kSmem = kOffBar + kStages * 8 + 1024; // + slack to align the base
     static constexpr int kMinBlocks = kPersist ? (kF32 ? 1 : 2) : (kF32 ? 2 : 3);
 };
@@ -390,7 +394,6 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
     extern __shared__ uint8_t dsmem[];
     const uint32_t base = smem_addr(dsmem);
     uint8_t* smem = dsmem + (((base + 1023u) & ~1023u) - base);
-    float(*csum)[kTile] = reinterpret_cast<float(*)[kTile]>(smem + C::kOffCsum);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     __shared__ float s_hist[kMaxJobs][kHistPrefetch];
     __shared__ float s_red[kMaxJobs][kThreads / 32];
@@ -481,7 +484,9 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         const E* stage = reinterpret_cast<const E*>(smem + s * C::kRawBytes);
         // The tile's fp8 bytes, 128 rows x 128 bytes, in the first 16 KB of stage s: the
         // 16-byte chunk c of row r lives at chunk c ^ ((r >> 4) & 7).
-        uint32_t* tile = reinterpret_cast<uint32_t*>(smem + C::kOffTile);
+        const int bsel = C::kBufs > 1 ? (it & 1) : 0;
+        uint32_t* tile = reinterpret_cast<uint32_t*>(smem + C::kOffTile + bsel * kTile * kTile);
+        float(*csum)[kTile] = reinterpret_cast<float(*)[kTile]>(smem + C::kOffCsum + bsel * 8 * kTile * 4);
 
         float tamax = 0.0f;                          // amax of the rows read element-wise
         typename In::Acc acc = In::acc_zero();       // amax of the rows read as raw chunks
@@ -626,7 +631,12 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
             }
         }
         }
-        __syncthreads();  // the byte tile and the column sums are free
+        // One buffer: the byte tile and the column sums are free for the next tile only after
+        // every thread's transposed stores.  Two: the next tile fills the other buffer, and the
+        // barrier after its conversion orders these reads before the buffer's next reuse; kept
+        // anyway when row-major bytes are written (measured on B200: the dual quantize loses
+        // 3-6% when its warps drift a tile apart, the transposed one gains 2%).
+        if (C::kBufs == 1 || batch.row_out_any) __syncthreads();
     }
 
     if (aborted) {
@@ -972,6 +982,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     WaitCtl ctl{};
     if (tiled) {
         b.tiles_total = static_cast<int>(tiles_total);
+        for (int i = 0; i < njobs; ++i) b.row_out_any |= jobs[i].out != nullptr ? 1 : 0;
         const int rc = wait_ctl(&ctl);
         if (rc) return rc;
     } else {
