@@ -386,7 +386,10 @@ __device__ __forceinline__ int tile_job(const QBatch& b, int tl) {
     return jb;
 }
 
-template <class In, int kFmt, int kFmtT, bool kPersist>
+// kTOnly (persistent only): every job of the batch writes transposed bytes and no row-major
+// ones, so full tiles take the stepped fast path; batches with row-major bytes keep the
+// general loop (measured on B200: the fast path in their instance slows the dual quantize).
+template <class In, int kFmt, int kFmtT, bool kPersist, bool kTOnly = false>
 __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
     quant_tiled_kernel(const __grid_constant__ QBatch batch, const WaitCtl ctl) {
     using C = TiledCfg<In, kPersist>;
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         const int s = kPersist ? it % (C::kStages > 0 ? C::kStages : 1) : 0;
         const int jb = tile_job(batch, tl);
         const QArgs& a = batch.job[jb];
-        const bool row_out = a.out != nullptr;
+        const bool row_out = !kTOnly && a.out != nullptr;
         const bool col_out = a.out_t != nullptr;  // transposed output (else row-major + column sums only)
         const bool colsum = a.colsum != nullptr;
         const float mult = __frcp_rn(__ldg(a.scale));
@@ -505,8 +508,8 @@ __global__ void __launch_bounds__(kThreads, TiledCfg<In, kPersist>::kMinBlocks)
         // a full tile with vector-aligned outputs: no per-row checks, addresses stepped (in the
         // one-tile-per-CTA kernel, which is issue-bound on small batches; the persistent one keeps
         // its register budget)
-        const bool full = !kPersist && (from_smem || interior) && r0 + kTile <= rows && c0 + kTile <= cols &&
-                          (!row_out || a.vec_out);
+        const bool full = (!kPersist || kTOnly) && (from_smem || interior) && r0 + kTile <= rows &&
+                          c0 + kTile <= cols && (!row_out || a.vec_out);
         if (full) {
             uint8_t* orow = row_out ? a.out + (r0 + rr) * cols + gc : nullptr;
             const int64_t ostep = 16 * cols;
@@ -827,10 +830,10 @@ int64_t persist_min_tiles() { return g_persist_min_tiles.load(); }
 // Tiled launch.  Persistent: grid = min(tiles, resident CTAs) and every CTA draws one ticket
 // per tensor, so each tensor's fold counts gridDim.x blocks.  One tile per CTA: grid = tiles,
 // inputs not read by TMA, and each tensor's fold counts that tensor's tiles.
-template <int kFmt, int kFmtT, class In, bool kPersist>
+template <int kFmt, int kFmtT, class In, bool kPersist, bool kTOnly = false>
 int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
     using C = TiledCfg<In, kPersist>;
-    auto kernel = quant_tiled_kernel<In, kFmt, kFmtT, kPersist>;
+    auto kernel = quant_tiled_kernel<In, kFmt, kFmtT, kPersist, kTOnly>;
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     static int per_sm = 0;
@@ -861,7 +864,14 @@ int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
 template <int kFmt, int kFmtT, class In>
 int launch_quant(QBatch& b, bool tiled, dim3 grid, const WaitCtl& ctl, cudaStream_t stream) {
     if (tiled) {
-        if (b.tiles_total > persist_min_tiles()) return launch_tiled<kFmt, kFmtT, In, true>(b, ctl, stream);
+        if (b.tiles_total > persist_min_tiles()) {
+            if constexpr (kFmtT == kFmt) {
+                bool t_only = true;
+                for (int i = 0; i < b.njobs; ++i) t_only = t_only && b.job[i].out == nullptr && b.job[i].colsum == nullptr;
+                if (t_only) return launch_tiled<kFmt, kFmtT, In, true, true>(b, ctl, stream);
+            }
+            return launch_tiled<kFmt, kFmtT, In, true>(b, ctl, stream);
+        }
         return launch_tiled<kFmt, kFmtT, In, false>(b, ctl, stream);
     }
     if constexpr (kFmtT == kFmt) {
@@ -970,9 +980,9 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
             const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
             a.tiles_x = static_cast<int>(tx);
             a.tiles_y = static_cast<int>(ty);
-            // measured (persistent kernel, B200): groups of 4 tile rows pay off only for the dual
-            // quantize with transposed rows at least 16 KB apart; row order everywhere else
-            a.tile_group = (job.out != nullptr && job.out_t != nullptr && job.rows >= 16384) ? 4 : 1;
+            // measured (persistent kernel, B200): groups of 4 tile rows pay off once transposed
+            // rows are at least 16 KB apart; row order everywhere else
+            a.tile_group = (job.out_t != nullptr && job.rows >= 16384) ? 4 : 1;
             a.tile_begin = static_cast<int>(tiles_total);
             tiles_total += tx * ty;
             if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 tiles");
