@@ -478,7 +478,8 @@ def time_fp8_output(F, W, torch, dev, m, n, k, fused, iters=20, warmup=5):
     return {"ms": ms, "tflops": 2.0 * m * n * k / (ms * 1e-3) / 1e12}
 
 
-def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5):
+def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5, fmt=None):
+    fmt = F.FP8_E4M3 if fmt is None else fmt
     per_set = rows * cols * (2 + (2 if mode == "dual" else 1))
     nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
     sets = []
@@ -488,7 +489,7 @@ def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5):
         out_t = torch.empty((cols, rows), dtype=torch.uint8, device=dev)
         st = torch.zeros(HIST + 4, dtype=torch.float32, device=dev)
         F.fp8_scale_ring_init(st, HIST)
-        ring = F.Ring(st, HIST, F.FP8_E4M3)
+        ring = F.Ring(st, HIST, fmt)
         F.fp8_scale_ring_seed(ring, x, F.FP8_IN_BF16, x.numel())
         sets.append((x, out, out_t, ring))
 
@@ -496,11 +497,11 @@ def time_quantize(F, W, torch, dev, rows, cols, mode, iters=20, warmup=5):
         x, out, out_t, ring = sets[i % nsets]
         step = ring.state[HIST:HIST + 1]
         if mode == "row":
-            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, 0, out, None, ring)
+            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, fmt, 0, out, None, ring)
         elif mode == "t":
-            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, 1, out_t, None, ring)
+            F.fp8_quantize(x, F.FP8_IN_BF16, rows, cols, step, fmt, 1, out_t, None, ring)
         else:
-            F.fp8_quantize_dual(x, F.FP8_IN_BF16, rows, cols, step, F.FP8_E4M3, out, out_t, None, ring)
+            F.fp8_quantize_dual(x, F.FP8_IN_BF16, rows, cols, step, fmt, out, out_t, None, ring)
         ring.advance()
 
     ms = _graph_time(torch, launch, iters, warmup)
@@ -560,11 +561,16 @@ def run_sweeps(F, W, torch, dev):
         key = f"{batch}x{m}x{n}x{k}" + ("(B bcast)" if bb == 1 and batch > 1 else "")
         out["gemm_skinny_batched"][key] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
                                            "frac": round(r["tflops"] / burst_fp8, 4)}
-    for rows, cols in ((4096, 4096), (8192, 8192), (16384, 16384)):
-        for mode in ("row", "t", "dual"):
-            r = time_quantize(F, W, torch, dev, rows, cols, mode)
-            out["quantize"][f"{mode}_{rows}x{cols}"] = {"gbs": round(r["gbs"], 1), "us": round(r["ms"] * 1e3, 2),
-                                                       "frac": round(r["gbs"] / peaks["hbm_gbs"], 4)}
+    # bf16 inputs of 2^24 .. 2^28 elements with a ring; E5M2 beside E4M3 at the two larger sizes
+    for rows, cols, fmts in ((8192, 2048, ("e4m3",)), (4096, 4096, ("e4m3",)), (8192, 8192, ("e4m3", "e5m2")),
+                             (16384, 16384, ("e4m3", "e5m2"))):
+        for fname in fmts:
+            for mode in ("row", "t", "dual"):
+                r = time_quantize(F, W, torch, dev, rows, cols, mode,
+                                  fmt=F.FP8_E4M3 if fname == "e4m3" else F.FP8_E5M2)
+                key = f"{mode}_{rows}x{cols}" + ("" if fname == "e4m3" else "_e5m2")
+                out["quantize"][key] = {"gbs": round(r["gbs"], 1), "us": round(r["ms"] * 1e3, 2),
+                                        "frac": round(r["gbs"] / peaks["hbm_gbs"], 4)}
     for m, n, k in ((2048, 3072, 1024), (2048, 4096, 1024), (4096, 4096, 4096)):
         fused = time_fp8_output(F, W, torch, dev, m, n, k, True)
         split = time_fp8_output(F, W, torch, dev, m, n, k, False)
