@@ -899,10 +899,13 @@ void plan_units(GemmArgs& g, int units, int64_t max_contrib, int64_t counter_wor
 template <int BN, bool kPair, bool kSplit, bool kOut8>
 cudaError_t kernel_setup(int* max_units_out) {
     using C = Cfg<BN, kPair>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    static int max_units = 0;
-    std::call_once(once, [] {
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_errs[kMaxDevices];
+    static int max_units_dev[kMaxDevices];
+    const int dev = current_device();
+    cudaError_t& attr_err = attr_errs[dev];
+    int& max_units = max_units_dev[dev];
+    std::call_once(once[dev], [&attr_err, &max_units] {
         attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN, kPair, kSplit, kOut8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::kSmem);
         if (attr_err != cudaSuccess) return;
@@ -914,7 +917,7 @@ cudaError_t kernel_setup(int* max_units_out) {
             at[0].val.clusterDim.x = 2;
             at[0].val.clusterDim.y = 1;
             at[0].val.clusterDim.z = 1;
-            cfg.gridDim = dim3(2 * 74, 1, 1);
+            cfg.gridDim = dim3(static_cast<unsigned>(2 * (sm_count() / 2)), 1, 1);
             cfg.blockDim = dim3(C::kThreads, 1, 1);
             cfg.dynamicSmemBytes = C::kSmem;
             cfg.attrs = at;

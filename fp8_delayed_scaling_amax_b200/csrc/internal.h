@@ -22,6 +22,10 @@ void clear_error();
 int check_device();
 // Number of SMs of the current device (cached per device).
 int sm_count();
+// The current CUDA device, clamped to the library's per-device tables (0 .. kMaxDevices - 1):
+// one-time kernel set-up (shared-memory attributes, occupancy) is cached per device.
+constexpr int kMaxDevices = 64;
+int current_device();
 
 // WaitCtl for the current device (status word address + timeout).
 int wait_ctl(WaitCtl* ctl);

@@ -834,10 +834,13 @@ template <int kFmt, int kFmtT, class In, bool kPersist, bool kTOnly = false>
 int launch_tiled(QBatch& b, const WaitCtl& ctl, cudaStream_t stream) {
     using C = TiledCfg<In, kPersist>;
     auto kernel = quant_tiled_kernel<In, kFmt, kFmtT, kPersist, kTOnly>;
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    static int per_sm = 0;
-    std::call_once(once, [kernel] {
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t errs[kMaxDevices];
+    static int per_sm_dev[kMaxDevices];
+    const int dev = current_device();
+    cudaError_t& err = errs[dev];
+    int& per_sm = per_sm_dev[dev];
+    std::call_once(once[dev], [kernel, &err, &per_sm] {
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (err == cudaSuccess) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, C::kSmem);
     });

@@ -17,8 +17,6 @@ namespace fp8dsa {
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 thread_local std::string t_last_error;
 
 std::mutex g_mutex;
@@ -84,6 +82,12 @@ int check_device() {
     if (g_cc_major[dev] != 10)
         return fail(FP8DSA_ERR_DEVICE, "fp8dsa kernels are built for sm_100a (compute capability 10.x)");
     return FP8DSA_OK;
+}
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    return dev < 0 ? 0 : (dev >= kMaxDevices ? kMaxDevices - 1 : dev);
 }
 
 int sm_count() {
