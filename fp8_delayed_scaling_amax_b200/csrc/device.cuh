@@ -420,6 +420,16 @@ __device__ __forceinline__ void add2_rn(float& a, float& b, float c, float d) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
 }
 
+// a = RN32(a * m + c), b = RN32(b * m + c) (fused, one rounding each) in one packed instruction.
+__device__ __forceinline__ void fma2_rn(float& a, float& b, float m, float c) {
+    unsigned long long p, q, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(q) : "f"(m));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(c));
+    asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(p) : "l"(q), "l"(r));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
+}
+
 // History-ring fold done after the quantize kernel that measured the amax (one thread; the
 // quantize blocks only left their maxima in the amax slot).  Ring layout [hist n | scale |
 // scale_used | amax | done]: scale_used = the step the quantize used (the current scale),

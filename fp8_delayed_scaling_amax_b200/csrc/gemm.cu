@@ -612,17 +612,33 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                     }
                 }
                 uint32_t packed[32];
+                if (P.bias_kind != 0) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float v0 = fmaf(__uint_as_float(r0[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e));
-                    const float v1 = fmaf(__uint_as_float(r0[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e + 1));
-                    packed[e] = pack_bf16x2(v0, v1);
-                }
+                    for (int e = 0; e < 16; ++e) {
+                        const float v0 = fmaf(__uint_as_float(r0[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e));
+                        const float v1 = fmaf(__uint_as_float(r0[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_lo, 2 * e + 1));
+                        packed[e] = pack_bf16x2(v0, v1);
+                    }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float v0 = fmaf(__uint_as_float(r1[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e));
-                    const float v1 = fmaf(__uint_as_float(r1[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e + 1));
-                    packed[16 + e] = pack_bf16x2(v0, v1);
+                    for (int e = 0; e < 16; ++e) {
+                        const float v0 = fmaf(__uint_as_float(r1[2 * e]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e));
+                        const float v1 = fmaf(__uint_as_float(r1[2 * e + 1]), scale, __shfl_sync(0xFFFFFFFFu, b_hi, 2 * e + 1));
+                        packed[16 + e] = pack_bf16x2(v0, v1);
+                    }
+                } else {
+                    // no bias: the same fma with a zero addend, two lanes per packed instruction
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float v0 = __uint_as_float(r0[2 * e]), v1 = __uint_as_float(r0[2 * e + 1]);
+                        fma2_rn(v0, v1, scale, 0.0f);
+                        packed[e] = pack_bf16x2(v0, v1);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float v0 = __uint_as_float(r1[2 * e]), v1 = __uint_as_float(r1[2 * e + 1]);
+                        fma2_rn(v0, v1, scale, 0.0f);
+                        packed[16 + e] = pack_bf16x2(v0, v1);
+                    }
                 }
                 const int colg = col0 + c;
                 if (P.tma_out) {
