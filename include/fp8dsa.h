@@ -367,9 +367,10 @@ int fp8_set_gemm_split_k(int splits);
 
 /* Transposed / dual quantize launches covering more than `min_tiles` 128 x 128 tiles (over all
  * tensors of the launch) run on the persistent TMA-fed kernel; smaller ones run one tile per
- * CTA.  Both give identical bytes, amax and ring updates; the choice only moves time.  Default
- * 1024; min_tiles < 0 is rejected (FP8DSA_ERR_INVALID_ARG).  Applies to later launches.  Not
- * on the pages. */
+ * CTA.  Launches that write only transposed bytes switch above min_tiles / 8.  Both kernels
+ * give identical bytes, amax and ring updates; the choice only moves time.  Default 1024;
+ * min_tiles < 0 is rejected (FP8DSA_ERR_INVALID_ARG).  Applies to later launches.  Not on the
+ * pages. */
 int fp8_set_tiled_persist_threshold(int64_t min_tiles);
 
 /* Test hook for the failure path: launches one block that waits on a barrier nothing ever
