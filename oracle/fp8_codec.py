@@ -18,8 +18,9 @@ saturation to the finite range (compare view, ``quantize.cuh``: the fp8x2
 conversion with ``__NV_SATFINITE``).  Readings taken where the pages are silent:
 
 * ``|v| >= FP8_MAX`` (including +-inf) encodes as +-FP8_MAX.
-* NaN encodes as the positive canonical NaN byte 0x7F (the device's NaN byte is
-  not pinned by the pages; no workload here contains NaN).
+* NaN encodes as the positive canonical NaN byte 0x7F -- parity unpinned: the
+  pages fix no NaN byte and no workload here contains NaN, so the GPU tests only
+  check that the device writes some NaN code for a NaN input.
 * The sign of zero is kept (a negative value that rounds to zero gives 0x80).
 """
 
