@@ -87,14 +87,15 @@ def dist_env():
 # ---------------------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------------------
-def oracle_linear_step(k, n, seed):
-    """The oracle's forward + backward of one training linear; returns (seconds, flops)."""
+def oracle_linear_step(k, n, seed, shrink=1):
+    """The oracle's forward + backward of one training linear (M = 2048 rows), every dimension
+    divided by `shrink` for a bounded sample; returns (seconds, flops)."""
     import numpy as np
     import workloads as W
     from oracle import linear as L
     from oracle import scaling as S
 
-    m = W.TRAINING_TOKENS
+    m, k, n = W.TRAINING_TOKENS // shrink, k // shrink, n // shrink
     t = W.training_linear(m, k, n, seed)
     bits = {key: W.bf16_bits(t[key]) for key in ("x", "w", "b", "g")}
     rx, rw, rg = S.Ring(HIST, "e4m3"), S.Ring(HIST, "e4m3"), S.Ring(HIST, "e5m2")
@@ -133,26 +134,49 @@ def cpu_baseline():
                       f"numpy oracle (fp64 GEMMs): {total_f / 1e9:.1f} GFLOP in {total_t:.1f} s"}
 
 
+REFERENCE_BUDGET_S = 150.0  # wall-clock budget of a whole --impl reference run
+
+
+def reference_shrink(steps, warmup):
+    """The factor (a power of two, at most 32) every dimension of the reference steps' training
+    linear is divided by, so that warm-up plus timed steps stay within REFERENCE_BUDGET_S.  The
+    oracle's wall-clock cost (input generation included) is calibrated on one step shrunk 16x
+    and taken to grow with the square of the factor it saves (a conservative bound: its GEMMs
+    grow with the cube)."""
+    oracle_linear_step(1024, 3072, seed=7998, shrink=32)  # first-call overheads out of the way
+    t0 = time.perf_counter()
+    for k, n in ((1024, 3072), (1024, 1024), (1024, 4096), (4096, 1024)):
+        oracle_linear_step(k, n, seed=7999, shrink=16)
+    cal = max((time.perf_counter() - t0) / 4, 1e-4)
+    per_step = REFERENCE_BUDGET_S / max(1, steps + warmup)
+    for shrink in (1, 2, 4, 8, 16):
+        if cal * (16 / shrink) ** 2 <= per_step:
+            return shrink
+    return 32
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     import workloads as W
+    shrink = reference_shrink(args.steps, args.warmup)
     for i in range(args.warmup):
         k, n = W.TRAINING_LINEARS[i % 4]
-        oracle_linear_step(k, n, seed=8000 + i)
+        oracle_linear_step(k, n, seed=8000 + i, shrink=shrink)
     total_t, total_f = 0.0, 0.0
     for i in range(args.steps):
         k, n = W.TRAINING_LINEARS[i % 4]
-        dt, fl = oracle_linear_step(k, n, seed=9000 + i)
+        dt, fl = oracle_linear_step(k, n, seed=9000 + i, shrink=shrink)
         total_t += dt
         total_f += fl
     value = total_f / total_t / 1e12
-    sample = (f"one training linear (M=2048, (K,N) cycling over the 4 shapes) forward + backward per step "
-              f"through the numpy oracle; {args.steps} steps, {total_t:.1f} s")
+    sample = (f"one training linear per step ((M,K,N) = (2048,K,N) / {shrink}, (K,N) cycling over the 4 "
+              f"shapes; sized so the run stays within about {REFERENCE_BUDGET_S:.0f} s) forward + backward "
+              f"through the numpy oracle; {args.steps} steps, {total_t:.1f} s timed")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t * 1e3 / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "sample": "one linear per step"},
+            "config": {"workload": WORKLOAD, "sample": f"one linear per step, every dimension / {shrink}"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
