@@ -91,6 +91,7 @@ struct GemmProblem {
     int a_batched, b_batched;
     int a_mn, b_mn;
     uint32_t idesc;
+    uint32_t idesc_half;  // the same MMA with N = 128 (a half tile of the last round)
     uint16_t* out;
     int64_t ldo, stride_o;
     int vec_out;
@@ -132,6 +133,7 @@ struct GemmArgs {
     int nprob;
     int num_tiles;
     int num_units, contrib_units;  // work units (tile, K range); the first contrib_units are split-K contributors
+    int half_begin;                // (no split-K) tiles from here on are run as two 256 x 128 halves
     int splitk;                    // some problem has k_splits > 1
     float* partial;                // split-K fp32 partial tiles: [contrib unit][CTA of the pair][BN/4][128][4]
     uint32_t* counters;            // split-K arrivals per (tile, CTA of the pair); zero at launch
@@ -178,14 +180,21 @@ __device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& pi
 // owner only ever waits for units that never wait themselves.
 struct Unit {
     int pi, tile, split, kb0, kb1;
+    int half;  // -1: the whole tile; 0 / 1: its left / right 128 columns
 };
 
 template <bool kSplit>
 __device__ __forceinline__ Unit decode_unit(int u, const GemmArgs& g) {
     Unit r;
-    if constexpr (!kSplit) {  // one unit per tile, the whole K range
-        r.pi = (g.nprob > 1 && u >= g.p[1].tile_begin) ? 1 : 0;
-        r.tile = u;
+    r.half = -1;
+    if constexpr (!kSplit) {  // one unit per tile, or per half of the tiles from half_begin on
+        if (u >= g.half_begin) {
+            r.tile = g.half_begin + ((u - g.half_begin) >> 1);
+            r.half = (u - g.half_begin) & 1;
+        } else {
+            r.tile = u;
+        }
+        r.pi = (g.nprob > 1 && r.tile >= g.p[1].tile_begin) ? 1 : 0;
         r.split = 0;
         r.kb0 = 0;
         r.kb1 = g.p[r.pi].k_blocks;
@@ -253,6 +262,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a0, const __grid_constant__ CUtensorMap tma_b0,
                     const __grid_constant__ CUtensorMap tma_o0, const __grid_constant__ CUtensorMap tma_a1,
                     const __grid_constant__ CUtensorMap tma_b1, const __grid_constant__ CUtensorMap tma_o1,
+                    const __grid_constant__ CUtensorMap tma_bh0, const __grid_constant__ CUtensorMap tma_bh1,
                     const __grid_constant__ GemmArgs g) {
     using C = Cfg<BN, kPair>;
     constexpr int S = C::kStages;
@@ -330,17 +340,22 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 decode_tile(w.tile, g, pi, b, tm, tn);
                 const GemmProblem& P = g.p[pi];
                 const CUtensorMap* ta = pi ? &tma_a1 : &tma_a0;
-                const CUtensorMap* tb = pi ? &tma_b1 : &tma_b0;
+                // a half tile (pairs, K-major B only): each CTA loads 64 rows of B through the
+                // 64-row map, and the stage carries that many fewer bytes
+                const bool half = kPair && w.half >= 0;
+                const CUtensorMap* tb = half ? (pi ? &tma_bh1 : &tma_bh0) : (pi ? &tma_b1 : &tma_b0);
                 const int ba = P.a_batched ? b : 0;
                 const int bb = P.b_batched ? b : 0;
                 const int arow = tm * C::kTileM + static_cast<int>(rank) * kBM;
-                const int brow = tn * BN + static_cast<int>(rank) * C::kBRows;
+                const int brow = half ? tn * BN + w.half * 128 + static_cast<int>(rank) * 64
+                                      : tn * BN + static_cast<int>(rank) * C::kBRows;
+                const uint32_t tx = half ? C::kTxBytes - (kPair ? 2u : 1u) * (C::kBStage / 2) : C::kTxBytes;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_bounded(empty + stage, phase ^ 1u, g.wait, abort_flag, kStatusWaitProducer)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(full + stage, C::kTxBytes);
+                    if (leader) mbar_arrive_expect_tx(full + stage, tx);
                     uint8_t* a_dst = sA + stage * C::kAStage;
                     uint8_t* b_dst = sB + stage * C::kBStage;
                     if constexpr (kPair) {
@@ -396,6 +411,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             for (int r = 0, u = unit; u < g.num_units && ok; u = snake_unit(++r, unit, units)) {
                 const Unit w = decode_unit<kSplit>(u, g);
                 const GemmProblem& P = g.p[w.pi];
+                const uint32_t idesc = w.half >= 0 ? P.idesc_half : P.idesc;
                 const bool got = kPair ? mbar_wait_bounded_cluster(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
                                                                    kStatusWaitMma)
                                        : mbar_wait_bounded(acc_empty + acc, acc_phase ^ 1u, g.wait, abort_flag,
@@ -424,9 +440,9 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                                                        : smem_desc(b_base + kk * kUmmaK, 16, 1024);
                             const uint32_t accumulate = (kb != w.kb0 || kk != 0) ? 1u : 0u;
                             if constexpr (kPair)
-                                umma_f8f6f4_pair(d_tmem, ad, bd, P.idesc, accumulate);
+                                umma_f8f6f4_pair(d_tmem, ad, bd, idesc, accumulate);
                             else
-                                umma_f8f6f4(d_tmem, ad, bd, P.idesc, accumulate);
+                                umma_f8f6f4(d_tmem, ad, bd, idesc, accumulate);
                         }
                         if constexpr (kPair)
                             umma_commit_pair_multicast(empty + stage, 0x3);
@@ -541,7 +557,10 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             const bool owner = kSplit && !contrib && P.k_splits > 1;  // add the partials, then write
             const CUtensorMap* to = pi ? &tma_o1 : &tma_o0;
             const float scale = pi ? sc[1] : sc[0];
-            const int col0 = tn * BN + cbase;
+            // a half tile's 128 accumulator columns: every epilogue warp takes 64 of them
+            const int ncols = w.half >= 0 ? kOutBox : C::kEpiCols;
+            const int cbase_u = w.half >= 0 ? (ew >> 2) * kOutBox : cbase;
+            const int col0 = tn * BN + (w.half >= 0 ? w.half * 128 : 0) + cbase_u;
             const int row0 = tm * C::kTileM + static_cast<int>(rank) * kBM + q * 32;
             const int64_t row = static_cast<int64_t>(row0) + lane;
             // this warp's bias columns col0 + 32 j + lane in bias_r[j], loaded before the wait
@@ -566,15 +585,16 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             }
 #pragma unroll
             for (int c = 0; c < C::kEpiCols; c += kOutBox) {
+                if (c >= ncols) break;
                 uint32_t r0[32], r1[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(acc * BN + cbase + c);
+                                       static_cast<uint32_t>(acc * BN + cbase_u + c);
                 tmem_load_32cols(taddr, r0);
                 tmem_load_32cols(taddr + 32, r1);
                 const float b_lo = bias_r[c / 32];
                 const float b_hi = bias_r[c / 32 + 1];
                 tmem_wait_ld();
-                const int cc = cbase + c;  // column within the tile
+                const int cc = cbase_u + c;  // column within the tile
                 // Partial tiles are stored as [column group of 4][row][4]: for each group the 32
                 // lanes (rows) of a warp cover 512 contiguous bytes, one coalesced access.
                 if (contrib) {
@@ -818,6 +838,38 @@ int range_len(const GemmProblem& P, int splits, int s) {
 // tile wherever the workspace and K allow (set by fp8_set_gemm_split_k).
 std::atomic<int> g_split_mode{1};
 
+// Makespan of a launch without split-K, in k-block times: the units dealt boustrophedon-wise to
+// `units` pairs, a whole tile costing its k-blocks and a half tile 0.87 of them (a 256 x 128 MMA
+// costs that much of a 256 x 256 one on B200), plus the last unit's epilogue (about 5.4 k-blocks
+// for a whole tile, half that for a half).  Units from `half_begin` on are halves.
+double plain_makespan(const GemmArgs& g, int units, int num_units, int half_begin) {
+    double worst = 0.0;
+    for (int c = 0; c < units; ++c) {
+        double t = 0.0, last_epi = 0.0;
+        for (int r = 0;; ++r) {
+            const int u = r * units + ((r & 1) ? units - 1 - c : c);
+            if (u >= num_units) break;
+            const bool half = u >= half_begin;
+            const int tile = half ? half_begin + ((u - half_begin) >> 1) : u;
+            const int pi = (g.nprob > 1 && tile >= g.p[1].tile_begin) ? 1 : 0;
+            t += (half ? 0.87 : 1.0) * g.p[pi].k_blocks;
+            last_epi = half ? 2.7 : 5.4;
+        }
+        worst = std::max(worst, t + last_epi);
+    }
+    return worst;
+}
+
+// Tuning override: FP8DSA_GEMM_HALF_TILES=0 keeps every tile of the last round whole (read
+// once; unset = half tiles where they shorten the launch).
+bool half_tiles_enabled() {
+    static const bool v = [] {
+        const char* e = std::getenv("FP8DSA_GEMM_HALF_TILES");
+        return e == nullptr || std::string(e) != "0";
+    }();
+    return v;
+}
+
 // Modelled makespan (us) of the unit schedule with `sp` ranges per problem on `units` CTAs.
 double simulate_plan(const GemmArgs& g, const int* sp, int units, std::vector<double>& mma_end,
                      std::vector<double>& epi_end, std::vector<double>& contrib_end) {
@@ -949,7 +1001,7 @@ cudaError_t kernel_setup(int* max_units_out) {
 }
 
 template <int BN, bool kPair>
-int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, const SplitWorkspace* split,
+int launch_cfg(const CUtensorMap (&maps)[8], GemmArgs& g, const int64_t* batch, const SplitWorkspace* split,
                cudaStream_t stream) {
     using C = Cfg<BN, kPair>;
     int max_units = 0;
@@ -961,6 +1013,7 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
         GemmProblem& P = g.p[i];
         P.tiles_m = (P.m + C::kTileM - 1) / C::kTileM;
         P.tiles_n = (P.n + BN - 1) / BN;
+        P.idesc_half = P.idesc | (static_cast<uint32_t>(128 >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
         P.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
         P.tile_begin = static_cast<int>(tiles);
         const int64_t pt = static_cast<int64_t>(P.tiles_m) * P.tiles_n * batch[i];
@@ -1006,9 +1059,28 @@ int launch_cfg(const CUtensorMap (&maps)[6], GemmArgs& g, const int64_t* batch, 
             kernel = fp8_gemm_kernel<BN, kPair, true, false>;
         }
     }
+    // A last round that would keep at most half of the pairs busy runs as twice as many 256 x 128
+    // half tiles (pairs, K-major B, the plain instance): the last epilogue, the launch's tail, is
+    // half as long, and the round's MMAs are spread over more pairs.
+    g.half_begin = g.num_tiles;
+    if (kPair && BN == 256 && !out8 && !g.splitk) {
+        bool k_major_b = true;
+        for (int i = 0; i < g.nprob; ++i) k_major_b = k_major_b && !g.p[i].b_mn;
+        const int64_t T = g.num_tiles, U = units;
+        const int64_t R = (T + U - 1) / U, L = T - (R - 1) * U;
+        // only where the dealt schedule gets shorter: halves that land on pairs already holding
+        // the longest units would lengthen it
+        if (k_major_b && half_tiles_enabled() && R >= 2 && 2 * L <= U &&
+            plain_makespan(g, units, static_cast<int>(T + L), static_cast<int>(T - L)) <
+                0.98 * plain_makespan(g, units, static_cast<int>(T), static_cast<int>(T))) {
+            g.half_begin = static_cast<int>(T - L);
+            g.num_units = static_cast<int>(T + L);
+        }
+    }
     const int grid_units = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g.num_units, units)));
     cudaError_t e = launch_ex(kernel, dim3(static_cast<unsigned>(grid_units * (kPair ? 2 : 1))), dim3(C::kThreads),
-                              C::kSmem, stream, kPair ? 2 : 1, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], g);
+                              C::kSmem, stream, kPair ? 2 : 1, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                              maps[6], maps[7], g);
     if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("fp8 gemm launch: ") + cudaGetErrorString(e));
     return FP8DSA_OK;
 }
@@ -1142,7 +1214,7 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
     const TileChoice tc = choose_tiles(work, nwork);
     const int b_rows = tc.pair ? tc.bn / 2 : tc.bn;  // rows of B each CTA loads
 
-    CUtensorMap maps[6];
+    CUtensorMap maps[8];  // per problem A, B, out; then per problem B in 64-row boxes (half tiles)
     GemmArgs g = fold_args;
     int64_t batch[kMaxProblems] = {1, 1};
     const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -1165,6 +1237,13 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
         else
             rc = make_map(&mb, u8, d.b, d.n, d.k, b_bat ? d.batch : 1, d.ldb, b_bat ? d.stride_b : d.ldb * d.k, 128, kBK);
         if (rc) return rc;
+        if (!d.b_mn && tc.pair && tc.bn == 256) {
+            rc = make_map(&maps[6 + i], u8, d.b, d.k, d.n, b_bat ? d.batch : 1, d.ldb,
+                          b_bat ? d.stride_b : d.ldb * d.n, 128, 64);
+            if (rc) return rc;
+        } else {
+            maps[6 + i] = mb;  // unused: no half tiles
+        }
         // TMA stores need 16-byte aligned rows and batches of the output
         const bool tma_out = d.out != nullptr && aligned16(d.out) && d.ldo % 8 == 0 &&
                              (d.batch == 1 || d.stride_o % 8 == 0);
@@ -1203,7 +1282,7 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
         P.out8_step_used = d.out8_step_used;
         batch[i] = d.batch;
     }
-    for (int i = nwork; i < kMaxProblems; ++i) maps[3 * i] = maps[3 * i + 1] = maps[3 * i + 2] = maps[0];
+    for (int i = nwork; i < kMaxProblems; ++i) maps[3 * i] = maps[3 * i + 1] = maps[3 * i + 2] = maps[6 + i] = maps[0];
     g.nprob = nwork;
     if (colsum) {
         g.colsum.partial = colsum_partial;

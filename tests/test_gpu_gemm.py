@@ -112,6 +112,14 @@ def test_batched_and_broadcast(bcast, layout):
     _run(layout, "e4m3", "e4m3", 130, 200, 160, batch=3, bcast=bcast, seed=7)
 
 
+@pytest.mark.parametrize("layout", ["NT", "TN"])
+def test_last_round_half_tiles(layout):
+    """80 pair tiles of 256 x 256 on the 74 pairs of a B200: the last round's 6 tiles run as 12
+    halves of 256 x 128 (K-major B).  Ragged M and N: the last tile column holds 96 valid
+    columns, so one of its halves lies wholly past n (nothing may be written there)."""
+    _run(layout, "e4m3", "e4m3", 2000, 2400, 384, bias="bf16", seed=21)
+
+
 def test_k_zero_writes_bias():
     _run("NT", "e4m3", "e4m3", 70, 90, 0, bias="bf16")
     _run("NT", "e4m3", "e4m3", 70, 90, 0, bias=None)
