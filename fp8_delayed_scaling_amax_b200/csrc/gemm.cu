@@ -1060,10 +1060,10 @@ int launch_cfg(const CUtensorMap (&maps)[8], GemmArgs& g, const int64_t* batch, 
         }
     }
     // A last round that would keep at most half of the pairs busy runs as twice as many 256 x 128
-    // half tiles (pairs, K-major B, the plain instance): the last epilogue, the launch's tail, is
+    // half tiles (pairs, K-major B, no split-K): the last epilogue, the launch's tail, is
     // half as long, and the round's MMAs are spread over more pairs.
     g.half_begin = g.num_tiles;
-    if (kPair && BN == 256 && !out8 && !g.splitk) {
+    if (kPair && BN == 256 && !g.splitk) {
         bool k_major_b = true;
         for (int i = 0; i < g.nprob; ++i) k_major_b = k_major_b && !g.p[i].b_mn;
         const int64_t T = g.num_tiles, U = units;
