@@ -1068,9 +1068,10 @@ int launch_cfg(const CUtensorMap (&maps)[8], GemmArgs& g, const int64_t* batch, 
         for (int i = 0; i < g.nprob; ++i) k_major_b = k_major_b && !g.p[i].b_mn;
         const int64_t T = g.num_tiles, U = units;
         const int64_t R = (T + U - 1) / U, L = T - (R - 1) * U;
-        // only where the dealt schedule gets shorter: halves that land on pairs already holding
-        // the longest units would lengthen it
-        if (k_major_b && half_tiles_enabled() && R >= 2 && 2 * L <= U &&
+        // only where the dealt schedule gets shorter (halves that land on pairs already holding
+        // the longest units would lengthen it), and only for launches of at most 8 rounds, so
+        // the model stays cheap and the tail it trims is still a visible share of the launch
+        if (k_major_b && half_tiles_enabled() && R >= 2 && R <= 8 && 2 * L <= U &&
             plain_makespan(g, units, static_cast<int>(T + L), static_cast<int>(T - L)) <
                 0.98 * plain_makespan(g, units, static_cast<int>(T), static_cast<int>(T))) {
             g.half_begin = static_cast<int>(T - L);
