@@ -287,3 +287,165 @@ def test_fp8_output_gemm_is_the_quantized_bf16_output():
             prod = np.float32(np.float32(y[i, j]) * mult)
             assert out8[i, j] == C.encode(np.array([prod], np.float64), "e5m2")[0]
     assert np.float32(am) == np.float32(np.max(np.abs(y)))
+
+
+# --- pre-quantized operands (AstrAI astrai/extension commit log: linear_forward_fp8 accepts a
+# pre-quantized w8 in the forward's format, skips the weight quantize and reports amax_w = 0;
+# the bias may be fp8 with bias_scale; the backward takes g / x / w as bf16 or fp8 in its
+# format, and a pre-quantized g folds no ring, reports amax_g = 0 and is dequantized before
+# the bias-gradient sum) ---------------------------------------------------------------------
+
+def _dec(codes, fmt):
+    return [[Fraction(C.decode_code(int(c), fmt)) for c in row] for row in np.atleast_2d(codes)]
+
+
+def test_forward_prequantized_weight_is_the_quantized_path():
+    """A weight quantized beforehand at the ring's step gives the same bytes, output and x ring
+    as quantizing it inside the forward; the weight's ring is left alone and amax_w is 0."""
+    rng = np.random.default_rng(40)
+    m, k, n = 24, 48, 40
+    x = _bits(rng.standard_normal((m, k)))
+    w = _bits(rng.standard_normal((n, k)) * 0.02)
+    b = _bits(rng.standard_normal(n) * 0.1)
+    wv = C.bf16_bits_to_f64(w).astype(np.float32)
+    xv = C.bf16_bits_to_f64(x).astype(np.float32)
+    rx1, rw1, rx2, rw2 = S.Ring(4, "e4m3"), S.Ring(4, "e4m3"), S.Ring(4, "e4m3"), S.Ring(4, "e4m3")
+    for r in (rx1, rx2):
+        r.seed(xv)
+    for r in (rw1, rw2):
+        r.seed(wv)
+    sw = rw1.scale
+    w8, _ = Q.quantize(wv, sw, "e4m3")
+    rw2_before = rw2.state.copy()
+    ref = L.forward(x, w, b, "e4m3", rx1, rw1)
+    pre = L.forward(x, None, b, "e4m3", rx2, rw2, w8=w8, w_step=sw)
+    assert np.array_equal(ref["y"], pre["y"]) and np.array_equal(ref["s_abs"], pre["s_abs"])
+    assert np.array_equal(ref["x8"], pre["x8"]) and np.array_equal(pre["w8"], w8)
+    assert pre["sw"] == sw and pre["amax_w"] == 0.0 and ref["amax_w"] > 0.0
+    assert np.array_equal(rx1.state.view(np.uint32), rx2.state.view(np.uint32))
+    assert np.array_equal(rw2.state.view(np.uint32), rw2_before.view(np.uint32))
+    # dynamic scaling: x is measured, the weight keeps the step it came with
+    sw_dyn = S.dynamic_scale(wv, "e4m3")
+    w8d, _ = Q.quantize(wv, sw_dyn, "e4m3")
+    assert np.array_equal(L.forward(x, w, b, "e4m3")["y"],
+                          L.forward(x, None, b, "e4m3", w8=w8d, w_step=sw_dyn)["y"])
+
+
+def test_forward_prequantized_weight_and_fp8_bias_brute_force():
+    """y = x8 . w8^T * RN32(sx * w_step) + dec(b8) * bias_scale, exactly (tiny shapes)."""
+    rng = np.random.default_rng(41)
+    for m, k, n in ((2, 16, 3), (5, 32, 7)):
+        x = _bits(rng.standard_normal((m, k)))
+        w8 = _rand_codes(rng, (n, k), "e4m3")
+        b8 = _rand_codes(rng, (n,), "e4m3")
+        w_step, bias_scale = np.float32(0.013), np.float32(0.0371)
+        out = L.forward(x, None, b8, "e4m3", w8=w8, w_step=w_step, bias_scale=bias_scale)
+        sc = Fraction(float(np.float32(out["sx"]) * w_step))
+        xs, ws, bs = _dec(out["x8"], "e4m3"), _dec(w8, "e4m3"), _dec(b8, "e4m3")[0]
+        for i in range(m):
+            for j in range(n):
+                exact = sum(xs[i][p] * ws[j][p] for p in range(k)) * sc + bs[j] * Fraction(float(bias_scale))
+                assert abs(Fraction(out["y"][i, j]) - exact) <= abs(exact) * Fraction(2) ** -50 + Fraction(2) ** -80
+
+
+def test_dynamic_steps_use_each_formats_fp8_max():
+    """Closed forms from FP8_MAX = 448 (E4M3) and 57344 (E5M2): planted maxima make every
+    dynamic step a power of two, and the planted element encodes as the format's largest
+    code.  The backward re-measures g, x and w at E5M2's maximum."""
+    rng = np.random.default_rng(42)
+    m, k, n = 32, 48, 40
+    gv = rng.standard_normal((m, n)) * 1e-3
+    xv = rng.standard_normal((m, k))
+    wv = rng.standard_normal((n, k)) * 0.02
+    gv[3, 5] = -57344.0 * 2.0 ** -10   # amax(g) = 56
+    xv[7, 9] = 57344.0 * 2.0 ** -3     # amax(x) = 7168
+    wv[11, 2] = 57344.0 * 2.0 ** -12   # amax(w) = 14
+    g, x, w = _bits(gv), _bits(xv), _bits(wv)
+    bwd = L.backward(g, x, w, "e5m2")
+    assert (bwd["sg"], bwd["sx"], bwd["sw"]) == (2.0 ** -10, 2.0 ** -3, 2.0 ** -12)
+    assert bwd["g8"][3, 5] == 0xFB and bwd["x8t"][9, 7] == 0x7B and bwd["w8t"][2, 11] == 0x7B
+    xf = xv.copy()
+    xf[7, 9] = 448.0 * 2.0 ** -2      # amax(x) = 112 in the forward (E4M3)
+    wf = wv.copy()
+    wf[11, 2] = 448.0 * 2.0 ** -7     # amax(w) = 3.5
+    fwd = L.forward(_bits(xf), _bits(wf), None, "e4m3")
+    assert (fwd["sx"], fwd["sw"]) == (2.0 ** -2, 2.0 ** -7)
+    assert fwd["x8"][7, 9] == 0x7E and fwd["w8"][11, 2] == 0x7E
+
+
+def test_backward_prequant_all_bf16_is_the_backward():
+    rng = np.random.default_rng(43)
+    m, k, n = 48, 32, 40
+    g = _bits(rng.standard_normal((m, n)) * 1e-3)
+    x = _bits(rng.standard_normal((m, k)))
+    w = _bits(rng.standard_normal((n, k)) * 0.02)
+    for delayed in (False, True):
+        r1, r2 = (S.Ring(4, "e5m2"), S.Ring(4, "e5m2")) if delayed else (None, None)
+        if delayed:
+            for r in (r1, r2):
+                r.seed(C.bf16_bits_to_f64(g).astype(np.float32))
+        sx, sw = (np.float32(3e-3), np.float32(1.1e-4)) if delayed else (None, None)
+        ref = L.backward(g, x, w, "e5m2", sx, sw, r1)
+        got = L.backward_prequant(g, x, w, "e5m2", sx=sx, sw=sw, ring_g=r2)
+        for key in ("dx", "dw", "dx_abs", "dw_abs", "grad_b", "g8"):
+            assert np.array_equal(ref[key], got[key]), key
+        assert (ref["sg"], ref["sx"], ref["sw"], ref["amax_g"]) == (got["sg"], got["sx"], got["sw"], got["amax_g"])
+        if delayed:
+            assert np.array_equal(r1.state.view(np.uint32), r2.state.view(np.uint32))
+
+
+def test_backward_prequant_operands_skip_their_quantize():
+    """Operands quantized beforehand at the same steps give the same grad_x / grad_w; a
+    pre-quantized g leaves the ring alone, reports amax_g = 0, and its grad_b is the column
+    sum of the dequantized bytes."""
+    rng = np.random.default_rng(44)
+    m, k, n = 40, 32, 48
+    gv = rng.standard_normal((m, n)) * 1e-3
+    g, x, w = _bits(gv), _bits(rng.standard_normal((m, k))), _bits(rng.standard_normal((n, k)) * 0.02)
+    sx, sw = np.float32(2.5e-3), np.float32(9e-5)
+    ring = S.Ring(4, "e5m2")
+    ring.seed(C.bf16_bits_to_f64(g).astype(np.float32))
+    sg = ring.scale
+    ref = L.backward(g, x, w, "e5m2", sx, sw, ring)
+    g8, _ = Q.quantize(C.bf16_bits_to_f64(g).astype(np.float32), sg, "e5m2")
+    x8, _ = Q.quantize(C.bf16_bits_to_f64(x).astype(np.float32), sx, "e5m2")
+    w8, _ = Q.quantize(C.bf16_bits_to_f64(w).astype(np.float32), sw, "e5m2")
+    for fl in ((1, 0, 0), (0, 1, 0), (0, 0, 1), (1, 1, 1)):
+        ops = [g8 if fl[0] else g, x8 if fl[1] else x, w8 if fl[2] else w]
+        r2 = S.Ring(4, "e5m2")
+        r2.seed(C.bf16_bits_to_f64(g).astype(np.float32))
+        before = r2.state.copy()
+        got = L.backward_prequant(*ops, "e5m2", *map(bool, fl), g_step=sg, sx=sx, sw=sw, ring_g=r2)
+        assert np.array_equal(ref["dx"], got["dx"]) and np.array_equal(ref["dw"], got["dw"]), fl
+        if fl[0]:
+            assert got["amax_g"] == 0.0
+            assert np.array_equal(r2.state.view(np.uint32), before.view(np.uint32))
+            want = C.round_to_bf16((C.decode(g8, "e5m2") * float(sg)).sum(0))
+            assert np.array_equal(got["grad_b"], want)
+        else:
+            assert got["amax_g"] == ref["amax_g"] and np.array_equal(got["grad_b"], ref["grad_b"])
+    # closed form: every code 1.0 at step 2^-7 over m rows sums to m * 2^-7 in every column
+    ones = np.full((m, n), 0x3C, np.uint8)
+    got = L.backward_prequant(ones, x, w, "e5m2", True, False, False, g_step=2.0 ** -7, sx=sx, sw=sw)
+    assert np.all(got["grad_b"] == m * 2.0 ** -7)
+
+
+def test_backward_prequant_equals_exact_brute_force():
+    rng = np.random.default_rng(45)
+    for m, k, n in ((2, 3, 4), (6, 5, 7)):
+        g8 = _rand_codes(rng, (m, n), "e5m2")
+        x8 = _rand_codes(rng, (m, k), "e5m2")
+        w8 = _rand_codes(rng, (n, k), "e5m2")
+        sg, sx, sw = np.float32(3e-5), np.float32(0.07), np.float32(2e-3)
+        out = L.backward_prequant(g8, x8, w8, "e5m2", True, True, True, g_step=sg, sx=sx, sw=sw)
+        gs, xs, ws = _dec(g8, "e5m2"), _dec(x8, "e5m2"), _dec(w8, "e5m2")
+        sc_x = Fraction(float(sg * sw))
+        sc_w = Fraction(float(sg * sx))
+        for i in range(m):
+            for j in range(k):
+                exact = sum(gs[i][p] * ws[p][j] for p in range(n)) * sc_x
+                assert abs(Fraction(out["dx"][i, j]) - exact) <= Fraction(2) ** -45 * Fraction(float(out["dx_abs"][i, j])) * sc_x
+        for i in range(n):
+            for j in range(k):
+                exact = sum(gs[p][i] * xs[p][j] for p in range(m)) * sc_w
+                assert abs(Fraction(out["dw"][i, j]) - exact) <= Fraction(2) ** -45 * Fraction(float(out["dw_abs"][i, j])) * sc_w
