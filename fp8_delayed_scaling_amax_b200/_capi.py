@@ -55,6 +55,9 @@ _SIGNATURES = {
     "linear_backward_fp8_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_backward_fp8": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, _P, _P,
                                     POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P, _P]),
+    "linear_backward_fp8_prequant": (c_int, [_P, c_int, _P, _P, c_int, _P, c_int, c_int64, c_int64, c_int64, c_int,
+                                             c_int, c_int, c_int, _P, _P, POINTER(fp8_ring_t), c_float, _P, _P,
+                                             c_size_t, _P, _P, _P, _P]),
     "linear_forward_fp8_keep": (c_int, [_P, _P, c_int, _P, _P, _P, c_int64, c_int64, c_int64, c_int,
                                         POINTER(fp8_ring_t), POINTER(fp8_ring_t), c_float, _P, _P, _P, _P, _P,
                                         c_size_t, _P, _P]),
@@ -252,6 +255,17 @@ def linear_backward_fp8(g, x, w, m, k, n, fmt, need_grad_x, need_grad_w, need_gr
         _ptr(g), _ptr(x), _ptr(w), int(m), int(k), int(n), int(fmt), int(bool(need_grad_x)), int(bool(need_grad_w)),
         int(bool(need_grad_b)), _ptr(sx_fwd), _ptr(sw_fwd), _ring(g_ring), float(pow2_margin), _ptr(sg_used),
         _ptr(workspace), int(workspace_bytes), _ptr(grad_x), _ptr(grad_w), _ptr(grad_b), _stream(stream)))
+
+
+def linear_backward_fp8_prequant(g, g_is_fp8, g_step, x, x_is_fp8, w, w_is_fp8, m, k, n, fmt, need_grad_x,
+                                 need_grad_w, need_grad_b, sx_fwd, sw_fwd, g_ring, pow2_margin, sg_used, workspace,
+                                 workspace_bytes, grad_x, grad_w, grad_b, stream=None):
+    """linear_backward_fp8 where g / x / w may each be fp8 bytes in fmt (flags *_is_fp8)."""
+    return _check("linear_backward_fp8_prequant", lib().linear_backward_fp8_prequant(
+        _ptr(g), int(bool(g_is_fp8)), _ptr(g_step), _ptr(x), int(bool(x_is_fp8)), _ptr(w), int(bool(w_is_fp8)),
+        int(m), int(k), int(n), int(fmt), int(bool(need_grad_x)), int(bool(need_grad_w)), int(bool(need_grad_b)),
+        _ptr(sx_fwd), _ptr(sw_fwd), _ring(g_ring), float(pow2_margin), _ptr(sg_used), _ptr(workspace),
+        int(workspace_bytes), _ptr(grad_x), _ptr(grad_w), _ptr(grad_b), _stream(stream)))
 
 
 def linear_forward_fp8_keep(x, w, w_is_fp8, w_step, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, pow2_margin,

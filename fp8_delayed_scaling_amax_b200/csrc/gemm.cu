@@ -1302,7 +1302,7 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
         rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, split, stream)
                           : launch_cfg<128, false>(maps, g, batch, split, stream);
     if (rc) return rc;
-    launch_end(kKindGemm, stream, flops);
+    launch_end(tc.pair ? kKindGemmPair : kKindGemmSingle, stream, flops);
     return check_launch("fp8 gemm kernel");
 }
 

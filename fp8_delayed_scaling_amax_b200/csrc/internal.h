@@ -30,8 +30,11 @@ int current_device();
 // WaitCtl for the current device (status word address + timeout).
 int wait_ctl(WaitCtl* ctl);
 
-// Kernel classes for the optional per-kernel timing.
-enum KernelKind : int { kKindQuantize = 0, kKindGemm = 1, kKindOther = 2 };
+// Kernel classes for the optional per-kernel timing.  GEMM launches are recorded under the
+// instance they ran (256-wide tiles on CTA pairs, or single-CTA tiles); reading kKindGemm
+// returns both.
+enum KernelKind : int { kKindQuantize = 0, kKindGemm = 1, kKindOther = 2, kKindGemmPair = 3, kKindGemmSingle = 4 };
+constexpr int kNumKinds = 5;
 
 // Bracket a launch with timing events when profiling is on.  `work` is the algorithmic
 // bytes (quantize, other) or flops (GEMM) the launch performs.
@@ -143,6 +146,12 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
 // grad_b[c] = RN_bf16(sum_t partial[t][c]) in a fixed order.
 int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, void* out_bf16,
                            cudaStream_t stream);
+
+// Per-tile column sums of fp8 bytes [rows][cols] (format fmt) times *step, in the layout the
+// dual quantize writes ([ceil(rows/128)][cols] fp32), for a bias gradient of a pre-quantized
+// g; `zero` / `zero_words` (optional) are also set to zero.  cols % 4 == 0.
+int launch_colsum_fp8(const uint8_t* g8, fp8_fmt_t fmt, int64_t rows, int64_t cols, const float* step,
+                      float* partial, uint32_t* zero, int64_t zero_words, cudaStream_t stream);
 
 // One GEMM of a launch, arguments already validated.
 struct GemmDesc {

@@ -498,6 +498,160 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
     return FP8DSA_OK;
 }
 
+int linear_backward_fp8_prequant(const void* g, int g_is_fp8, const float* g_step, const void* x, int x_is_fp8,
+                                 const void* w, int w_is_fp8, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
+                                 int need_grad_x, int need_grad_w, int need_grad_b, const float* sx_fwd,
+                                 const float* sw_fwd, const fp8_ring_t* g_ring, float pow2_margin, float* sg_used,
+                                 void* workspace, size_t workspace_bytes, void* grad_x, void* grad_w, void* grad_b,
+                                 cudaStream_t stream) {
+    clear_error();
+    if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
+    if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (w == nullptr || grad_x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
+    if (need_grad_w && (x == nullptr || grad_w == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
+    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
+    if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
+    if (g_is_fp8 && g_step == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "a pre-quantized g needs g_step");
+    const bool dynamic = g_ring == nullptr;
+    // the steps of x and w: the forward's (delayed, or any pre-quantized operand), else measured
+    const bool want_sx = need_grad_w && (!dynamic || x_is_fp8);
+    const bool want_sw = need_grad_x && (!dynamic || w_is_fp8);
+    if ((want_sx && sx_fwd == nullptr) || (want_sw && sw_fwd == nullptr))
+        return fail(FP8DSA_ERR_INVALID_ARG, "sx_fwd / sw_fwd are required (delayed scaling or a pre-quantized x / w)");
+    if ((g_is_fp8 && !aligned16(g)) || (need_grad_w && x_is_fp8 && !aligned16(x)) || (need_grad_x && w_is_fp8 && !aligned16(w)))
+        return fail(FP8DSA_ERR_UNSUPPORTED, "pre-quantized operands must be 16-byte aligned");
+    if (dynamic && !(pow2_margin > 0.0f)) return fail(FP8DSA_ERR_INVALID_ARG, "pow2_margin must be > 0");
+    int rc = check_ring_arg(g_is_fp8 ? nullptr : g_ring, "g_ring");
+    if (rc) return rc;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    const BwdLayout L = bwd_layout(m, k, n);
+    if (workspace_bytes < L.total)
+        return fail(FP8DSA_ERR_WORKSPACE, "workspace too small: need " + std::to_string(L.total) + " bytes");
+    rc = check_device();
+    if (rc) return rc;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* colsum = reinterpret_cast<float*>(ws + L.colsum);
+    uint32_t* scratch = reinterpret_cast<uint32_t*>(ws + L.scratch);
+    float* internal = reinterpret_cast<float*>(ws + L.scratch + 64);
+    // a pre-quantized g is read at its own step; a bf16 g's step is measured or taken from the ring
+    const float* sg = g_is_fp8 ? g_step : (sg_used ? sg_used : internal);
+    const float* sx = sx_fwd;
+    const float* sw = sw_fwd;
+    if (g_is_fp8 && sg_used != nullptr) {
+        cudaError_t e = cudaMemcpyAsync(sg_used, g_step, sizeof(float), cudaMemcpyDeviceToDevice, stream);
+        if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("copy g_step: ") + cudaGetErrorString(e));
+    }
+    if (dynamic) {  // measure the bf16 operands only
+        AmaxJob jobs[3];
+        int nj = 0;
+        auto add = [&](const void* t, int64_t numel, float* out) {
+            jobs[nj].x = t;
+            jobs[nj].numel = numel;
+            jobs[nj].fp8_max = fmt_max(fmt);
+            jobs[nj].pow2_margin = pow2_margin;
+            jobs[nj].scale_out = out;
+            ++nj;
+        };
+        if (!g_is_fp8) add(g, m * n, const_cast<float*>(sg));
+        if (need_grad_w && !x_is_fp8) {
+            add(x, m * k, internal + 1);
+            sx = internal + 1;
+        }
+        if (need_grad_x && !w_is_fp8) {
+            add(w, n * k, internal + 2);
+            sw = internal + 2;
+        }
+        if (nj > 0) {
+            cudaError_t e = cudaMemsetAsync(scratch, 0, 64, stream);
+            if (e != cudaSuccess) return fail(FP8DSA_ERR_CUDA, std::string("memset scratch: ") + cudaGetErrorString(e));
+            rc = launch_amax_jobs(jobs, nj, scratch, stream);
+            if (rc) return rc;
+        }
+    }
+    // the operands the GEMMs read: a bf16 operand's bytes in the workspace (K-major), a
+    // pre-quantized one in place (MN-major where the GEMM needs it transposed)
+    const uint8_t* g8 = g_is_fp8 ? static_cast<const uint8_t*>(g) : ws + L.g8;
+    uint8_t* g8t = ws + L.g8t;
+    uint8_t* x8t = ws + L.x8t;
+    uint8_t* w8t = ws + L.w8t;
+    QuantJob jobs[3];
+    int nq = 0;
+    if (!g_is_fp8) {  // g: both orientations, ring fold, per-tile column sums
+        QuantJob& q = jobs[nq++];
+        q.x = g;
+        q.rows = m;
+        q.cols = n;
+        q.fmt = fmt;
+        q.out = ws + L.g8;
+        q.out_t = g8t;
+        q.colsum_partial = need_grad_b ? colsum : nullptr;
+        if (dynamic) {
+            q.scale = sg;
+        } else {
+            q.scale = g_ring->state + g_ring->hist_len;
+            q.ring = g_ring;
+            q.scale_used_out = const_cast<float*>(sg);
+            q.defer_fold = true;  // folded by the GEMM launch below
+        }
+    }
+    if (need_grad_w && !x_is_fp8) {
+        QuantJob& q = jobs[nq++];
+        q.x = x;
+        q.rows = m;
+        q.cols = k;
+        q.fmt = fmt;
+        q.out_t = x8t;
+        q.scale = sx;
+    }
+    if (need_grad_x && !w_is_fp8) {
+        QuantJob& q = jobs[nq++];
+        q.x = w;
+        q.rows = n;
+        q.cols = k;
+        q.fmt = fmt;
+        q.out_t = w8t;
+        q.scale = sw;
+    }
+    SplitWorkspace split;
+    split.counters = reinterpret_cast<uint32_t*>(ws + L.counters);
+    split.counter_words = L.counter_words;
+    split.partial = reinterpret_cast<float*>(ws + L.partial);
+    split.partial_bytes = L.total - L.partial;
+    bool zeroed = false;  // the split-K counters are zeroed by the first launch below
+    if (nq > 0) {
+        rc = launch_quantize_batch(jobs, nq, stream, split.counters, split.counter_words);
+        if (rc) return rc;
+        zeroed = true;
+    }
+    if (g_is_fp8 && need_grad_b && m > 0) {  // the bias gradient of the dequantized g
+        rc = launch_colsum_fp8(g8, fmt, m, n, g_step, colsum, zeroed ? nullptr : split.counters,
+                               zeroed ? 0 : split.counter_words, stream);
+        if (rc) return rc;
+        zeroed = true;
+    }
+    GemmDesc gd[2];
+    int ng = 0;
+    if (need_grad_x)  // grad_x [m][k] = g8 [m][n] . (w8t [k][n])^T, or . w8 [n][k] read as B = [K][N]
+        gd[ng++] = w_is_fp8 ? GemmDesc{g8, static_cast<const uint8_t*>(w), fmt, fmt, 0, 1, m, k, n, n, k, k, 1, 0, 0, 0,
+                                       sg, sw, nullptr, 0, nullptr, grad_x}
+                            : GemmDesc{g8, w8t, fmt, fmt, 0, 0, m, k, n, n, n, k, 1, 0, 0, 0, sg, sw, nullptr, 0,
+                                       nullptr, grad_x};
+    if (need_grad_w) {  // grad_w [n][k] = g^T [n][m] . x [m][k]
+        const uint8_t* a = g_is_fp8 ? g8 : g8t;                  // A = g8 [m][n] as [K][M], or g8t [n][m]
+        const uint8_t* b = x_is_fp8 ? static_cast<const uint8_t*>(x) : x8t;  // B = x8 [m][k] as [K][N], or x8t [k][m]
+        gd[ng++] = GemmDesc{a, b, fmt, fmt, g_is_fp8 ? 1 : 0, x_is_fp8 ? 1 : 0, n, k, m, g_is_fp8 ? n : m,
+                            x_is_fp8 ? k : m, k, 1, 0, 0, 0, sg, sx, nullptr, 0, nullptr, grad_w};
+    }
+    const int64_t tiles = m > 0 ? (m + 127) / 128 : 0;
+    const bool fold = !g_is_fp8 && !dynamic && ring_fold_in_call();
+    return gemm_launch_group(gd, ng, need_grad_b ? colsum : nullptr, need_grad_b ? tiles : 0, need_grad_b ? n : 0,
+                             need_grad_b ? grad_b : nullptr, zeroed ? &split : nullptr, g_ring, fold ? 1 : 0, stream);
+}
+
 size_t linear_backward_fp8_saved_t_workspace_size(int64_t m, int64_t k, int64_t n) {
     if (m < 0 || k < 0 || n < 0) return 0;
     return saved_layout(m, k, n).total;

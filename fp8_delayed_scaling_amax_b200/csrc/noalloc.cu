@@ -1,22 +1,25 @@
 // linear_forward_fp8 for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocator) at the point where they run the
-// forward pass.  Examples: code that runs inside a CUDA stream capture, where allocating is
-// not permitted and a caching allocator may not be reachable; plug-ins embedded in a host
-// application that owns the device-memory budget; and services that must keep a fixed
+// forward pass.  Examples: plug-ins embedded in a host application that owns the
+// device-memory budget and gives them no allocator, and services that must keep a fixed
 // device footprint after start-up.  This entry point takes the same arguments as
 // linear_forward_fp8 except the workspace: its scratch (the x8 / w8 operand buffers and the
 // amax scratch) lives in one file-scope __device__ array of FP8DSA_NOALLOC_WORKSPACE_BYTES,
 // which every GPU that loads the library holds until the process exits.
 //
 // Set-up: the first call on each device looks up that array's device address with
-// cudaGetSymbolAddress, with that device current, and caches it; make that first call
-// before any stream capture.  Afterwards the call enqueues what linear_forward_fp8 enqueues,
-// except that its GEMM never splits K (the array holds only the operand buffers and the
-// scale scratch), and it allocates nothing.  Every call shares the one array, which keeps the
-// last call's contents: the operand buffers are rewritten in full by each call and the
-// dynamic-scaling amax scratch is cleared by each call, but calls that overlap on the GPU
-// (different streams without ordering between them) race on the array.
+// cudaGetSymbolAddress, with that device current, and caches it for the life of the process;
+// make that first call before any stream capture.  The cached address belongs to the device
+// context that first call saw: after cudaDeviceReset (or a primary context released and
+// created again) the library must not be called again in the same process.
+//
+// Afterwards the call enqueues what linear_forward_fp8 enqueues, except that its GEMM never
+// splits K (the array holds only the operand buffers and the scale scratch), and it
+// allocates nothing.  Every call shares the one array, which keeps the last call's contents:
+// the operand buffers are rewritten in full by each call and the dynamic-scaling amax scratch
+// is cleared by each call, but calls that overlap on the GPU (different streams without
+// ordering between them) race on the array.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -63,6 +66,11 @@ extern "C" int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is
                                           float* sw_used, void* y, cudaStream_t stream) {
     clear_error();
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
+    // m * k and n * k must not wrap before they are compared with the array's size
+    constexpr int64_t kCap = static_cast<int64_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES);
+    if (k > 0 && (m > kCap / k || n > kCap / k))
+        return fail(FP8DSA_ERR_WORKSPACE, "linear_forward_fp8_noalloc: m * k or n * k exceeds the built-in array (" +
+                                              std::to_string(kCap) + " bytes)");
     const size_t need = linear_forward_base_workspace(m, k, n);
     if (need > static_cast<size_t>(FP8DSA_NOALLOC_WORKSPACE_BYTES))
         return fail(FP8DSA_ERR_WORKSPACE, "linear_forward_fp8_noalloc: this shape needs " + std::to_string(need) +

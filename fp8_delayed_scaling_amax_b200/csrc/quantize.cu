@@ -811,6 +811,39 @@ __global__ void __launch_bounds__(kThreads) colsum_finalize_kernel(const float* 
     out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
 }
 
+// Per-tile column sums of a pre-quantized operand (the bias gradient of a g that arrives as
+// fp8): partial[t][c] = RN32(sum over the rows r of tile t of dec(g8[r][c])) * step, rows in
+// order.  Each thread sums four adjacent columns of one 128-row tile (a warp reads 128
+// contiguous bytes per row); block (0, 0) also zeroes `zero[0 .. zero_words)`.
+template <int kFmt>
+__global__ void __launch_bounds__(kThreads) colsum_fp8_kernel(const uint8_t* g8, int64_t rows, int64_t cols,
+                                                              const float* step, float* partial, uint32_t* zero,
+                                                              int64_t zero_words) {
+    pdl_trigger();
+    pdl_wait();
+    if (zero_words > 0 && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int64_t i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
+    const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    if (c >= cols) return;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTile;
+    const int64_t r1 = r0 + kTile < rows ? r0 + kTile : rows;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    for (int64_t r = r0; r < r1; ++r) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(g8 + r * cols + c));
+        s0 += fp8_to_float<kFmt>(static_cast<uint8_t>(v));
+        s1 += fp8_to_float<kFmt>(static_cast<uint8_t>(v >> 8));
+        s2 += fp8_to_float<kFmt>(static_cast<uint8_t>(v >> 16));
+        s3 += fp8_to_float<kFmt>(static_cast<uint8_t>(v >> 24));
+    }
+    const float st = __ldg(step);
+    float4 out;
+    out.x = __fmul_rn(s0, st);
+    out.y = __fmul_rn(s1, st);
+    out.z = __fmul_rn(s2, st);
+    out.w = __fmul_rn(s3, st);
+    *reinterpret_cast<float4*>(partial + static_cast<int64_t>(blockIdx.y) * cols + c) = out;
+}
+
 // Waves of resident blocks a row-major launch is sized to (measured on B200: one wave, each
 // block looping over its share, beats several waves of shorter blocks).
 constexpr int kFlatWaves = 1;
@@ -1073,6 +1106,25 @@ int launch_colsum_finalize(const float* partial, int64_t tiles, int64_t cols, vo
               static_cast<uint16_t*>(out_bf16));
     launch_end(kKindOther, stream, static_cast<double>(tiles) * cols * 4 + cols * 2);
     return check_launch("colsum finalize kernel");
+}
+
+int launch_colsum_fp8(const uint8_t* g8, fp8_fmt_t fmt, int64_t rows, int64_t cols, const float* step,
+                      float* partial, uint32_t* zero, int64_t zero_words, cudaStream_t stream) {
+    if (rows <= 0 || cols <= 0) return FP8DSA_OK;
+    if (cols % 4 != 0 || (reinterpret_cast<uintptr_t>(g8) & 3) != 0 || (reinterpret_cast<uintptr_t>(partial) & 15) != 0)
+        return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 column sums need cols % 4 == 0, a 4-byte aligned g8 and 16-byte aligned partials");
+    const int64_t tiles = (rows + kTile - 1) / kTile;
+    if (tiles > 65535) return fail(FP8DSA_ERR_UNSUPPORTED, "too many row tiles for the fp8 column sums");
+    const dim3 grid(static_cast<unsigned>((cols / 4 + kThreads - 1) / kThreads), static_cast<unsigned>(tiles));
+    launch_begin(kKindOther, stream);
+    if (fmt == FP8_E4M3)
+        launch_ex(colsum_fp8_kernel<0>, grid, dim3(kThreads), 0, stream, 1, g8, rows, cols, step, partial, zero,
+                  zero != nullptr ? zero_words : int64_t(0));
+    else
+        launch_ex(colsum_fp8_kernel<1>, grid, dim3(kThreads), 0, stream, 1, g8, rows, cols, step, partial, zero,
+                  zero != nullptr ? zero_words : int64_t(0));
+    launch_end(kKindOther, stream, static_cast<double>(rows) * cols + static_cast<double>(tiles) * cols * 4);
+    return check_launch("fp8 column-sum kernel");
 }
 
 }  // namespace fp8dsa

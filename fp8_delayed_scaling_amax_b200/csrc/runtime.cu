@@ -32,7 +32,7 @@ struct TimedLaunch {
     double work;
 };
 std::atomic<bool> g_profile{false};
-std::vector<TimedLaunch> g_timed[3];
+std::vector<TimedLaunch> g_timed[kNumKinds];
 std::vector<cudaEvent_t> g_event_pool;
 thread_local cudaEvent_t t_pending_start = nullptr;
 
@@ -266,24 +266,28 @@ int fp8_profiler_enable(int on) {
 
 int fp8_profiler_read(int kind, double* total_ms, int64_t* launches, double* work) {
     clear_error();
-    if (kind < 0 || kind > 2) return fail(FP8DSA_ERR_INVALID_ARG, "kind must be 0, 1 or 2");
+    if (kind < 0 || kind >= kNumKinds) return fail(FP8DSA_ERR_INVALID_ARG, "kind must be 0 .. 4");
     std::lock_guard<std::mutex> lock(g_mutex);
     double ms_sum = 0.0, work_sum = 0.0;
     int64_t count = 0;
     int rc = FP8DSA_OK;
-    for (auto& t : g_timed[kind]) {
-        cudaError_t e = cudaEventSynchronize(t.stop);
-        float ms = 0.f;
-        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, t.start, t.stop);
-        if (e != cudaSuccess && rc == FP8DSA_OK)
-            rc = fail(FP8DSA_ERR_CUDA, std::string("profiler event: ") + cudaGetErrorString(e));
-        ms_sum += ms;
-        work_sum += t.work;
-        ++count;
-        g_event_pool.push_back(t.start);
-        g_event_pool.push_back(t.stop);
+    const int kinds[2] = {kind == kKindGemm ? kKindGemmPair : kind, kind == kKindGemm ? kKindGemmSingle : -1};
+    for (int kk : kinds) {
+        if (kk < 0) continue;
+        for (auto& t : g_timed[kk]) {
+            cudaError_t e = cudaEventSynchronize(t.stop);
+            float ms = 0.f;
+            if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, t.start, t.stop);
+            if (e != cudaSuccess && rc == FP8DSA_OK)
+                rc = fail(FP8DSA_ERR_CUDA, std::string("profiler event: ") + cudaGetErrorString(e));
+            ms_sum += ms;
+            work_sum += t.work;
+            ++count;
+            g_event_pool.push_back(t.start);
+            g_event_pool.push_back(t.stop);
+        }
+        g_timed[kk].clear();
     }
-    g_timed[kind].clear();
     if (total_ms) *total_ms = ms_sum;
     if (launches) *launches = count;
     if (work) *work = work_sum;

@@ -206,18 +206,19 @@ int linear_forward_fp8(const void* x, const void* w, int w_is_fp8, const float* 
 /* Size of the scratch array linear_forward_fp8_noalloc uses instead of a caller workspace. */
 #define FP8DSA_NOALLOC_WORKSPACE_BYTES (16u << 20)
 
-/* linear_forward_fp8 for callers that cannot allocate device memory -- for example code that
- * runs inside a CUDA stream capture (where allocating is not allowed), a plug-in whose host
- * application owns the device-memory budget, or a service that must keep a fixed device
- * footprint.  The pages have no counterpart to this entry point.
+/* linear_forward_fp8 for callers that cannot allocate device memory -- for example a plug-in
+ * whose host application owns the device-memory budget and hands it no allocator, or a
+ * service that must keep a fixed device footprint after start-up.  The pages have no
+ * counterpart to this entry point.
  * Same arguments and results as linear_forward_fp8, without the workspace: the scratch lives
  * in one built-in device array of FP8DSA_NOALLOC_WORKSPACE_BYTES (16 MiB), held by every GPU
  * that loads the library until the process exits.  The array holds the x8 / w8 operand
  * buffers and the scale scratch (about m*k + n*k bytes), and the GEMM here never splits K;
  * shapes whose buffers exceed the array return FP8DSA_ERR_WORKSPACE with a message.
- * The first call on each device looks up the array's address (make it before any stream
- * capture); no call allocates.  All calls share the array: calls ordered on one stream are
- * safe, calls that overlap on the GPU race. */
+ * The first call on each device looks up the array's address and caches it for the process
+ * (make that call before any stream capture; the address belongs to the device context it
+ * saw, so do not call again after cudaDeviceReset); no call allocates.  All calls share the
+ * array: calls ordered on one stream are safe, calls that overlap on the GPU race. */
 int linear_forward_fp8_noalloc(const void* x, const void* w, int w_is_fp8, const float* w_step,
                                const void* bias, const float* bias_scale, int64_t m, int64_t k,
                                int64_t n, fp8_fmt_t fmt, const fp8_ring_t* x_ring,
@@ -265,6 +266,36 @@ int linear_forward_fp8_keep(const void* x, const void* w, int w_is_fp8, const fl
                             const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                             float* sw_used, uint8_t* x8_out, uint8_t* w8_out, void* workspace,
                             size_t workspace_bytes, void* y, cudaStream_t stream);
+
+/* FP8 linear backward whose operands may each arrive pre-quantized [AstrAI astrai/extension
+ * commit log: g / x / w may each be bf16 or pre-quantized fp8 matching fmt, and a
+ * pre-quantized operand skips its quantize kernel; a pre-quantized g dequantizes before the
+ * bias-sum; compare view, the linear backward binding in an earlier state: a pre-quantized g
+ * does not finalize its ring and reports amax_g = 0]:
+ *   g: dev [m][n], bf16, or fp8 bytes in fmt (g_is_fp8) at step *g_step;
+ *   x: dev [m][k], bf16, or fp8 bytes in fmt (x_is_fp8) at step *sx_fwd;
+ *   w: dev [n][k], bf16, or fp8 bytes in fmt (w_is_fp8) at step *sw_fwd.
+ *   A bf16 operand is quantized as in linear_backward_fp8 (g in both orientations at the
+ *   ring's step, folding g_ring, or at its dynamic step; x / w transposed at sx_fwd / sw_fwd,
+ *   or at their dynamic steps when g_ring == NULL).  A pre-quantized operand is read by the
+ *   GEMM in place (as an MN-major operand where the product needs its transpose); a
+ *   pre-quantized g leaves g_ring untouched (neither read nor folded) and *sg_used = *g_step.
+ *       grad_x [m][k] = g8 . w8 * RN32(sg * sw)
+ *       grad_w [n][k] = g8^T . x8 * RN32(sg * sx)
+ *       grad_b [n]    = RN_bf16(sum over rows of g), a pre-quantized g summed as dec(g8) * sg
+ *   sx_fwd / sw_fwd: required for grad_w / grad_x under delayed scaling and whenever x / w
+ *   is pre-quantized.  Pre-quantized operands must be 16-byte aligned.  workspace: dev,
+ *   >= linear_backward_fp8_workspace_size(m, k, n) bytes, 256-byte aligned.  k and n must be
+ *   multiples of 16 (m too for grad_w).  Launches: at most one amax launch (dynamic), one
+ *   quantize launch for the bf16 operands, one column-sum launch for a pre-quantized g's
+ *   grad_b, and one GEMM launch for grad_x and grad_w. */
+int linear_backward_fp8_prequant(const void* g, int g_is_fp8, const float* g_step, const void* x,
+                                 int x_is_fp8, const void* w, int w_is_fp8, int64_t m, int64_t k,
+                                 int64_t n, fp8_fmt_t fmt, int need_grad_x, int need_grad_w,
+                                 int need_grad_b, const float* sx_fwd, const float* sw_fwd,
+                                 const fp8_ring_t* g_ring, float pow2_margin, float* sg_used,
+                                 void* workspace, size_t workspace_bytes, void* grad_x,
+                                 void* grad_w, void* grad_b, cudaStream_t stream);
 
 /* Workspace bytes linear_backward_fp8_mixed needs for (m, k, n): g8, the per-tile column sums,
  * scale scratch and the GEMM's split-K region. */
@@ -382,8 +413,9 @@ int fp8_debug_stalled_wait(cudaStream_t stream);
  * events on its own stream (inside a stream capture, by external event-record nodes, so each
  * replay of the graph re-times them).  fp8_profiler_read synchronises, returns the total
  * device milliseconds, launch count and algorithmic bytes (quantize, other) or flops (GEMM)
- * of kernel class `kind` (0 quantize, 1 GEMM, 2 other) recorded since the last read, then
- * resets that class.  Not on the pages (they time with CUDA events from Python; [by-author]). */
+ * of kernel class `kind` recorded since the last read, then resets that class: 0 quantize,
+ * 1 GEMM (both instances), 2 other, 3 the GEMM instance with 256-wide tiles on CTA pairs,
+ * 4 the GEMM instance with single-CTA tiles.  Not on the pages (they time with CUDA events from Python; [by-author]). */
 int fp8_profiler_enable(int on);
 int fp8_profiler_read(int kind, double* total_ms, int64_t* launches, double* bytes_or_flops);
 

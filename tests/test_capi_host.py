@@ -146,6 +146,33 @@ def test_keep_forward_and_mixed_backward_argument_checks():
     assert call(margin=0.0) == INVALID       # dynamic scaling needs a positive margin
 
 
+def test_prequant_backward_argument_checks():
+    pb = F.lib().linear_backward_fp8_prequant
+    wsb = F.linear_backward_fp8_workspace_size(64, 64, 64)
+    ring = F.fp8_ring_t(256, 16, 0, 57344.0, 1.0)
+    args = dict(g=256, gf=1, gs=512, x=4096, xf=0, w=8192, wf=0, m=64, k=64, n=64, fmt=1, gx=1, gw=1, gb=1,
+                sx=768, sw=1024, ring=ctypes.byref(ring), margin=1.0, sg=None, ws=1024, wsb=wsb, dx=16384, dw=32768,
+                db=65536)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return pb(a["g"], a["gf"], a["gs"], a["x"], a["xf"], a["w"], a["wf"], a["m"], a["k"], a["n"], a["fmt"],
+                  a["gx"], a["gw"], a["gb"], a["sx"], a["sw"], a["ring"], a["margin"], a["sg"], a["ws"], a["wsb"],
+                  a["dx"], a["dw"], a["db"], None)
+    assert call(fmt=7) == INVALID
+    assert call(gs=None) == INVALID            # a pre-quantized g needs its step
+    assert call(sx=None) == INVALID            # delayed scaling needs the forward's steps
+    assert call(ring=None, xf=1, sx=None) == INVALID  # a pre-quantized x needs its step even when dynamic
+    assert call(g=260) == UNSUPPORTED          # pre-quantized g not 16-byte aligned
+    assert call(xf=1, x=4100) == UNSUPPORTED   # pre-quantized x not 16-byte aligned
+    assert call(n=40) == UNSUPPORTED
+    assert call(m=40) == UNSUPPORTED           # grad_w needs m % 16 == 0
+    assert call(ws=1040) == UNSUPPORTED
+    assert call(wsb=wsb - 256) == WORKSPACE
+    assert call(db=None) == INVALID
+    assert call(ring=None, gf=0, margin=0.0) == INVALID
+
+
 def test_saved_transpose_forward_and_backward_argument_checks():
     lib = F.lib()
     ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
