@@ -6,20 +6,22 @@ gradient) of every linear of a 12-layer, dim-1024 transformer trained at batch 4
 tokens (M = 2048 rows); per layer the (K, N) = (1024, 3072), (1024, 1024), (1024, 4096),
 (4096, 1024) projections.  HYBRID formats (E4M3 forward, E5M2 backward), delayed scaling with
 history 16 and margin 0, bias fused into the forward GEMM.  Per linear and step (default
-``--path saved``): one quantize launch (x and w, each written row-major in E4M3 and transposed
-in E5M2 with the forward's steps) + one GEMM launch forward (the GEMM also folds the two
-rings), one quantize launch (g in both orientations with per-tile column sums) + one GEMM
-launch (dX and dW, grad_b reduced by its epilogue warps, the g ring folded) backward.
-``--path requant`` runs the pages' own split of the same work (the forward quantizes x, w
-row-major; the backward re-quantizes x^T, w^T beside g); both give identical numbers, and the
-line reports the other one as a variant.
+``--path rowmajor``): one row-major quantize launch (x and w, each written in E4M3 for the
+forward and in E5M2 with the forward's steps for the backward, from the same products) + one
+GEMM launch forward (the GEMM also folds the two rings), one quantize launch (g row-major with
+per-tile column sums) + one GEMM launch backward (dX = g8 . w8 and dW = g8^T . x8 with the
+operands read in place as MN-major tiles, grad_b reduced by its epilogue warps, the g ring
+folded).  ``--path saved`` writes x^T / w^T in the forward instead and quantizes g in both
+orientations; ``--path requant`` runs the pages' own split of the same work (the forward
+quantizes x, w row-major; the backward re-quantizes x^T, w^T beside g).  All three give the
+same numbers (the pages' HYBRID backward), and the line reports the other two as variants.
 
 Timing: every layer has its own weights, activations and gradients (about 3 GB, far above
 the 126 MB L2).  The step is captured as CUDA graphs (one per history-ring slot, since the
 slot index is a host-side argument) and replayed; device time from CUDA events with a
 synchronize on both sides, max over ranks.  Per-kernel durations for the roofline come from
 the library's own CUDA-event profiler over instrumented replays of the same step.  Beside the
-headline the line reports the other composition and the mixed-format backward (variants), and
+headline the line reports the other compositions and the mixed-format backward (variants), and
 the sweeps of single GEMMs and quantizes.
 
 ``--impl reference`` times the CPU oracle (the plain restatement of the method, on the host
@@ -63,8 +65,8 @@ def parse_args():
     p.add_argument("--no-sweeps", action="store_true")
     p.add_argument("--no-variants", action="store_true", help="skip the variant steps")
     p.add_argument("--path", default=STEP_PATH[0], choices=PATHS,
-                   help="headline step: x^T / w^T saved by the forward's quantize launch, or re-quantized "
-                        "by the backward's (identical numbers)")
+                   help="headline step: the backward's copies of x / w saved row-major or transposed by the "
+                        "forward's quantize launch, or re-quantized by the backward's (identical numbers)")
     p.add_argument("--dp-fold", action="store_true",
                    help="fold the rings once per step after an amax all-reduce (always on with several GPUs)")
     p.add_argument("--kernel", default=None, choices=["gemm", "quantize", "linear"],
@@ -266,6 +268,33 @@ class Linear:
                                       1, 1, 1, self.steps[0:1], self.steps[1:2], self.rg, 1.0, self.steps[2:3],
                                       self.sws, self.sws_n, self.gx, self.gw, self.gb)
 
+    def fwd_save_rm(self):
+        """Forward whose row-major quantize launch also writes x and w in E5M2 (the forward's
+        steps), row-major, for the backward."""
+        F = self.F
+        if not hasattr(self, "x8b"):
+            import torch
+            self.x8b = torch.empty((self.m, self.k), dtype=torch.uint8, device=self.x.device)
+            self.w8b = torch.empty((self.n, self.k), dtype=torch.uint8, device=self.x.device)
+            self.rws_n = F.linear_backward_fp8_mixed_workspace_size(self.m, self.k, self.n)
+            self.rws = torch.empty(self.rws_n, dtype=torch.uint8, device=self.x.device)
+        F.linear_forward_fp8_save_rm(self.x, self.w, self.b, None, self.m, self.k, self.n, F.FP8_E4M3, F.FP8_E5M2,
+                                     self.rx, self.rw, self.steps[0:1], self.steps[1:2], self.x8b, self.w8b, self.fws,
+                                     self.fws_n, self.y)
+
+    def bwd_saved_rm(self):
+        """Backward that quantizes only g (row-major) and reads the forward's E5M2 x / w in place."""
+        F = self.F
+        F.linear_backward_fp8_mixed(self.g, self.x8b, self.w8b, self.m, self.k, self.n, F.FP8_E5M2, F.FP8_E5M2,
+                                    F.FP8_E5M2, 1, 1, 1, self.steps[0:1], self.steps[1:2], self.rg, 1.0,
+                                    self.steps[2:3], self.rws, self.rws_n, self.gx, self.gw, self.gb)
+
+    @property
+    def quant_bytes_saved_rm(self):
+        m, k, n = self.m, self.k, self.n
+        # fwd: x, w row-major in two formats (2 B in, 1 + 1 B out); bwd: g row-major (2 + 1)
+        return 4 * (m * k + n * k) + 3 * m * n
+
     @property
     def quant_bytes_saved(self):
         m, k, n = self.m, self.k, self.n
@@ -297,13 +326,20 @@ def build_workload(F, W, torch, dev, seed_base):
     return lins
 
 
-PATHS = ("saved", "requant")
+PATHS = ("rowmajor", "saved", "requant")
 PATH_WHAT = {
+    "rowmajor": "x and w also written in E5M2 (the forward's steps), row-major, by the forward's quantize "
+                "launch; the backward quantizes only g (row-major) and its GEMMs read g8, x8 and w8 in place "
+                "(MN-major operands)",
     "saved": "x^T / w^T (E5M2, the forward's steps) written by the forward's quantize launch; the backward "
              "quantizes only g",
     "requant": "the backward's quantize launch re-quantizes x^T / w^T (E5M2, the forward's steps) beside g",
 }
-STEP_PATH = ["saved"]  # the headline step's composition (--path)
+STEP_PATH = ["rowmajor"]  # the headline step's composition (--path)
+
+
+def quant_bytes_of(lin, path):
+    return {"rowmajor": lin.quant_bytes_saved_rm, "saved": lin.quant_bytes_saved, "requant": lin.quant_bytes}[path]
 
 
 def run_step(lins, slot, mixed=False, path=None):
@@ -317,6 +353,8 @@ def run_step(lins, slot, mixed=False, path=None):
     for lin in lins:
         if mixed:
             lin.fwd_keep()
+        elif path == "rowmajor":
+            lin.fwd_save_rm()
         elif path == "saved":
             lin.fwd_save()
         else:
@@ -324,6 +362,8 @@ def run_step(lins, slot, mixed=False, path=None):
     for lin in reversed(lins):
         if mixed:
             lin.bwd_mixed()
+        elif path == "rowmajor":
+            lin.bwd_saved_rm()
         elif path == "saved":
             lin.bwd_saved()
         else:
@@ -633,7 +673,7 @@ def main():
     STEP_PATH[0] = args.path
     lins = build_workload(F, W, torch, dev, seed_base=100000 * rank)
     flops_step = sum(l.gemm_flops for l in lins)
-    qbytes_step = sum(l.quant_bytes_saved if args.path == "saved" else l.quant_bytes for l in lins)
+    qbytes_step = sum(quant_bytes_of(l, args.path) for l in lins)
 
     # Data parallel over several GPUs: the linears leave each ring's amax in its slot and, after
     # every step, the ranks reduce all rings' amax (one all-reduce MAX) and fold them, so every
@@ -738,11 +778,13 @@ def main():
 
     variants = {}
     if not args.no_variants:
-        other = "requant" if args.path == "saved" else "saved"
-        v = time_variant(False, other)
-        v["quantize_bytes_per_step"] = sum(l.quant_bytes if other == "requant" else l.quant_bytes_saved for l in lins)
-        v["what"] = PATH_WHAT[other] + " (the same numbers as the headline step)"
-        variants[f"path_{other}"] = v
+        for other in PATHS:
+            if other == args.path:
+                continue
+            v = time_variant(False, other)
+            v["quantize_bytes_per_step"] = sum(quant_bytes_of(l, other) for l in lins)
+            v["what"] = PATH_WHAT[other] + " (the same numbers as the headline step)"
+            variants[f"path_{other}"] = v
         v = time_variant(True, None)
         v["quantize_bytes_per_step"] = sum(l.quant_bytes_mixed for l in lins)
         v["what"] = ("forward keeps its E4M3 x8 / w8; backward quantizes only g (E5M2, row-major + column sums) "

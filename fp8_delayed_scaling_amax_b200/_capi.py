@@ -68,6 +68,9 @@ _SIGNATURES = {
     "linear_forward_fp8_save_t": (c_int, [_P, _P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int,
                                           POINTER(fp8_ring_t), POINTER(fp8_ring_t), _P, _P, _P, _P, _P, c_size_t,
                                           _P, _P]),
+    "linear_forward_fp8_save_rm": (c_int, [_P, _P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int,
+                                           POINTER(fp8_ring_t), POINTER(fp8_ring_t), _P, _P, _P, _P, _P, c_size_t,
+                                           _P, _P]),
     "linear_backward_fp8_saved_t_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "linear_backward_fp8_saved_t": (c_int, [_P, _P, _P, c_int64, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int,
                                             _P, _P, POINTER(fp8_ring_t), c_float, _P, _P, c_size_t, _P, _P, _P,
@@ -299,6 +302,16 @@ def linear_forward_fp8_save_t(x, w, bias, bias_scale, m, k, n, fmt, fmt_t, x_rin
     return _check("linear_forward_fp8_save_t", lib().linear_forward_fp8_save_t(
         _ptr(x), _ptr(w), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n), int(fmt), int(fmt_t), _ring(x_ring),
         _ring(w_ring), _ptr(sx_used), _ptr(sw_used), _ptr(x8t_out), _ptr(w8t_out), _ptr(workspace),
+        int(workspace_bytes), _ptr(y), _stream(stream)))
+
+
+def linear_forward_fp8_save_rm(x, w, bias, bias_scale, m, k, n, fmt, fmt_b, x_ring, w_ring, sx_used, sw_used,
+                               x8b_out, w8b_out, workspace, workspace_bytes, y, stream=None):
+    """Delayed-scaling forward that also writes x and w row-major in fmt_b (for
+    linear_backward_fp8_mixed with every format fmt_b)."""
+    return _check("linear_forward_fp8_save_rm", lib().linear_forward_fp8_save_rm(
+        _ptr(x), _ptr(w), _ptr(bias), _ptr(bias_scale), int(m), int(k), int(n), int(fmt), int(fmt_b), _ring(x_ring),
+        _ring(w_ring), _ptr(sx_used), _ptr(sw_used), _ptr(x8b_out), _ptr(w8b_out), _ptr(workspace),
         int(workspace_bytes), _ptr(y), _stream(stream)))
 
 

@@ -129,6 +129,7 @@ struct QuantJob {
     int fmt_t = -1;             // format of out_t (-1: fmt); the same product, a second rounding
     uint8_t* out = nullptr;     // [rows][cols] or nullptr
     uint8_t* out_t = nullptr;   // [cols][rows] or nullptr
+    uint8_t* out2 = nullptr;    // [rows][cols] in fmt_t (row-major launches only) or nullptr
     float* amax_out = nullptr;  // final amax (may be nullptr)
     const fp8_ring_t* ring = nullptr;
     float* scale_used_out = nullptr;  // the step used, written once (may be nullptr)
@@ -208,14 +209,15 @@ size_t linear_forward_base_workspace(int64_t m, int64_t k, int64_t n);
 
 // linear_forward_fp8 with choices: x8_keep / w8_keep (may be null) receive the quantized
 // operands instead of the workspace; x8t_keep / w8t_keep (both or neither; delayed scaling,
-// bf16 w) also receive x^T and w^T in format fmt_t from the same products; allow_split =
-// false needs only the base workspace and runs the GEMM without split-K.
+// bf16 w) also receive x^T and w^T in format fmt_t from the same products, or, with
+// copies_row_major, x and w in format fmt_t row-major; allow_split = false needs only the
+// base workspace and runs the GEMM without split-K.
 int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float* w_step, const void* bias,
                         const float* bias_scale, int64_t m, int64_t k, int64_t n, fp8_fmt_t fmt,
                         const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                         float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, uint8_t* x8t_keep, uint8_t* w8t_keep,
                         fp8_fmt_t fmt_t, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool copies_row_major = false);
 
 // The GEMM entry with arguments already validated (used by the linear compositions).
 int gemm_launch(const uint8_t* a, const uint8_t* b, int fmt_a, int fmt_b, int a_mn_major,

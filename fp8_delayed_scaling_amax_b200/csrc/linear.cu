@@ -202,6 +202,18 @@ int linear_forward_fp8_save_t(const void* x, const void* w, const void* bias, co
                                stream);
 }
 
+int linear_forward_fp8_save_rm(const void* x, const void* w, const void* bias, const float* bias_scale, int64_t m,
+                               int64_t k, int64_t n, fp8_fmt_t fmt, fp8_fmt_t fmt_b, const fp8_ring_t* x_ring,
+                               const fp8_ring_t* w_ring, float* sx_used, float* sw_used, uint8_t* x8b_out,
+                               uint8_t* w8b_out, void* workspace, size_t workspace_bytes, void* y,
+                               cudaStream_t stream) {
+    clear_error();
+    if (x8b_out == nullptr || w8b_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x8b_out and w8b_out are required");
+    return linear_forward_impl(x, w, 0, nullptr, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, 1.0f, sx_used,
+                               sw_used, nullptr, nullptr, x8b_out, w8b_out, fmt_b, workspace, workspace_bytes, true, y,
+                               stream, true);
+}
+
 size_t linear_backward_fp8_workspace_size(int64_t m, int64_t k, int64_t n) {
     if (m < 0 || k < 0 || n < 0) return 0;
     return bwd_layout(m, k, n).total;
@@ -221,7 +233,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
                         const fp8_ring_t* x_ring, const fp8_ring_t* w_ring, float pow2_margin, float* sx_used,
                         float* sw_used, uint8_t* x8_keep, uint8_t* w8_keep, uint8_t* x8t_keep, uint8_t* w8t_keep,
                         fp8_fmt_t fmt_t, void* workspace, size_t workspace_bytes, bool allow_split, void* y,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool copies_row_major) {
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
@@ -254,7 +266,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
             return fail(FP8DSA_ERR_INVALID_ARG, "transposed copies need x_ring, w_ring, a bf16 w and both outputs");
         if (!aligned16(x8t_keep) || !aligned16(w8t_keep))
             return fail(FP8DSA_ERR_UNSUPPORTED, "x8t_out / w8t_out must be 16-byte aligned");
-        if (m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for x8t_out");
+        if (!copies_row_major && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for x8t_out");
     }
     rc = check_device();
     if (rc) return rc;
@@ -299,8 +311,8 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     qx.cols = k;
     qx.fmt = fmt;
     qx.out = x8;
-    if (save_t) {  // the backward's x^T from the same products, in its own format
-        qx.out_t = x8t_keep;
+    if (save_t) {  // the backward's copy of x from the same products, in its own format
+        (copies_row_major ? qx.out2 : qx.out_t) = x8t_keep;
         qx.fmt_t = fmt_t;
     }
     if (dynamic) {
@@ -322,7 +334,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
         qw.fmt = fmt;
         qw.out = w8;
         if (save_t) {
-            qw.out_t = w8t_keep;
+            (copies_row_major ? qw.out2 : qw.out_t) = w8t_keep;
             qw.fmt_t = fmt_t;
         }
         if (dynamic) {

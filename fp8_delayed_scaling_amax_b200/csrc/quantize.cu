@@ -133,6 +133,7 @@ struct QArgs {
     const float* scale;        // step s; every element is multiplied by RN32(1/s)
     uint8_t* out;              // [rows][cols] or null
     uint8_t* out_t;            // [cols][rows] or null
+    uint8_t* out2;             // row-major kernel: [rows][cols] in the second format, or null
     float* amax_accum;         // block maxima land here (ring amax slot or amax_out), or null
     float* amax_out;           // ring mode: receives the final amax
     float* ring_state;         // null = no fold
@@ -275,7 +276,9 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
 // ----------------------------------------------------------------------------------------
 // Row-major quantize: flat, grid-stride, 16 elements per thread per iteration.
 // ----------------------------------------------------------------------------------------
-template <class In, int kFmt>
+// A tensor with out2 also gets its bytes in format kFmt2 (the same products, rounded once
+// more; kFmt2 == kFmt copies the same bytes), row-major like out.
+template <class In, int kFmt, int kFmt2>
 __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_constant__ QBatch batch) {
     pdl_trigger();
     pdl_wait();
@@ -290,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     const float step = __ldg(a.scale);
     const float mult = __frcp_rn(step);
     const auto* x = static_cast<const typename In::E*>(a.x);
+    uint8_t* const out2 = a.out2;
     float amax = 0.0f;
     typename In::Acc acc = In::acc_zero();  // running max of |x| over the vector chunks
     const int64_t gstride = static_cast<int64_t>(a.nblocks) * blockDim.x;
@@ -313,6 +317,11 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
         const uint2 lo = quant8<kFmt>(f0, mult);
         const uint2 hi = quant8<kFmt>(f1, mult);
         *reinterpret_cast<uint4*>(a.out + g * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        if (out2 != nullptr) {
+            const uint2 lo2 = second_format<kFmt, kFmt2>(f0, lo);
+            const uint2 hi2 = second_format<kFmt, kFmt2>(f1, hi);
+            *reinterpret_cast<uint4*>(out2 + g * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
+        }
         if (has1) {
             In::acc_max(acc, r2);
             In::acc_max(acc, r3);
@@ -321,6 +330,11 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
             const uint2 lo1 = quant8<kFmt>(f0, mult);
             const uint2 hi1 = quant8<kFmt>(f1, mult);
             *reinterpret_cast<uint4*>(a.out + g1 * 16) = make_uint4(lo1.x, lo1.y, hi1.x, hi1.y);
+            if (out2 != nullptr) {
+                const uint2 lo2 = second_format<kFmt, kFmt2>(f0, lo1);
+                const uint2 hi2 = second_format<kFmt, kFmt2>(f1, hi1);
+                *reinterpret_cast<uint4*>(out2 + g1 * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
+            }
         }
     }
     amax = In::acc_value(acc);
@@ -328,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
         const float v = In::cvt(x[i]);
         amax = fmaxf(amax, fabsf(v));
         a.out[i] = convert1<kFmt>(v, mult);
+        if (out2 != nullptr) out2[i] = convert1<kFmt2>(v, mult);
     }
     ring_stash(a, hist_v, s_hist);
     block_finish(a, amax, step, lb == 0, s_hist);
@@ -851,9 +866,9 @@ constexpr int kFlatWaves = 1;
 // Resident 256-thread blocks per SM of the row-major kernel (its launch bounds ask for 4).
 int flat_blocks_per_sm() { return 4; }
 
-template <int kFmt, class In>
+template <int kFmt, int kFmt2, class In>
 void launch_flat(const QBatch& b, dim3 grid, cudaStream_t stream) {
-    launch_ex(quant_flat_kernel<In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+    launch_ex(quant_flat_kernel<In, kFmt, kFmt2>, grid, dim3(kThreads), 0, stream, 1, b);
 }
 
 // Batches of more tiles than this run persistent; smaller ones one tile per CTA.
@@ -912,12 +927,9 @@ int launch_quant(QBatch& b, bool tiled, dim3 grid, const WaitCtl& ctl, cudaStrea
         if (b.tiles_total > thr) return launch_tiled<kFmt, kFmtT, In, true>(b, ctl, stream);
         return launch_tiled<kFmt, kFmtT, In, false>(b, ctl, stream);
     }
-    if constexpr (kFmtT == kFmt) {
-        launch_flat<kFmt, In>(b, grid, stream);
-        return FP8DSA_OK;
-    } else {
-        return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output");
-    }
+    // the row-major kernel writes a second format only as a second row-major copy (out2)
+    launch_flat<kFmt, kFmtT, In>(b, grid, stream);
+    return FP8DSA_OK;
 }
 
 template <int kFmt, int kFmtT>
@@ -958,7 +970,11 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         if (jobs[i].fmt != fmt || (jobs[i].fmt_t < 0 ? fmt : static_cast<fp8_fmt_t>(jobs[i].fmt_t)) != fmt_t ||
             jobs[i].in_type != in_type || wants_tiles(jobs[i]) != tiled)
             return fail(FP8DSA_ERR_INVALID_ARG, "a quantize batch shares formats, input type and orientation");
-    if (fmt_t != fmt && !tiled) return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output");
+    bool any_out2 = false;
+    for (int i = 0; i < njobs; ++i) any_out2 = any_out2 || jobs[i].out2 != nullptr;
+    if (any_out2 && tiled) return fail(FP8DSA_ERR_INVALID_ARG, "a second row-major copy is a row-major launch");
+    if (fmt_t != fmt && !tiled && !any_out2)
+        return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output or a second row-major copy");
     QBatch b{};
     b.njobs = njobs;
     b.zero = zero;
@@ -976,6 +992,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         a.scale = job.scale;
         a.out = job.out;
         a.out_t = job.out_t;
+        a.out2 = job.out2;
         a.scale_used_out = job.scale_used_out;
         a.colsum = job.colsum_partial;
         a.defer_fold = job.ring != nullptr && job.defer_fold ? 1 : 0;
@@ -999,6 +1016,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         a.vec_in = aligned16(job.x) && (tiled ? rows_vec : true);
         a.vec_out = (job.out == nullptr) ||
                     (tiled ? ((reinterpret_cast<uintptr_t>(job.out) & 7) == 0 && job.cols % 8 == 0) : aligned16(job.out));
+        if (job.out2 != nullptr && !aligned16(job.out2)) a.vec_out = 0;
         a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
         if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
         if (tiled && a.vec_in && job.rows > 0 && job.cols > 0 && job.rows < (int64_t(1) << 31) &&
@@ -1011,7 +1029,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
             else
                 clear_error();  // fall back to direct loads for this tensor
         }
-        bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0));
+        bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0) + (job.out2 ? 1 : 0));
         if (tiled) {
             // an empty tensor still gets one (empty) tile
             const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);

@@ -346,6 +346,25 @@ int linear_forward_fp8_save_t(const void* x, const void* w, const void* bias,
                               uint8_t* x8t_out, uint8_t* w8t_out, void* workspace,
                               size_t workspace_bytes, void* y, cudaStream_t stream);
 
+/* Delayed-scaling forward that also saves the backward's copies of x and w row-major (the
+ * pages' backward quantizes x and w with the forward's steps in the backward's format
+ * [AstrAI compare view, astrai/extension/fp8.py, _LinearFp8.backward]; this entry forms those
+ * bytes in the forward's row-major quantize launch, from the same products, and keeps them
+ * in the orientation they are read in, so no transpose is written):
+ *   everything as linear_forward_fp8 with w bf16 (no w_is_fp8) and both rings given, plus
+ *   x8b_out: dev [m][k] bytes of x in fmt_b at step *sx_used; w8b_out: dev [n][k] bytes of w
+ *   in fmt_b at step *sw_used; both 16-byte aligned.
+ *   linear_backward_fp8_mixed(g, x8b_out, w8b_out, ..., fmt_g = fmt_x = fmt_w = fmt_b,
+ *   sx_used, sw_used, ...) then reads them in place (MN-major operands) and computes the
+ *   pages' backward (g, x and w all in fmt_b at the forward's steps) with one quantize launch
+ *   for g.  One quantize launch (x and w, two formats each) and one GEMM launch. */
+int linear_forward_fp8_save_rm(const void* x, const void* w, const void* bias,
+                               const float* bias_scale, int64_t m, int64_t k, int64_t n,
+                               fp8_fmt_t fmt, fp8_fmt_t fmt_b, const fp8_ring_t* x_ring,
+                               const fp8_ring_t* w_ring, float* sx_used, float* sw_used,
+                               uint8_t* x8b_out, uint8_t* w8b_out, void* workspace,
+                               size_t workspace_bytes, void* y, cudaStream_t stream);
+
 /* Workspace bytes linear_backward_fp8_saved_t needs for (m, k, n): g8, g8t, the per-tile
  * column sums, scale scratch and the GEMM's split-K region. */
 size_t linear_backward_fp8_saved_t_workspace_size(int64_t m, int64_t k, int64_t n);

@@ -146,6 +146,21 @@ def test_keep_forward_and_mixed_backward_argument_checks():
     assert call(margin=0.0) == INVALID       # dynamic scaling needs a positive margin
 
 
+def test_save_rm_forward_argument_checks():
+    f = F.lib().linear_forward_fp8_save_rm
+    ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
+    ring = F.fp8_ring_t(256, 16, 0, 448.0, 1.0)
+    r = ctypes.byref(ring)
+    # both copies are required
+    assert f(256, 256, None, None, 64, 64, 64, 0, 1, r, r, None, None, None, 4096, 1024, ws, 2048, None) == INVALID
+    # delayed scaling only (both rings)
+    assert f(256, 256, None, None, 64, 64, 64, 0, 1, None, None, None, None, 4096, 8192, 1024, ws, 2048, None) == INVALID
+    # the copies must be 16-byte aligned
+    assert f(256, 256, None, None, 64, 64, 64, 0, 1, r, r, None, None, 4100, 8192, 1024, ws, 2048, None) == UNSUPPORTED
+    # bad second format
+    assert f(256, 256, None, None, 64, 64, 64, 0, 5, r, r, None, None, 4096, 8192, 1024, ws, 2048, None) == INVALID
+
+
 def test_prequant_backward_argument_checks():
     pb = F.lib().linear_backward_fp8_prequant
     wsb = F.linear_backward_fp8_workspace_size(64, 64, 64)
