@@ -55,28 +55,36 @@ constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
 
 constexpr int kOutBox = 64;                       // output columns per TMA store (128 bytes of bf16)
 constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 columns
+#ifndef FP8DSA_GEMM_OUT_BUFS
+#define FP8DSA_GEMM_OUT_BUFS 2
+#endif
+constexpr int kOutBufs = FP8DSA_GEMM_OUT_BUFS;    // staged boxes per epilogue warp (TMA stores in flight)
+constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 232448;                // dynamic shared memory per CTA on sm_100
 constexpr int kMaxProblems = 2;
 
 // kPair: a 2-CTA cluster computes a 256 x BN tile with one M = 256 MMA across both SMs; each CTA
 // holds 128 rows of A and BN/2 rows of B, so each SM's shared memory feeds half the B operand.
-// Epilogue warps: 8 (two per TMEM lane quarter, each owning half the columns) when the stages
-// leave room for their staging buffers, else 4.
+// Epilogue warps: 8 (two per TMEM lane quarter, each owning half the columns) for tiles at
+// least 128 wide when the stages leave room for their staging buffers, else 4.  BN = 64
+// (single CTA, K-major B) serves short, wide problems: more tiles, so more SMs stream B.
 template <int BN, bool kPair>
 struct Cfg {
     static constexpr int kTileM = kPair ? 2 * kBM : kBM;
     static constexpr int kBRows = kPair ? BN / 2 : BN;  // rows of B (along N) this CTA loads
     static constexpr int kAStage = kBM * kBK;
     static constexpr int kBStage = kBRows * kBK;
-    static constexpr int kEpiWarps = (kAStage + kBStage) <= 32768 ? 8 : 4;
+    static constexpr int kEpiWarps = (BN >= 128 && (kAStage + kBStage) <= 32768) ? 8 : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kEpiThreads = 32 * kEpiWarps;
     static constexpr int kEpiCols = BN / (kEpiWarps / 4);  // columns of the tile each epilogue warp owns
-    static constexpr int kOutBytes = kEpiWarps * 2 * kOutStageBytes;
+    static constexpr int kOutBytes = kEpiWarps * kOutBufs * kOutStageBytes;
     static constexpr int kBarBytes = 256;
     static constexpr int kFixed = 1024 + kOutBytes + kBarBytes;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / (kAStage + kBStage);
-    static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
+    static constexpr int kStages = kStagesFit < kMaxStages ? kStagesFit : kMaxStages;
+    static_assert(kEpiCols % kOutBox == 0, "each epilogue warp owns whole 64-column boxes");
+    static_assert(!kPair || BN >= 128, "pair tiles are at least 128 wide");
     static constexpr int kSmem = kFixed + kStages * (kAStage + kBStage);
     static constexpr uint32_t kTxBytes = (kPair ? 2u : 1u) * (kAStage + kBStage);
     static_assert(kStages >= 3, "too few pipeline stages");
@@ -488,7 +496,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
         const int ew = warp - 2;
         const int q = warp & 3;
         const int cbase = (ew >> 2) * C::kEpiCols;
-        uint8_t* my_stage = sOut + ew * 2 * kOutStageBytes;
+        uint8_t* my_stage = sOut + ew * kOutBufs * kOutStageBytes;
 
         // side job: the deferred ring folds of the quantize launch before (one thread)
         if (g.nfolds > 0 && blockIdx.x == 0 && ew == 0 && lane == 0) {
@@ -663,7 +671,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                 const int colg = col0 + c;
                 if (P.tma_out) {
                     uint8_t* sb = my_stage + buf * kOutStageBytes;
-                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used this buffer has read it
+                    if (lane == 0) bulk_wait_group_read<kOutBufs - 1>();  // the store that last used this buffer has read it
                     __syncwarp();
                     // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r % 8)
 #pragma unroll
@@ -676,7 +684,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                         tma_store_3d(to, sb, colg, row0, b);
                         bulk_commit_group();
                     }
-                    buf ^= 1;
+                    buf = buf + 1 == kOutBufs ? 0 : buf + 1;
                 } else if (P.out != nullptr && row < P.m && colg < P.n) {
                     uint16_t* orow = P.out + static_cast<int64_t>(b) * P.stride_o + row * P.ldo;
                     if (P.vec_out && colg + kOutBox <= P.n) {
@@ -1097,7 +1105,7 @@ struct TileChoice {
     bool pair;
 };
 
-// Tuning override: FP8DSA_GEMM_TILE = "256p", "128p", "256" or "128" forces that tile shape
+// Tuning override: FP8DSA_GEMM_TILE = "256p", "128p", "256", "128" or "64" forces that tile shape
 // wherever the problem admits it (read once; unset = the default choice below).
 int tile_override() {
     static const int v = [] {
@@ -1108,9 +1116,37 @@ int tile_override() {
         if (t == "128p") return 2;
         if (t == "256") return 3;
         if (t == "128") return 4;
+        if (t == "64") return 5;
         return 0;
     }();
     return v;
+}
+
+// Single-CTA tile width for launches the pair tiles do not suit (some M at most 128, or some
+// N at most 128): the BN in {64, 128, 256} with the fewest rounds of tiles times the bytes a
+// CTA loads per k-block (A's 128 rows plus BN rows of B), the wider one on ties -- so a short,
+// wide problem (M = 64, N = 8192) spreads B over most SMs in 64-column tiles instead of
+// leaving them idle.  64-wide tiles need a K-major B; 256-wide ones an N above 128.
+int single_cta_width(const GemmDesc* d, int n, bool b_mn) {
+    int best = 128;
+    int64_t best_cost = -1;
+    for (int bn : {256, 128, 64}) {
+        if (bn == 64 && b_mn) continue;
+        bool fits = true;
+        int64_t tiles = 0;
+        for (int i = 0; i < n; ++i) {
+            if (bn == 256 && d[i].n <= 128) fits = false;
+            tiles += ((d[i].m + kBM - 1) / kBM) * ((d[i].n + bn - 1) / bn) * d[i].batch;
+        }
+        if (!fits) continue;
+        const int64_t rounds = (tiles + sm_count() - 1) / sm_count();
+        const int64_t cost = rounds * static_cast<int64_t>(kBM * kBK + bn * kBK);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
 }
 
 TileChoice choose_tiles(const GemmDesc* d, int n) {
@@ -1120,13 +1156,13 @@ TileChoice choose_tiles(const GemmDesc* d, int n) {
         short_m = short_m || d[i].m <= kBM;
         b_mn = b_mn || d[i].b_mn;
     }
-    if (narrow) return {128, false};
-    if (short_m) return {256, false};
+    if (narrow || short_m) return {single_cta_width(d, n, b_mn), false};
     switch (tile_override()) {
         case 1: return {256, true};
         case 2: if (!b_mn) return {128, true}; break;
         case 3: return {256, false};
         case 4: return {128, false};
+        case 5: if (!b_mn) return {64, false}; break;
         default: break;
     }
     // Few output tiles: when the 256 x 256 pair tiles would keep at most half of the CTA pairs
@@ -1298,9 +1334,12 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
     if (tc.pair)
         rc = tc.bn == 256 ? launch_cfg<256, true>(maps, g, batch, split, stream)
                           : launch_cfg<128, true>(maps, g, batch, split, stream);
+    else if (tc.bn == 256)
+        rc = launch_cfg<256, false>(maps, g, batch, split, stream);
+    else if (tc.bn == 128)
+        rc = launch_cfg<128, false>(maps, g, batch, split, stream);
     else
-        rc = tc.bn == 256 ? launch_cfg<256, false>(maps, g, batch, split, stream)
-                          : launch_cfg<128, false>(maps, g, batch, split, stream);
+        rc = launch_cfg<64, false>(maps, g, batch, split, stream);
     if (rc) return rc;
     launch_end(tc.pair ? kKindGemmPair : kKindGemmSingle, stream, flops);
     return check_launch("fp8 gemm kernel");
