@@ -30,6 +30,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 
@@ -169,6 +170,12 @@ __device__ __forceinline__ void zero_side_job(const QBatch& b) {
         for (int64_t i = threadIdx.x; i < b.zero_words; i += blockDim.x) b.zero[i] = 0u;
 }
 
+// Chunks of 16 elements each thread of the row-major kernel has in flight (16-bit inputs).
+#ifndef FP8DSA_FLAT_DEPTH
+#define FP8DSA_FLAT_DEPTH 2
+#endif
+constexpr int kFlatDepth = FP8DSA_FLAT_DEPTH;
+
 // Eight floats -> eight fp8 bytes (two words): each byte is the RN, saturating encoding of
 // RN32(f * mult), the products taken two per packed instruction; amax is kept by the caller.
 template <int kFmt>
@@ -299,41 +306,35 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     const int64_t gstride = static_cast<int64_t>(a.nblocks) * blockDim.x;
     const int64_t tid = lb * blockDim.x + threadIdx.x;
     const int64_t n16 = a.vec_in ? a.numel / 16 : 0;
-    for (int64_t g = tid; g < n16; g += 2 * gstride) {
-        const int64_t g1 = g + gstride;
-        const bool has1 = g1 < n16;
-        typename In::Raw r0 = In::load_raw(x + g * 16);
-        typename In::Raw r1 = In::load_raw(x + g * 16 + 8);
-        typename In::Raw r2, r3;
-        if (has1) {
-            r2 = In::load_raw(x + g1 * 16);
-            r3 = In::load_raw(x + g1 * 16 + 8);
+    // kDepth chunks of 16 elements per thread in flight: every load of a round is issued before
+    // the round's first conversion
+    constexpr int kDepth = sizeof(typename In::E) == 4 ? 2 : kFlatDepth;
+    for (int64_t g = tid; g < n16; g += kDepth * gstride) {
+        typename In::Raw r[kDepth][2];
+#pragma unroll
+        for (int d = 0; d < kDepth; ++d) {
+            const int64_t gd = g + d * gstride;
+            if (gd < n16) {
+                r[d][0] = In::load_raw(x + gd * 16);
+                r[d][1] = In::load_raw(x + gd * 16 + 8);
+            }
         }
-        float f0[8], f1[8];
-        In::acc_max(acc, r0);
-        In::acc_max(acc, r1);
-        In::unpack(r0, f0);
-        In::unpack(r1, f1);
-        const uint2 lo = quant8<kFmt>(f0, mult);
-        const uint2 hi = quant8<kFmt>(f1, mult);
-        *reinterpret_cast<uint4*>(a.out + g * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        if (out2 != nullptr) {
-            const uint2 lo2 = second_format<kFmt, kFmt2>(f0, lo);
-            const uint2 hi2 = second_format<kFmt, kFmt2>(f1, hi);
-            *reinterpret_cast<uint4*>(out2 + g * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
-        }
-        if (has1) {
-            In::acc_max(acc, r2);
-            In::acc_max(acc, r3);
-            In::unpack(r2, f0);
-            In::unpack(r3, f1);
-            const uint2 lo1 = quant8<kFmt>(f0, mult);
-            const uint2 hi1 = quant8<kFmt>(f1, mult);
-            *reinterpret_cast<uint4*>(a.out + g1 * 16) = make_uint4(lo1.x, lo1.y, hi1.x, hi1.y);
+#pragma unroll
+        for (int d = 0; d < kDepth; ++d) {
+            const int64_t gd = g + d * gstride;
+            if (gd >= n16) break;
+            float f0[8], f1[8];
+            In::acc_max(acc, r[d][0]);
+            In::acc_max(acc, r[d][1]);
+            In::unpack(r[d][0], f0);
+            In::unpack(r[d][1], f1);
+            const uint2 lo = quant8<kFmt>(f0, mult);
+            const uint2 hi = quant8<kFmt>(f1, mult);
+            *reinterpret_cast<uint4*>(a.out + gd * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
             if (out2 != nullptr) {
-                const uint2 lo2 = second_format<kFmt, kFmt2>(f0, lo1);
-                const uint2 hi2 = second_format<kFmt, kFmt2>(f1, hi1);
-                *reinterpret_cast<uint4*>(out2 + g1 * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
+                const uint2 lo2 = second_format<kFmt, kFmt2>(f0, lo);
+                const uint2 hi2 = second_format<kFmt, kFmt2>(f1, hi);
+                *reinterpret_cast<uint4*>(out2 + gd * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
             }
         }
     }
@@ -346,6 +347,113 @@ __global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_co
     }
     ring_stash(a, hist_v, s_hist);
     block_finish(a, amax, step, lb == 0, s_hist);
+}
+
+// ----------------------------------------------------------------------------------------
+// Row-major bytes plus per-tile column sums (a gradient quantized for the bias gradient), for
+// batches that write no transposed bytes.  Each block covers 128 rows x 64 columns of one
+// tensor, so small tensors still spread over many blocks: thread t owns the 8 columns
+// 8 * (t % 8) .. + 7 and the rows t / 8 + 32 i (i = 0..3), issues its four 16-byte loads at
+// once, and keeps the 8 column sums of its rows in registers.  The 32 row threads of a column
+// group reduce through two shuffles and an 8-warp shared-memory sum, in a fixed order, into
+// colsum[tile row][column] (the layout the dual quantize writes).
+// ----------------------------------------------------------------------------------------
+constexpr int kRcCols = 64;
+
+template <class In, int kFmt>
+__global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __grid_constant__ QBatch batch) {
+    pdl_trigger();
+    pdl_wait();
+    zero_side_job(batch);
+    int jb = 0;
+    while (jb + 1 < batch.njobs && static_cast<int>(blockIdx.x) >= batch.job[jb + 1].tile_begin) ++jb;
+    const QArgs& a = batch.job[jb];
+    const int local = static_cast<int>(blockIdx.x) - a.tile_begin;
+    const int ty = local / a.tiles_x, tx = local - (local / a.tiles_x) * a.tiles_x;
+    __shared__ float s_hist[kHistPrefetch];
+    __shared__ float s_cs[kThreads / 32][kRcCols];
+    const float hist_v = ring_peek(a);
+    const float step = __ldg(a.scale);
+    const float mult = __frcp_rn(step);
+    const auto* x = static_cast<const typename In::E*>(a.x);
+    const int64_t rows = a.rows, cols = a.cols;
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    const int cg = t & 7, rt = t >> 3;
+    const int64_t r0 = static_cast<int64_t>(ty) * kTile;
+    const int64_t gc = static_cast<int64_t>(tx) * kRcCols + 8 * cg;
+    const bool colsum = a.colsum != nullptr;
+    float cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0f;
+    float amax = 0.0f;
+    typename In::Acc acc = In::acc_zero();
+    if (a.vec_in && a.vec_out && r0 + kTile <= rows && gc + 8 <= cols) {
+        typename In::Raw raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) raw[i] = In::load_raw(x + (r0 + rt + 32 * i) * cols + gc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float f[8];
+            In::acc_max(acc, raw[i]);
+            In::unpack(raw[i], f);
+            if (colsum) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
+            }
+            *reinterpret_cast<uint2*>(a.out + (r0 + rt + 32 * i) * cols + gc) = quant8<kFmt>(f, mult);
+        }
+    } else {
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+            const int64_t gr = r0 + rt + 32 * i;
+            float f[8];
+            if (gr < rows && a.vec_in && gc + 8 <= cols) {
+                In::load8(x + gr * cols + gc, f);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = (gr < rows && gc + e < cols) ? In::cvt(x[gr * cols + gc + e]) : 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+            if (colsum) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
+            }
+            const uint2 q = quant8<kFmt>(f, mult);
+            if (gr < rows && gc < cols) {
+                uint8_t* dst = a.out + gr * cols + gc;
+                if (a.vec_out && gc + 8 <= cols) {
+                    *reinterpret_cast<uint2*>(dst) = q;
+                } else {
+                    const uint32_t qq[2] = {q.x, q.y};
+                    for (int e = 0; e < 8 && gc + e < cols; ++e) dst[e] = static_cast<uint8_t>(qq[e >> 2] >> (8 * (e & 3)));
+                }
+            }
+        }
+    }
+    amax = fmaxf(amax, In::acc_value(acc));
+    if (colsum) {
+        // lanes l, l ^ 8, l ^ 16, l ^ 24 share the column group; then the 8 warps in order
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 8);
+            cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
+        }
+        if (lane < 8) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s_cs[w][8 * lane + e] = cs[e];
+        }
+        __syncthreads();
+        const int64_t c = static_cast<int64_t>(tx) * kRcCols + t;
+        if (t < kRcCols && c < cols) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int v = 0; v < kThreads / 32; ++v) sum += s_cs[v][t];
+            a.colsum[static_cast<int64_t>(ty) * cols + c] = sum;
+        }
+    }
+    ring_stash(a, hist_v, s_hist);
+    block_finish(a, amax, step, local == 0, s_hist);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -939,6 +1047,28 @@ int launch_quant_in(fp8_in_t in_type, QBatch& b, bool tiled, dim3 grid, const Wa
     return launch_quant<kFmt, kFmtT, F32In>(b, tiled, grid, ctl, stream);
 }
 
+template <int kFmt>
+int launch_rows_colsum(fp8_in_t in_type, const QBatch& b, cudaStream_t stream) {
+    const dim3 grid(static_cast<unsigned>(b.tiles_total));
+    if (in_type == FP8_IN_BF16)
+        launch_ex(quant_rows_colsum_kernel<Bf16In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+    else if (in_type == FP8_IN_F16)
+        launch_ex(quant_rows_colsum_kernel<F16In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+    else
+        launch_ex(quant_rows_colsum_kernel<F32In, kFmt>, grid, dim3(kThreads), 0, stream, 1, b);
+    return FP8DSA_OK;
+}
+
+// Tuning override: FP8DSA_ROWS_COLSUM=0 sends row-major + column-sum batches to the 128 x 128
+// tiled kernel instead of the 128 x 64 block kernel (read once).
+bool row_colsum_enabled() {
+    static const bool v = [] {
+        const char* e = std::getenv("FP8DSA_ROWS_COLSUM");
+        return e == nullptr || std::string(e) != "0";
+    }();
+    return v;
+}
+
 CUtensorMapDataType map_type(fp8_in_t t) {
     return t == FP8_IN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                            : (t == FP8_IN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
@@ -975,6 +1105,10 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     if (any_out2 && tiled) return fail(FP8DSA_ERR_INVALID_ARG, "a second row-major copy is a row-major launch");
     if (fmt_t != fmt && !tiled && !any_out2)
         return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output or a second row-major copy");
+    // row-major bytes + column sums and no transposed bytes: the 128 x 64 block kernel
+    bool rows_colsum = tiled && fmt_t == fmt && row_colsum_enabled();
+    for (int i = 0; i < njobs; ++i)
+        rows_colsum = rows_colsum && jobs[i].out_t == nullptr && jobs[i].out != nullptr && jobs[i].colsum_partial != nullptr;
     QBatch b{};
     b.njobs = njobs;
     b.zero = zero;
@@ -1019,7 +1153,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         if (job.out2 != nullptr && !aligned16(job.out2)) a.vec_out = 0;
         a.vec_out_t = job.out_t != nullptr && aligned16(job.out_t) && job.rows % 16 == 0;
         if (!tiled && !(a.vec_in && a.vec_out)) a.vec_in = 0;  // flat kernel: both or neither
-        if (tiled && a.vec_in && job.rows > 0 && job.cols > 0 && job.rows < (int64_t(1) << 31) &&
+        if (tiled && !rows_colsum && a.vec_in && job.rows > 0 && job.cols > 0 && job.rows < (int64_t(1) << 31) &&
             job.cols < (int64_t(1) << 31)) {
             // TMA needs a 16-byte aligned base and row stride (both implied by vec_in here)
             const int64_t ld = job.cols * eb;
@@ -1030,7 +1164,18 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
                 clear_error();  // fall back to direct loads for this tensor
         }
         bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0) + (job.out2 ? 1 : 0));
-        if (tiled) {
+        if (tiled && rows_colsum) {
+            // 128 x 64 blocks of the row-major + column-sum kernel (an empty tensor: one block)
+            const int64_t tx = std::max<int64_t>(1, (job.cols + kRcCols - 1) / kRcCols);
+            const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
+            a.tiles_x = static_cast<int>(tx);
+            a.tiles_y = static_cast<int>(ty);
+            a.tile_group = 1;
+            a.tile_begin = static_cast<int>(tiles_total);
+            a.nblocks = static_cast<unsigned>(tx * ty);
+            tiles_total += tx * ty;
+            if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 64 blocks");
+        } else if (tiled) {
             // an empty tensor still gets one (empty) tile
             const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);
             const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
@@ -1073,6 +1218,16 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     }
     launch_begin(kKindQuantize, stream);
     int rc;
+    if (rows_colsum) {
+        b.tiles_total = static_cast<int>(tiles_total);
+        if (fmt == FP8_E4M3)
+            rc = launch_rows_colsum<0>(in_type, b, stream);
+        else
+            rc = launch_rows_colsum<1>(in_type, b, stream);
+        launch_end(kKindQuantize, stream, bytes);
+        if (rc) return rc;
+        return check_launch("fp8 quantize kernel");
+    }
     if (fmt == FP8_E4M3)
         rc = fmt_t == FP8_E4M3 ? launch_quant_in<0, 0>(in_type, b, tiled, grid, ctl, stream)
                                : launch_quant_in<0, 1>(in_type, b, tiled, grid, ctl, stream);
