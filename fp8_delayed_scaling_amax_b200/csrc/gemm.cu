@@ -56,7 +56,7 @@ constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
 constexpr int kOutBox = 64;                       // output columns per TMA store (128 bytes of bf16)
 constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 columns
 #ifndef FP8DSA_GEMM_OUT_BUFS
-#define FP8DSA_GEMM_OUT_BUFS 2
+#define FP8DSA_GEMM_OUT_BUFS 1
 #endif
 constexpr int kOutBufs = FP8DSA_GEMM_OUT_BUFS;    // staged boxes per epilogue warp (TMA stores in flight)
 constexpr int kMaxStages = 8;
@@ -74,7 +74,13 @@ struct Cfg {
     static constexpr int kBRows = kPair ? BN / 2 : BN;  // rows of B (along N) this CTA loads
     static constexpr int kAStage = kBM * kBK;
     static constexpr int kBStage = kBRows * kBK;
-    static constexpr int kEpiWarps = (BN >= 128 && (kAStage + kBStage) <= 32768) ? 8 : 4;
+    // N of one MMA instruction (at most 256); a 512-wide pair tile issues two per K step, into
+    // TMEM columns 0..255 and 256..511, and has a single accumulator (the tile fills TMEM)
+    static constexpr int kMmaN = BN > 256 ? 256 : BN;
+    static constexpr int kNMma = BN / kMmaN;
+    static constexpr int kAccBufs = 2 * BN <= 512 ? 2 : 1;
+    static constexpr int kTmemCols = kAccBufs * BN;
+    static constexpr int kEpiWarps = (BN >= 128 && ((kAStage + kBStage) <= 32768 || BN == 512)) ? 8 : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kEpiThreads = 32 * kEpiWarps;
     static constexpr int kEpiCols = BN / (kEpiWarps / 4);  // columns of the tile each epilogue warp owns
@@ -85,6 +91,8 @@ struct Cfg {
     static constexpr int kStages = kStagesFit < kMaxStages ? kStagesFit : kMaxStages;
     static_assert(kEpiCols % kOutBox == 0, "each epilogue warp owns whole 64-column boxes");
     static_assert(!kPair || BN >= 128, "pair tiles are at least 128 wide");
+    static_assert(kPair || BN <= 256, "single-CTA tiles are at most 256 wide");
+    static_assert(kTmemCols <= 512, "accumulators exceed TMEM");
     static constexpr int kSmem = kFixed + kStages * (kAStage + kBStage);
     static constexpr uint32_t kTxBytes = (kPair ? 2u : 1u) * (kAStage + kBStage);
     static_assert(kStages >= 3, "too few pipeline stages");
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < C::kAccBufs; ++a) {
             mbar_init(acc_full + a, 1);
             // the leader's accumulator is released by both CTAs' epilogue threads
             mbar_init(acc_empty + a, C::kEpiThreads * (kPair ? 2 : 1));
@@ -321,10 +329,10 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
     }
     if (warp == 1) {
         if constexpr (kPair) {
-            tmem_alloc_pair(tmem_slot, 2 * BN);
+            tmem_alloc_pair(tmem_slot, C::kTmemCols);
             tmem_relinquish_pair();
         } else {
-            tmem_alloc(tmem_slot, 2 * BN);
+            tmem_alloc(tmem_slot, C::kTmemCols);
             tmem_relinquish();
         }
     }
@@ -373,7 +381,15 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                         else
                             tma_load_3d_pair(a_dst, ta, fb, arow, kb * kBK, ba);
                         if (!P.b_mn) {
-                            tma_load_3d_pair(b_dst, tb, fb, kb * kBK, brow, bb);
+                            if constexpr (C::kNMma == 1) {
+                                tma_load_3d_pair(b_dst, tb, fb, kb * kBK, brow, bb);
+                            } else {
+                                // this CTA's half of each MMA's 256 columns: rows j * 256 + rank * 128
+#pragma unroll
+                                for (int j = 0; j < C::kNMma; ++j)
+                                    tma_load_3d_pair(b_dst + j * (C::kMmaN / 2) * kBK, tb, fb, kb * kBK,
+                                                     tn * BN + j * C::kMmaN + static_cast<int>(rank) * (C::kMmaN / 2), bb);
+                            }
                         } else {
 #pragma unroll
                             for (int h = 0; h < C::kBRows / 128; ++h)
@@ -447,10 +463,16 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                             const uint64_t bd = P.b_mn ? smem_desc(b_base + kk * kUmmaK * 128, kLboB, 1024)
                                                        : smem_desc(b_base + kk * kUmmaK, 16, 1024);
                             const uint32_t accumulate = (kb != w.kb0 || kk != 0) ? 1u : 0u;
-                            if constexpr (kPair)
-                                umma_f8f6f4_pair(d_tmem, ad, bd, idesc, accumulate);
-                            else
-                                umma_f8f6f4(d_tmem, ad, bd, idesc, accumulate);
+#pragma unroll
+                            for (int j = 0; j < C::kNMma; ++j) {
+                                // the j-th 256 columns: B rows j * (kMmaN / 2) of this CTA's stage
+                                const uint64_t bdj = bd + ((static_cast<uint64_t>(j * (C::kMmaN / 2) * kBK) >> 4) & 0x3FFFu);
+                                const uint32_t dj = d_tmem + static_cast<uint32_t>(j * C::kMmaN);
+                                if constexpr (kPair)
+                                    umma_f8f6f4_pair(dj, ad, bdj, idesc, accumulate);
+                                else
+                                    umma_f8f6f4(dj, ad, bdj, idesc, accumulate);
+                            }
                         }
                         if constexpr (kPair)
                             umma_commit_pair_multicast(empty + stage, 0x3);
@@ -471,7 +493,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                         umma_commit(acc_full + acc);
                 }
                 __syncwarp();
-                if (++acc == 2) {
+                if (++acc == C::kAccBufs) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
@@ -765,7 +787,7 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
                     counter_add_release(g.counters + 2 * w.tile + rank, 1u);
                 }
             }
-            if (++acc == 2) {
+            if (++acc == C::kAccBufs) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
@@ -780,9 +802,9 @@ __global__ void __launch_bounds__(Cfg<BN, kPair>::kThreads, 1)
     tc_fence_after_sync();
     if (warp == 1) {
         if constexpr (kPair)
-            tmem_dealloc_pair(tmem_base, 2 * BN);
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
         else
-            tmem_dealloc(tmem_base, 2 * BN);
+            tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
@@ -1022,7 +1044,7 @@ int launch_cfg(const CUtensorMap (&maps)[8], GemmArgs& g, const int64_t* batch, 
         P.tiles_m = (P.m + C::kTileM - 1) / C::kTileM;
         P.tiles_n = (P.n + BN - 1) / BN;
         P.idesc_half = P.idesc | (static_cast<uint32_t>(128 >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
-        P.idesc |= (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
+        P.idesc |= (static_cast<uint32_t>(C::kMmaN >> 3) << 17) | (static_cast<uint32_t>(C::kTileM >> 4) << 24);
         P.tile_begin = static_cast<int>(tiles);
         const int64_t pt = static_cast<int64_t>(P.tiles_m) * P.tiles_n * batch[i];
         tiles += pt;
@@ -1117,6 +1139,7 @@ int tile_override() {
         if (t == "256") return 3;
         if (t == "128") return 4;
         if (t == "64") return 5;
+        if (t == "512p") return 6;
         return 0;
     }();
     return v;
@@ -1149,6 +1172,34 @@ int single_cta_width(const GemmDesc* d, int n, bool b_mn) {
     return best;
 }
 
+// Modelled time (us) of a launch on CTA pairs with `width`-wide tiles (256 or 512): the tiles,
+// longest K first, each go to the least-loaded pair.  A tile costs its k-blocks times the time
+// a k-block takes at that width -- the mainloop is bound by how fast each SM's TMA engine fills
+// shared memory, 32 KB per k-block and SM at 256 wide, 48 KB at 512 -- plus, at 512 wide (one
+// accumulator, so the epilogue cannot overlap the next tile's MMAs), its epilogue; at 256 wide
+// only each pair's last epilogue shows.  Constants measured on B200.
+double pair_width_cost(const GemmDesc* d, int n, int width, int pairs) {
+    const double kb_us = width == 512 ? 0.60 : 0.40;
+    const double epi_us = width == 512 ? 2.6 : 1.3;
+    std::vector<std::pair<int64_t, int64_t>> probs;  // (k-blocks, tiles)
+    for (int i = 0; i < n; ++i)
+        probs.push_back({(d[i].k + kBK - 1) / kBK, ((d[i].m + 255) / 256) * ((d[i].n + width - 1) / width) * d[i].batch});
+    std::sort(probs.begin(), probs.end(), [](const auto& x, const auto& y) { return x.first > y.first; });
+    std::vector<double> load(static_cast<size_t>(pairs), 0.0);
+    for (const auto& pr : probs) {
+        const double cost = static_cast<double>(pr.first) * kb_us + (width == 512 ? epi_us : 0.0);
+        // whole rounds go to every pair at once; the remainder to the least-loaded pairs
+        const int64_t rounds = pr.second / pairs;
+        if (rounds > 0)
+            for (double& l : load) l += static_cast<double>(rounds) * cost;
+        for (int64_t t = rounds * pairs; t < pr.second; ++t) {
+            auto it = std::min_element(load.begin(), load.end());
+            *it += cost;
+        }
+    }
+    return *std::max_element(load.begin(), load.end()) + (width == 512 ? 0.0 : epi_us);
+}
+
 TileChoice choose_tiles(const GemmDesc* d, int n) {
     bool narrow = false, short_m = false, b_mn = false;
     for (int i = 0; i < n; ++i) {
@@ -1163,6 +1214,7 @@ TileChoice choose_tiles(const GemmDesc* d, int n) {
         case 3: return {256, false};
         case 4: return {128, false};
         case 5: if (!b_mn) return {64, false}; break;
+        case 6: if (!b_mn) return {512, true}; break;
         default: break;
     }
     // Few output tiles: when the 256 x 256 pair tiles would keep at most half of the CTA pairs
@@ -1171,6 +1223,11 @@ TileChoice choose_tiles(const GemmDesc* d, int n) {
     int64_t pair_tiles = 0;
     for (int i = 0; i < n; ++i) pair_tiles += ((d[i].m + 255) / 256) * ((d[i].n + 255) / 256) * d[i].batch;
     if (4 * pair_tiles <= sm_count()) return {128, false};
+    // 512-wide pair tiles where the model says the launch gets shorter (K-major B only)
+    if (!b_mn) {
+        const int pairs = std::max(1, sm_count() / 2);
+        if (pair_width_cost(d, n, 512, pairs) < 0.93 * pair_width_cost(d, n, 256, pairs)) return {512, true};
+    }
     return {256, true};
 }
 
@@ -1249,7 +1306,8 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
     }
     if (colsum_cols > 0x7FFFFFFF || colsum_tiles > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "bias gradient too wide");
     const TileChoice tc = choose_tiles(work, nwork);
-    const int b_rows = tc.pair ? tc.bn / 2 : tc.bn;  // rows of B each CTA loads
+    // rows of B per TMA box: a CTA's share of one MMA's columns (two boxes per stage at 512 wide)
+    const int b_rows = tc.pair ? std::min(tc.bn / 2, 128) : tc.bn;
 
     CUtensorMap maps[8];  // per problem A, B, out; then per problem B in 64-row boxes (half tiles)
     GemmArgs g = fold_args;
@@ -1331,7 +1389,9 @@ int gemm_launch_group(const GemmDesc* descs, int ndesc, const float* colsum_part
     if (rc) return rc;
 
     launch_begin(kKindGemm, stream);
-    if (tc.pair)
+    if (tc.pair && tc.bn == 512)
+        rc = launch_cfg<512, true>(maps, g, batch, split, stream);
+    else if (tc.pair)
         rc = tc.bn == 256 ? launch_cfg<256, true>(maps, g, batch, split, stream)
                           : launch_cfg<128, true>(maps, g, batch, split, stream);
     else if (tc.bn == 256)

@@ -121,6 +121,14 @@ def test_last_round_half_tiles(layout):
     _run(layout, "e4m3", "e4m3", 2000, 2400, 384, bias="bf16", seed=21)
 
 
+@pytest.mark.parametrize("layout", ["NT", "TN"])
+def test_wide_pair_tiles(layout):
+    """A problem large enough for 256 x 512 pair tiles (two N = 256 MMAs per K step into one
+    512-column accumulator): ragged M and N, so the last tile column holds 416 valid columns and
+    its second MMA half is partly past n."""
+    _run(layout, "e4m3", "e4m3", 4000, 4000, 2048, bias="bf16", seed=23)
+
+
 def test_k_zero_writes_bias():
     _run("NT", "e4m3", "e4m3", 70, 90, 0, bias="bf16")
     _run("NT", "e4m3", "e4m3", 70, 90, 0, bias=None)
