@@ -1226,7 +1226,7 @@ TileChoice choose_tiles(const GemmDesc* d, int n) {
     // 512-wide pair tiles where the model says the launch gets shorter (K-major B only)
     if (!b_mn) {
         const int pairs = std::max(1, sm_count() / 2);
-        if (pair_width_cost(d, n, 512, pairs) < 0.93 * pair_width_cost(d, n, 256, pairs)) return {512, true};
+        if (pair_width_cost(d, n, 512, pairs) < 0.88 * pair_width_cost(d, n, 256, pairs)) return {512, true};
     }
     return {256, true};
 }
