@@ -60,6 +60,9 @@ constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 col
 #endif
 constexpr int kOutBufs = FP8DSA_GEMM_OUT_BUFS;    // staged boxes per epilogue warp (TMA stores in flight)
 constexpr int kMaxStages = 8;
+#ifndef FP8DSA_GEMM_EPI_WARPS
+#define FP8DSA_GEMM_EPI_WARPS 8  // at most this many epilogue warps (8 or 4)
+#endif
 constexpr int kSmemLimit = 232448;                // dynamic shared memory per CTA on sm_100
 constexpr int kMaxProblems = 2;
 
@@ -80,7 +83,8 @@ struct Cfg {
     static constexpr int kNMma = BN / kMmaN;
     static constexpr int kAccBufs = 2 * BN <= 512 ? 2 : 1;
     static constexpr int kTmemCols = kAccBufs * BN;
-    static constexpr int kEpiWarps = (BN >= 128 && ((kAStage + kBStage) <= 32768 || BN == 512)) ? 8 : 4;
+    static constexpr int kEpiWarps =
+        (FP8DSA_GEMM_EPI_WARPS >= 8 && BN >= 128 && ((kAStage + kBStage) <= 32768 || BN == 512)) ? 8 : 4;
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kEpiThreads = 32 * kEpiWarps;
     static constexpr int kEpiCols = BN / (kEpiWarps / 4);  // columns of the tile each epilogue warp owns
