@@ -91,6 +91,21 @@ def test_fp8_output_batched_with_padding():
     assert np.float32(am) == Q.amax(yv)
 
 
+def test_fp8_output_ragged_half_tiles_with_padding():
+    """80 pair tiles on 74 pairs: the last round runs as 256 x 128 half tiles, and with n = 2400
+    the last tile column holds 96 valid columns, so one half lies wholly past n.  Padded rows
+    (ldo > n): neither bf16 nor fp8 bytes may land past n, and the amax covers only the valid
+    columns."""
+    m, n, k, pad = 2000, 2400, 384, 32
+    o8, y, am, (ref, s_abs, sc) = _case("NT", m, n, k, ldo_pad=pad, out8_fmt="e4m3", step=0.05, seed=31)
+    yv = C.bf16_bits_to_f64(y[0][:, :n].copy()).astype(np.float32)
+    assert_within_gemm_bound(yv.astype(np.float64), ref, s_abs, sc, "bf16 output")
+    assert np.array_equal(o8[0][:, :n], Q.quantize_values(yv, 0.05, "e4m3"))
+    assert (o8[0][:, n:] == 0xAB).all(), "fp8 bytes written past n"
+    assert (y[0][:, n:] == 0x7FC1).all(), "bf16 values written past n"
+    assert np.float32(am) == Q.amax(yv)
+
+
 def test_fp8_output_feeds_a_ring():
     """out8_step = a ring's step and out8_amax = its amax slot: after fp8_scale_ring_fold the
     ring equals the oracle's ring folded with the amax of the bf16 output."""
