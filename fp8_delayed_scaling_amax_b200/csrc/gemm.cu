@@ -60,6 +60,9 @@ constexpr int kOutStageBytes = 32 * kOutBox * 2;  // one warp's 32 rows x 64 col
 #endif
 constexpr int kOutBufs = FP8DSA_GEMM_OUT_BUFS;    // staged boxes per epilogue warp (TMA stores in flight)
 constexpr int kMaxStages = 8;
+#ifndef FP8DSA_GEMM_GROUP_M
+#define FP8DSA_GEMM_GROUP_M 16  // tile rows per group of the grouped raster
+#endif
 #ifndef FP8DSA_GEMM_EPI_WARPS
 #define FP8DSA_GEMM_EPI_WARPS 8  // at most this many epilogue warps (8 or 4)
 #endif
@@ -172,9 +175,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-// Tile -> (problem, batch, tile row, tile column); grouped raster of 8 tile rows per problem.
+// Tile -> (problem, batch, tile row, tile column); grouped raster of FP8DSA_GEMM_GROUP_M tile rows per problem.
 __device__ __forceinline__ void decode_tile(int tile, const GemmArgs& g, int& pi, int& b, int& tm, int& tn) {
-    constexpr int kGroupM = 8;
+    constexpr int kGroupM = FP8DSA_GEMM_GROUP_M;
     pi = (g.nprob > 1 && tile >= g.p[1].tile_begin) ? 1 : 0;
     const GemmProblem& P = g.p[pi];
     const int t = tile - P.tile_begin;
