@@ -283,3 +283,44 @@ def test_saved_row_major_pair_equals_saved_transpose_pair(mkn):
     assert torch.equal(torch.cat([sx, sw, sg]), torch.cat([sx2, sw2, sg2]))
     for a, b in zip((xr, wr, gr), (xr2, wr2, gr2)):
         assert np.array_equal(_state_bits(a), _state_bits(b))
+
+
+def test_weight_gradient_split_from_the_backward_on_another_stream():
+    """The row-major backward run as grad_x + grad_b first (linear_backward_fp8_mixed without
+    grad_w; its g8 stays at the start of its workspace), then grad_w on a second stream from those
+    bytes (linear_backward_fp8_prequant with g and x pre-quantized): every output and the ring
+    bit-identical to the one-launch backward."""
+    m, k, n = 512, 384, 640
+    _, d, _ = _tensors(m, k, n, 6400)
+    rings = []
+    for _ in range(2):
+        rs = (_ring(16, F.FP8_E4M3), _ring(16, F.FP8_E4M3), _ring(16, F.FP8_E5M2))
+        for rr, key in zip(rs, ("x", "w", "g")):
+            F.fp8_scale_ring_seed(rr, d[key], F.FP8_IN_BF16, d[key].numel())
+        rings.append(rs)
+    (xr, wr, gr), (xr2, wr2, gr2) = rings
+    y, x8b, w8b, sx, sw = _forward_save_rm(d["x"], d["w"], d["b"], xr, wr)
+    gx, gw, gb, sg = _backward_rm(d["g"], x8b, w8b, sx, sw, gr)
+    # the split: grad_x + grad_b, then grad_w on a side stream
+    nb = F.linear_backward_fp8_mixed_workspace_size(m, k, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device=DEV)
+    gx2 = torch.empty_like(gx)
+    gw2 = torch.full_like(gw, float("nan"))
+    gb2 = torch.empty_like(gb)
+    sg2 = torch.zeros(1, device=DEV)
+    F.linear_backward_fp8_mixed(d["g"], x8b, w8b, m, k, n, F.FP8_E5M2, F.FP8_E5M2, F.FP8_E5M2, 1, 0, 1, sx, sw, gr2,
+                                1.0, sg2, ws, nb, gx2, None, gb2)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    nq = F.linear_backward_fp8_workspace_size(m, k, n)
+    wsq = torch.empty(nq, dtype=torch.uint8, device=DEV)
+    with torch.cuda.stream(side):
+        F.linear_backward_fp8_prequant(ws, 1, sg2, x8b, 1, None, 0, m, k, n, F.FP8_E5M2, 0, 1, 0, sx, None, None, 1.0,
+                                       None, wsq, nq, None, gw2, None)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert F.fp8_get_device_status() == 0
+    for a, b in ((gx, gx2), (gw, gw2), (gb, gb2)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(sg, sg2)
+    assert np.array_equal(_state_bits(gr), _state_bits(gr2))
