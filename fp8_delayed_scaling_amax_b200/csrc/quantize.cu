@@ -172,9 +172,14 @@ __device__ __forceinline__ void zero_side_job(const QBatch& b) {
 
 // Chunks of 16 elements each thread of the row-major kernel has in flight (16-bit inputs).
 #ifndef FP8DSA_FLAT_DEPTH
-#define FP8DSA_FLAT_DEPTH 2
+#define FP8DSA_FLAT_DEPTH 3
 #endif
 constexpr int kFlatDepth = FP8DSA_FLAT_DEPTH;
+// Resident 256-thread blocks per SM the row-major kernel is built for (its launch bounds).
+#ifndef FP8DSA_FLAT_BLOCKS
+#define FP8DSA_FLAT_BLOCKS 3
+#endif
+constexpr int kFlatBlocks = FP8DSA_FLAT_BLOCKS;
 
 // Eight floats -> eight fp8 bytes (two words): each byte is the RN, saturating encoding of
 // RN32(f * mult), the products taken two per packed instruction; amax is kept by the caller.
@@ -286,7 +291,7 @@ __device__ __forceinline__ void block_finish(const QArgs& a, float amax, float s
 // A tensor with out2 also gets its bytes in format kFmt2 (the same products, rounded once
 // more; kFmt2 == kFmt copies the same bytes), row-major like out.
 template <class In, int kFmt, int kFmt2>
-__global__ void __launch_bounds__(kThreads, 4) quant_flat_kernel(const __grid_constant__ QBatch batch) {
+__global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const __grid_constant__ QBatch batch) {
     pdl_trigger();
     pdl_wait();
     zero_side_job(batch);
@@ -971,8 +976,8 @@ __global__ void __launch_bounds__(kThreads) colsum_fp8_kernel(const uint8_t* g8,
 // block looping over its share, beats several waves of shorter blocks).
 constexpr int kFlatWaves = 1;
 
-// Resident 256-thread blocks per SM of the row-major kernel (its launch bounds ask for 4).
-int flat_blocks_per_sm() { return 4; }
+// Resident 256-thread blocks per SM of the row-major kernel (its launch bounds ask for as many).
+int flat_blocks_per_sm() { return kFlatBlocks; }
 
 template <int kFmt, int kFmt2, class In>
 void launch_flat(const QBatch& b, dim3 grid, cudaStream_t stream) {
