@@ -202,13 +202,15 @@ def _forward_save_rm(x, w, b, xr, wr, fmt_b=F.FP8_E5M2):
 
 
 def _backward_rm(g, x8b, w8b, sx, sw, gr, need=(1, 1, 1), fmt_b=F.FP8_E5M2):
+    # outputs pre-filled with a finite sentinel (the saved-transpose helper uses NaN), so an
+    # output that neither composition writes cannot compare equal
     m, n = g.shape
     k = x8b.shape[1]
     nbytes = F.linear_backward_fp8_mixed_workspace_size(m, k, n)
     ws = torch.full((nbytes,), 0xC3, dtype=torch.uint8, device=DEV)
-    gx = torch.full((m, k), float("nan"), dtype=torch.bfloat16, device=DEV)
-    gw = torch.full((n, k), float("nan"), dtype=torch.bfloat16, device=DEV)
-    gb = torch.full((n,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    gx = torch.full((m, k), -1234.5, dtype=torch.bfloat16, device=DEV)
+    gw = torch.full((n, k), -1234.5, dtype=torch.bfloat16, device=DEV)
+    gb = torch.full((n,), -1234.5, dtype=torch.bfloat16, device=DEV)
     sg = torch.zeros(1, device=DEV)
     F.linear_backward_fp8_mixed(g, x8b, w8b, m, k, n, F.FP8_E5M2, fmt_b, fmt_b, need[0], need[1], need[2], sx, sw,
                                 gr, 1.0, sg, ws, nbytes, gx, gw, gb)
