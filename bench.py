@@ -486,9 +486,11 @@ def _graph_time(torch, launch, iters, warmup, slots=1):
     return e0.elapsed_time(e1) / (iters * slots)
 
 
-def time_gemm(F, W, torch, dev, m, n, k, iters=20, warmup=5, batch=1, bcast_b=False):
+def time_gemm(F, W, torch, dev, m, n, k, iters=20, warmup=5, batch=1, bcast_b=False, hot=False):
+    """hot=False: enough operand sets rotated that each launch reads from HBM; hot=True: one
+    set, so operands smaller than L2 stay resident (the pages time their GEMMs this way)."""
     per_set = batch * m * k + (1 if bcast_b else batch) * n * k + batch * m * n * 2
-    nsets = max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
+    nsets = 1 if hot else max(1, min(16, (2 * L2_BYTES) // max(per_set, 1) + 1))
     sets = []
     for i in range(nsets):
         a = W.fp8_bytes((batch, m, k), seed=31 + i, device=dev)
@@ -615,16 +617,22 @@ def run_sweeps(F, W, torch, dev):
     peaks = measured_peaks()
     burst_fp8 = 2.0 * peaks["bf16_tflops"]
     out = {"gemm_square": {}, "gemm_skinny_batched": {}, "quantize": {}, "gemm_fp8_output": {}}
+    def gemm_entry(m, n, k, batch=1, bcast_b=False, iters=20):
+        r = time_gemm(F, W, torch, dev, m, n, k, iters=iters, batch=batch, bcast_b=bcast_b)
+        e = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2), "frac": round(r["tflops"] / burst_fp8, 4)}
+        # operands that fit in L2 are also timed hot (one operand set, as the pages time them)
+        per_set = batch * m * k + (1 if bcast_b else batch) * n * k + batch * m * n * 2
+        if per_set < L2_BYTES // 2:
+            h = time_gemm(F, W, torch, dev, m, n, k, iters=iters, batch=batch, bcast_b=bcast_b, hot=True)
+            e.update(hot_tflops=round(h["tflops"], 1), hot_us=round(h["ms"] * 1e3, 2))
+        return e
+
     for s in W.SQUARE_SIZES:
-        r = time_gemm(F, W, torch, dev, s, s, s, iters=20 if s < 8192 else 10)
-        out["gemm_square"][str(s)] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
-                                      "frac": round(r["tflops"] / burst_fp8, 4)}
+        out["gemm_square"][str(s)] = gemm_entry(s, s, s, iters=20 if s < 8192 else 10)
     for ba, bb, m, n, k in W.SKINNY_BATCHED:
         batch = max(ba, bb)
-        r = time_gemm(F, W, torch, dev, m, n, k, batch=batch, bcast_b=(bb == 1 and batch > 1))
         key = f"{batch}x{m}x{n}x{k}" + ("(B bcast)" if bb == 1 and batch > 1 else "")
-        out["gemm_skinny_batched"][key] = {"tflops": round(r["tflops"], 1), "us": round(r["ms"] * 1e3, 2),
-                                           "frac": round(r["tflops"] / burst_fp8, 4)}
+        out["gemm_skinny_batched"][key] = gemm_entry(m, n, k, batch=batch, bcast_b=(bb == 1 and batch > 1))
     # bf16 inputs of 2^24 .. 2^28 elements with a ring; E5M2 beside E4M3 at the two larger sizes
     for rows, cols, fmts in ((8192, 2048, ("e4m3",)), (4096, 4096, ("e4m3",)), (8192, 8192, ("e4m3", "e5m2")),
                              (16384, 16384, ("e4m3", "e5m2"))):

@@ -175,6 +175,11 @@ __device__ __forceinline__ void zero_side_job(const QBatch& b) {
 #define FP8DSA_FLAT_DEPTH 3
 #endif
 constexpr int kFlatDepth = FP8DSA_FLAT_DEPTH;
+// 1: the row-major kernel's rounds are software-pipelined (round r + 1 loads while round r
+// converts); 0: each round loads, then converts.
+#ifndef FP8DSA_FLAT_PIPE
+#define FP8DSA_FLAT_PIPE 0
+#endif
 // Resident 256-thread blocks per SM the row-major kernel is built for (its launch bounds).
 #ifndef FP8DSA_FLAT_BLOCKS
 #define FP8DSA_FLAT_BLOCKS 3
@@ -314,8 +319,7 @@ __global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const
     // kDepth chunks of 16 elements per thread in flight: every load of a round is issued before
     // the round's first conversion
     constexpr int kDepth = sizeof(typename In::E) == 4 ? 2 : kFlatDepth;
-    for (int64_t g = tid; g < n16; g += kDepth * gstride) {
-        typename In::Raw r[kDepth][2];
+    auto load_round = [&](int64_t g, typename In::Raw (&r)[kDepth][2]) {
 #pragma unroll
         for (int d = 0; d < kDepth; ++d) {
             const int64_t gd = g + d * gstride;
@@ -324,6 +328,8 @@ __global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const
                 r[d][1] = In::load_raw(x + gd * 16 + 8);
             }
         }
+    };
+    auto convert_round = [&](int64_t g, const typename In::Raw (&r)[kDepth][2]) {
 #pragma unroll
         for (int d = 0; d < kDepth; ++d) {
             const int64_t gd = g + d * gstride;
@@ -342,7 +348,34 @@ __global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const
                 *reinterpret_cast<uint4*>(out2 + gd * 16) = make_uint4(lo2.x, lo2.y, hi2.x, hi2.y);
             }
         }
+    };
+#if FP8DSA_FLAT_PIPE
+    // software-pipelined: the next round's loads are in flight while this round converts
+    {
+        typename In::Raw r[kDepth][2];
+        int64_t g = tid;
+        if (g < n16) load_round(g, r);
+        for (; g < n16; g += kDepth * gstride) {
+            typename In::Raw nx[kDepth][2];
+            const int64_t gn = g + kDepth * gstride;
+            if (gn < n16) load_round(gn, nx);
+            convert_round(g, r);
+            if (gn < n16) {
+#pragma unroll
+                for (int d = 0; d < kDepth; ++d) {
+                    r[d][0] = nx[d][0];
+                    r[d][1] = nx[d][1];
+                }
+            }
+        }
     }
+#else
+    for (int64_t g = tid; g < n16; g += kDepth * gstride) {
+        typename In::Raw r[kDepth][2];
+        load_round(g, r);
+        convert_round(g, r);
+    }
+#endif
     amax = In::acc_value(acc);
     for (int64_t i = n16 * 16 + tid; i < a.numel; i += gstride) {
         const float v = In::cvt(x[i]);
