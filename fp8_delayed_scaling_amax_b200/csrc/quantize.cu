@@ -389,17 +389,22 @@ __global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const
 
 // ----------------------------------------------------------------------------------------
 // Row-major bytes plus per-tile column sums (a gradient quantized for the bias gradient), for
-// batches that write no transposed bytes.  Each block covers 128 rows x 64 columns of one
-// tensor, so small tensors still spread over many blocks: thread t owns the 8 columns
-// 8 * (t % 8) .. + 7 and the rows t / 8 + 32 i (i = 0..3), issues its four 16-byte loads at
-// once, and keeps the 8 column sums of its rows in registers.  The 32 row threads of a column
-// group reduce through two shuffles and an 8-warp shared-memory sum, in a fixed order, into
-// colsum[tile row][column] (the layout the dual quantize writes).
+// batches that write no transposed bytes.  Each block covers 128 rows x 128 columns of one
+// tensor: thread t owns the 8 columns 8 * (t % 16) .. + 7 and the rows t / 16 + 16 i
+// (i = 0..7), issues its eight 16-byte loads at once (a warp reads two 256-byte row pieces per
+// load), and keeps the 8 column sums of its rows in registers.  The two row threads of a
+// column group in a warp combine through one shuffle, then the 8 warps in order through shared
+// memory, into colsum[tile row][column] (the layout the dual quantize writes; the summation
+// order is this kernel's own).  Eight rows per thread keep the reduction a small share of the
+// work (measured on B200: 128 x 64 blocks of four rows per thread spent most of their
+// instructions on it).
 // ----------------------------------------------------------------------------------------
-constexpr int kRcCols = 64;
+constexpr int kRcCols = 128;
+constexpr int kRcRows = 8;  // rows per thread
 
 template <class In, int kFmt>
-__global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __grid_constant__ QBatch batch) {
+__global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
+    quant_rows_colsum_kernel(const __grid_constant__ QBatch batch) {
     pdl_trigger();
     pdl_wait();
     zero_side_job(batch);
@@ -416,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __
     const auto* x = static_cast<const typename In::E*>(a.x);
     const int64_t rows = a.rows, cols = a.cols;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    const int cg = t & 7, rt = t >> 3;
+    const int cg = t & 15, rt = t >> 4;
     const int64_t r0 = static_cast<int64_t>(ty) * kTile;
     const int64_t gc = static_cast<int64_t>(tx) * kRcCols + 8 * cg;
     const bool colsum = a.colsum != nullptr;
@@ -426,11 +431,11 @@ __global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __
     float amax = 0.0f;
     typename In::Acc acc = In::acc_zero();
     if (a.vec_in && a.vec_out && r0 + kTile <= rows && gc + 8 <= cols) {
-        typename In::Raw raw[4];
+        typename In::Raw raw[kRcRows];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) raw[i] = In::load_raw(x + (r0 + rt + 32 * i) * cols + gc);
+        for (int i = 0; i < kRcRows; ++i) raw[i] = In::load_raw(x + (r0 + rt + 16 * i) * cols + gc);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kRcRows; ++i) {
             float f[8];
             In::acc_max(acc, raw[i]);
             In::unpack(raw[i], f);
@@ -438,12 +443,12 @@ __global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
             }
-            *reinterpret_cast<uint2*>(a.out + (r0 + rt + 32 * i) * cols + gc) = quant8<kFmt>(f, mult);
+            *reinterpret_cast<uint2*>(a.out + (r0 + rt + 16 * i) * cols + gc) = quant8<kFmt>(f, mult);
         }
     } else {
 #pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-            const int64_t gr = r0 + rt + 32 * i;
+        for (int i = 0; i < kRcRows; ++i) {
+            const int64_t gr = r0 + rt + 16 * i;
             float f[8];
             if (gr < rows && a.vec_in && gc + 8 <= cols) {
                 In::load8(x + gr * cols + gc, f);
@@ -471,13 +476,11 @@ __global__ void __launch_bounds__(kThreads, 6) quant_rows_colsum_kernel(const __
     }
     amax = fmaxf(amax, In::acc_value(acc));
     if (colsum) {
-        // lanes l, l ^ 8, l ^ 16, l ^ 24 share the column group; then the 8 warps in order
+        // lanes l and l ^ 16 share the column group (rows t / 16 and t / 16 + 1); then the 8
+        // warps in order
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 8);
-            cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
-        }
-        if (lane < 8) {
+        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
+        if (lane < 16) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) s_cs[w][8 * lane + e] = cs[e];
         }
@@ -1097,8 +1100,8 @@ int launch_rows_colsum(fp8_in_t in_type, const QBatch& b, cudaStream_t stream) {
     return FP8DSA_OK;
 }
 
-// Tuning override: FP8DSA_ROWS_COLSUM=0 sends row-major + column-sum batches to the 128 x 128
-// tiled kernel instead of the 128 x 64 block kernel (read once).
+// Tuning override: FP8DSA_ROWS_COLSUM=0 sends row-major + column-sum batches to the tiled
+// kernel instead of the row-major column-sum kernel (read once).
 bool row_colsum_enabled() {
     static const bool v = [] {
         const char* e = std::getenv("FP8DSA_ROWS_COLSUM");
@@ -1143,7 +1146,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
     if (any_out2 && tiled) return fail(FP8DSA_ERR_INVALID_ARG, "a second row-major copy is a row-major launch");
     if (fmt_t != fmt && !tiled && !any_out2)
         return fail(FP8DSA_ERR_INVALID_ARG, "a second format needs the transposed output or a second row-major copy");
-    // row-major bytes + column sums and no transposed bytes: the 128 x 64 block kernel
+    // row-major bytes + column sums and no transposed bytes: the 128 x 128 block kernel
     bool rows_colsum = tiled && fmt_t == fmt && row_colsum_enabled();
     for (int i = 0; i < njobs; ++i)
         rows_colsum = rows_colsum && jobs[i].out_t == nullptr && jobs[i].out != nullptr && jobs[i].colsum_partial != nullptr;
@@ -1203,7 +1206,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
         }
         bytes += static_cast<double>(a.numel) * (eb + (job.out ? 1 : 0) + (job.out_t ? 1 : 0) + (job.out2 ? 1 : 0));
         if (tiled && rows_colsum) {
-            // 128 x 64 blocks of the row-major + column-sum kernel (an empty tensor: one block)
+            // 128 x 128 blocks of the row-major + column-sum kernel (an empty tensor: one block)
             const int64_t tx = std::max<int64_t>(1, (job.cols + kRcCols - 1) / kRcCols);
             const int64_t ty = std::max<int64_t>(1, (job.rows + kTile - 1) / kTile);
             a.tiles_x = static_cast<int>(tx);
@@ -1212,7 +1215,7 @@ int launch_quantize_batch(const QuantJob* jobs, int njobs, cudaStream_t stream, 
             a.tile_begin = static_cast<int>(tiles_total);
             a.nblocks = static_cast<unsigned>(tx * ty);
             tiles_total += tx * ty;
-            if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 64 blocks");
+            if (tiles_total > kMaxTiles) return fail(FP8DSA_ERR_UNSUPPORTED, "too many 128 x 128 blocks");
         } else if (tiled) {
             // an empty tensor still gets one (empty) tile
             const int64_t tx = std::max<int64_t>(1, (job.cols + kTile - 1) / kTile);
