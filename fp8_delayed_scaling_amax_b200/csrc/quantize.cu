@@ -399,11 +399,17 @@ __global__ void __launch_bounds__(kThreads, kFlatBlocks) quant_flat_kernel(const
 // work (measured on B200: 128 x 64 blocks of four rows per thread spent most of their
 // instructions on it).
 // ----------------------------------------------------------------------------------------
-constexpr int kRcCols = 128;
-constexpr int kRcRows = 8;  // rows per thread
+#ifndef FP8DSA_RC_ROWS
+#define FP8DSA_RC_ROWS 8
+#endif
+constexpr int kRcRows = FP8DSA_RC_ROWS;             // rows per thread (8 or 16)
+constexpr int kRcGroups = 2 * kRcRows;              // 8-column groups per block
+constexpr int kRcCols = 8 * kRcGroups;              // 128 (or 256) columns per block
+constexpr int kRcStride = kTile / kRcRows;          // row distance between a thread's rows
+static_assert(kRcRows == 8 || kRcRows == 16, "8 or 16 rows per thread");
 
 template <class In, int kFmt>
-__global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, (sizeof(typename In::E) == 4 || kRcRows > 8) ? 2 : 3)
     quant_rows_colsum_kernel(const __grid_constant__ QBatch batch) {
     pdl_trigger();
     pdl_wait();
@@ -421,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
     const auto* x = static_cast<const typename In::E*>(a.x);
     const int64_t rows = a.rows, cols = a.cols;
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    const int cg = t & 15, rt = t >> 4;
+    const int cg = t % kRcGroups, rt = t / kRcGroups;
     const int64_t r0 = static_cast<int64_t>(ty) * kTile;
     const int64_t gc = static_cast<int64_t>(tx) * kRcCols + 8 * cg;
     const bool colsum = a.colsum != nullptr;
@@ -433,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
     if (a.vec_in && a.vec_out && r0 + kTile <= rows && gc + 8 <= cols) {
         typename In::Raw raw[kRcRows];
 #pragma unroll
-        for (int i = 0; i < kRcRows; ++i) raw[i] = In::load_raw(x + (r0 + rt + 16 * i) * cols + gc);
+        for (int i = 0; i < kRcRows; ++i) raw[i] = In::load_raw(x + (r0 + rt + kRcStride * i) * cols + gc);
 #pragma unroll
         for (int i = 0; i < kRcRows; ++i) {
             float f[8];
@@ -443,12 +449,12 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) add2_rn(cs[e], cs[e + 1], f[e], f[e + 1]);
             }
-            *reinterpret_cast<uint2*>(a.out + (r0 + rt + 16 * i) * cols + gc) = quant8<kFmt>(f, mult);
+            *reinterpret_cast<uint2*>(a.out + (r0 + rt + kRcStride * i) * cols + gc) = quant8<kFmt>(f, mult);
         }
     } else {
 #pragma unroll 1
         for (int i = 0; i < kRcRows; ++i) {
-            const int64_t gr = r0 + rt + 16 * i;
+            const int64_t gr = r0 + rt + kRcStride * i;
             float f[8];
             if (gr < rows && a.vec_in && gc + 8 <= cols) {
                 In::load8(x + gr * cols + gc, f);
@@ -476,11 +482,13 @@ __global__ void __launch_bounds__(kThreads, sizeof(typename In::E) == 4 ? 2 : 3)
     }
     amax = fmaxf(amax, In::acc_value(acc));
     if (colsum) {
-        // lanes l and l ^ 16 share the column group (rows t / 16 and t / 16 + 1); then the 8
-        // warps in order
+        // with 8 rows per thread, lanes l and l ^ 16 share the column group (rows t / 16 and
+        // t / 16 + 1); then the 8 warps in order
+        if constexpr (kRcGroups < 32) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
-        if (lane < 16) {
+            for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xFFFFFFFFu, cs[e], 16);
+        }
+        if (lane < kRcGroups) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) s_cs[w][8 * lane + e] = cs[e];
         }
