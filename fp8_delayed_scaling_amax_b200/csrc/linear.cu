@@ -148,6 +148,10 @@ SavedLayout saved_layout(int64_t m, int64_t k, int64_t n) {
     return L;
 }
 
+// A tensor's pointer is required only when the tensor has elements (an empty batch may come
+// with null pointers, as empty framework tensors do).
+inline bool missing(const void* p, int64_t elems) { return p == nullptr && elems > 0; }
+
 int check_ring_arg(const fp8_ring_t* r, const char* name) {
     if (r == nullptr) return FP8DSA_OK;
     if (r->state == nullptr || r->hist_len < 1 || r->hist_idx < 0 || r->hist_idx >= r->hist_len ||
@@ -196,7 +200,8 @@ int linear_forward_fp8_save_t(const void* x, const void* w, const void* bias, co
                               const fp8_ring_t* w_ring, float* sx_used, float* sw_used, uint8_t* x8t_out,
                               uint8_t* w8t_out, void* workspace, size_t workspace_bytes, void* y, cudaStream_t stream) {
     clear_error();
-    if (x8t_out == nullptr || w8t_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x8t_out and w8t_out are required");
+    if (missing(x8t_out, m * k) || missing(w8t_out, n * k))
+        return fail(FP8DSA_ERR_INVALID_ARG, "x8t_out and w8t_out are required");
     return linear_forward_impl(x, w, 0, nullptr, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, 1.0f, sx_used,
                                sw_used, nullptr, nullptr, x8t_out, w8t_out, fmt_t, workspace, workspace_bytes, true, y,
                                stream);
@@ -208,7 +213,8 @@ int linear_forward_fp8_save_rm(const void* x, const void* w, const void* bias, c
                                uint8_t* w8b_out, void* workspace, size_t workspace_bytes, void* y,
                                cudaStream_t stream) {
     clear_error();
-    if (x8b_out == nullptr || w8b_out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "x8b_out and w8b_out are required");
+    if (missing(x8b_out, m * k) || missing(w8b_out, n * k))
+        return fail(FP8DSA_ERR_INVALID_ARG, "x8b_out and w8b_out are required");
     return linear_forward_impl(x, w, 0, nullptr, bias, bias_scale, m, k, n, fmt, x_ring, w_ring, 1.0f, sx_used,
                                sw_used, nullptr, nullptr, x8b_out, w8b_out, fmt_b, workspace, workspace_bytes, true, y,
                                stream, true);
@@ -237,7 +243,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    if (x == nullptr || w == nullptr || y == nullptr || workspace == nullptr)
+    if (missing(x, m * k) || missing(w, n * k) || missing(y, m * n) || workspace == nullptr)
         return fail(FP8DSA_ERR_INVALID_ARG, "x, w, y and workspace are required");
     if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
     if (w_is_fp8 && w_step == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "w_is_fp8 needs w_step");
@@ -259,10 +265,12 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     if (w_is_fp8 && !aligned16(w)) return fail(FP8DSA_ERR_UNSUPPORTED, "fp8 w must be 16-byte aligned");
     if ((x8_keep != nullptr && !aligned16(x8_keep)) || (!w_is_fp8 && w8_keep != nullptr && !aligned16(w8_keep)))
         return fail(FP8DSA_ERR_UNSUPPORTED, "x8_out / w8_out must be 16-byte aligned");
-    const bool save_t = x8t_keep != nullptr;
+    // the backward's copies are asked for by either output (one of them is null when its tensor
+    // is empty)
+    const bool save_t = x8t_keep != nullptr || w8t_keep != nullptr;
     if (save_t) {
         if (!valid_fmt(fmt_t)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt_t must be FP8_E4M3 or FP8_E5M2");
-        if (dynamic || w_is_fp8 || w8t_keep == nullptr)
+        if (dynamic || w_is_fp8 || missing(x8t_keep, m * k) || missing(w8t_keep, n * k))
             return fail(FP8DSA_ERR_INVALID_ARG, "transposed copies need x_ring, w_ring, a bf16 w and both outputs");
         if (!aligned16(x8t_keep) || !aligned16(w8t_keep))
             return fail(FP8DSA_ERR_UNSUPPORTED, "x8t_out / w8t_out must be 16-byte aligned");
@@ -312,7 +320,8 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
     qx.fmt = fmt;
     qx.out = x8;
     if (save_t) {  // the backward's copy of x from the same products, in its own format
-        (copies_row_major ? qx.out2 : qx.out_t) = x8t_keep;
+        // an empty x writes no bytes; a placeholder keeps its job in the launch's orientation
+        (copies_row_major ? qx.out2 : qx.out_t) = x8t_keep != nullptr ? x8t_keep : ws;
         qx.fmt_t = fmt_t;
     }
     if (dynamic) {
@@ -334,7 +343,7 @@ int linear_forward_impl(const void* x, const void* w, int w_is_fp8, const float*
         qw.fmt = fmt;
         qw.out = w8;
         if (save_t) {
-            (copies_row_major ? qw.out2 : qw.out_t) = w8t_keep;
+            (copies_row_major ? qw.out2 : qw.out_t) = w8t_keep != nullptr ? w8t_keep : ws;
             qw.fmt_t = fmt_t;
         }
         if (dynamic) {
@@ -381,10 +390,12 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
-    if (need_grad_x && (w == nullptr || grad_x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
-    if (need_grad_w && (x == nullptr || grad_w == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
-    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (missing(g, m * n) || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (missing(w, n * k) || missing(grad_x, m * k)))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
+    if (need_grad_w && (missing(x, m * k) || missing(grad_w, n * k)))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
+    if (need_grad_b && missing(grad_b, n)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
     if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
     if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
     const bool dynamic = g_ring == nullptr;
@@ -456,7 +467,7 @@ int linear_backward_fp8(const void* g, const void* x, const void* w, int64_t m, 
     qg.fmt = fmt;
     qg.out = g8;
     qg.out_t = g8t;
-    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    qg.colsum_partial = need_grad_b && m > 0 ? colsum : nullptr;  // no rows: grad_b is zero, no partials
     if (dynamic) {
         qg.scale = sg;
     } else {
@@ -519,10 +530,12 @@ int linear_backward_fp8_prequant(const void* g, int g_is_fp8, const float* g_ste
     clear_error();
     if (!valid_fmt(fmt)) return fail(FP8DSA_ERR_INVALID_ARG, "fmt must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
-    if (need_grad_x && (w == nullptr || grad_x == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
-    if (need_grad_w && (x == nullptr || grad_w == nullptr)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
-    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (missing(g, m * n) || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (missing(w, n * k) || missing(grad_x, m * k)))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w and grad_x");
+    if (need_grad_w && (missing(x, m * k) || missing(grad_w, n * k)))
+        return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x and grad_w");
+    if (need_grad_b && missing(grad_b, n)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
     if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
     if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
     if (g_is_fp8 && g_step == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "a pre-quantized g needs g_step");
@@ -600,7 +613,7 @@ int linear_backward_fp8_prequant(const void* g, int g_is_fp8, const float* g_ste
         q.fmt = fmt;
         q.out = ws + L.g8;
         q.out_t = g8t;
-        q.colsum_partial = need_grad_b ? colsum : nullptr;
+        q.colsum_partial = need_grad_b && m > 0 ? colsum : nullptr;
         if (dynamic) {
             q.scale = sg;
         } else {
@@ -677,12 +690,12 @@ int linear_backward_fp8_saved_t(const void* g, const uint8_t* x8t, const uint8_t
     clear_error();
     if (!valid_fmt(fmt) || !valid_fmt(fmt_t)) return fail(FP8DSA_ERR_INVALID_ARG, "formats must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
-    if (need_grad_x && (w8t == nullptr || sw == nullptr || grad_x == nullptr))
+    if (missing(g, m * n) || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (missing(w8t, n * k) || sw == nullptr || missing(grad_x, m * k)))
         return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w8t, sw and grad_x");
-    if (need_grad_w && (x8t == nullptr || sx == nullptr || grad_w == nullptr))
+    if (need_grad_w && (missing(x8t, m * k) || sx == nullptr || missing(grad_w, n * k)))
         return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x8t, sx and grad_w");
-    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (need_grad_b && missing(grad_b, n)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
     if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
     if (need_grad_w && m % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "m must be a multiple of 16 for grad_w");
     if ((need_grad_w && !aligned16(x8t)) || (need_grad_x && !aligned16(w8t)))
@@ -727,7 +740,7 @@ int linear_backward_fp8_saved_t(const void* g, const uint8_t* x8t, const uint8_t
     qg.fmt = fmt;
     qg.out = g8;
     qg.out_t = g8t;
-    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    qg.colsum_partial = need_grad_b && m > 0 ? colsum : nullptr;  // no rows: grad_b is zero, no partials
     if (dynamic) {
         qg.scale = sg;
     } else {
@@ -769,12 +782,12 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
     if (!valid_fmt(fmt_g) || !valid_fmt(fmt_x) || !valid_fmt(fmt_w))
         return fail(FP8DSA_ERR_INVALID_ARG, "formats must be FP8_E4M3 or FP8_E5M2");
     if (m < 0 || k < 0 || n < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
-    if (g == nullptr || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
-    if (need_grad_x && (w8 == nullptr || sw == nullptr || grad_x == nullptr))
+    if (missing(g, m * n) || workspace == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "g and workspace are required");
+    if (need_grad_x && (missing(w8, n * k) || sw == nullptr || missing(grad_x, m * k)))
         return fail(FP8DSA_ERR_INVALID_ARG, "grad_x needs w8, sw and grad_x");
-    if (need_grad_w && (x8 == nullptr || sx == nullptr || grad_w == nullptr))
+    if (need_grad_w && (missing(x8, m * k) || sx == nullptr || missing(grad_w, n * k)))
         return fail(FP8DSA_ERR_INVALID_ARG, "grad_w needs x8, sx and grad_w");
-    if (need_grad_b && grad_b == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
+    if (need_grad_b && missing(grad_b, n)) return fail(FP8DSA_ERR_INVALID_ARG, "grad_b is NULL");
     if (k % 16 != 0 || n % 16 != 0) return fail(FP8DSA_ERR_UNSUPPORTED, "k and n must be multiples of 16");
     if ((need_grad_w && !aligned16(x8)) || (need_grad_x && !aligned16(w8)))
         return fail(FP8DSA_ERR_UNSUPPORTED, "x8 and w8 must be 16-byte aligned");
@@ -816,7 +829,7 @@ int linear_backward_fp8_mixed(const void* g, const uint8_t* x8, const uint8_t* w
     qg.cols = n;
     qg.fmt = fmt_g;
     qg.out = g8;
-    qg.colsum_partial = need_grad_b ? colsum : nullptr;
+    qg.colsum_partial = need_grad_b && m > 0 ? colsum : nullptr;  // no rows: grad_b is zero, no partials
     if (dynamic) {
         qg.scale = sg;
     } else {

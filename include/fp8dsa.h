@@ -22,6 +22,11 @@
  *   FP8DSA_ERR_CUDA, and fp8_last_error() returns a thread-local message.
  * - fp8 bytes: E4M3FN (max 448) or E5M2 (max 57344) [compare: csrc/kernels/fp8/common.h,
  *   FP8Format].  bf16 / f16 / f32 inputs are IEEE bit patterns.
+ * - Empty tensors: a tensor argument without elements (a batch of m = 0 rows, k = 0, ...) may be
+ *   NULL, as empty framework tensors are.  The linear entries then compute what the
+ *   definition gives: an empty tensor's amax is 0 and is recorded by its ring; y and grad_x of
+ *   no rows have no elements; grad_w and grad_b, sums over no rows, are zero; with k = 0, y is
+ *   the bias (or zero).  Rings, step buffers and the workspace follow their usual rules.
  */
 #ifndef FP8DSA_H
 #define FP8DSA_H
