@@ -1,10 +1,12 @@
-"""GPU parity on the degenerate batch: no rows (m = 0), and no inner dimension (k = 0).
+"""GPU parity on the degenerate batch: no rows (m = 0), no output columns (n = 0), and no inner
+dimension (k = 0).
 
 An empty batch comes with null pointers for its empty tensors (framework tensors without
 elements have none).  The linear entries accept them and do what the definition gives for no
 rows: the quantize of an empty x or g measures an amax of 0, and the ring records it; y and
 grad_x have no elements; grad_w = g^T . x over no rows and grad_b = the column sum of no rows are
-zero.  With k = 0 the product is empty and y is the bias.  Checked against the oracle's forward /
+zero.  With n = 0, grad_x = g . w over no columns is zero and y, grad_w, grad_b have no
+elements.  With k = 0 the product is empty and y is the bias.  Checked against the oracle's forward /
 backward on the same tensors: every ring state and step bit-exact, grad_w and grad_b exactly zero,
 y exactly the bias, for the pages' split, the row-major and transposed compositions, the
 pre-quantized-operand backward and dynamic scaling.
@@ -59,10 +61,11 @@ def _out(shape, dtype=torch.bfloat16):
         torch.full(shape, 0xA5, dtype=dtype, device=DEV)
 
 
+@pytest.mark.parametrize("mkn", [(0, 256, 384), (256, 128, 0)])
 @pytest.mark.parametrize("path", ["split", "rowmajor", "transposed", "prequant"])
-def test_no_rows_delayed(path):
-    m, k, n = 0, 256, 384
-    t, d, bits, (xr, wr, gr), (oxr, owr, ogr) = _setup(m, k, n, 9100)
+def test_empty_batch_delayed(path, mkn):
+    m, k, n = mkn
+    t, d, bits, (xr, wr, gr), (oxr, owr, ogr) = _setup(m, k, n, 9100 + n)
     steps = torch.zeros(3, device=DEV)
     y = _out((m, n))
     gx, gw, gb = _out((m, k)), _out((n, k)), _out((n,))
@@ -105,8 +108,12 @@ def test_no_rows_delayed(path):
     assert (steps[0].item(), steps[1].item(), steps[2].item()) == (f["sx"], f["sw"], r["sg"])
     for dev_r, ora_r in ((xr, oxr), (wr, owr), (gr, ogr)):
         assert np.array_equal(_bits(dev_r), ora_r.state.view(np.uint32))
-    assert _zeros_bits(gw) and _zeros_bits(gb)  # the sums over no rows
-    assert not np.abs(r["dw"]).any() and not np.abs(r["grad_b"]).any()
+    if m == 0:  # the sums over no rows
+        assert _zeros_bits(gw) and _zeros_bits(gb)
+        assert not np.abs(r["dw"]).any() and not np.abs(r["grad_b"]).any()
+    if n == 0:  # the sum over no columns
+        assert _zeros_bits(gx)
+        assert not np.abs(r["dx"]).any()
 
 
 def test_no_rows_dynamic():
