@@ -1444,7 +1444,8 @@ int gemm_entry(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8_fmt_t fm
     if (m < 0 || n < 0 || k < 0 || batch < 0) return fail(FP8DSA_ERR_INVALID_ARG, "negative size");
     if (m > 0x7FFFFFFF || n > 0x7FFFFFFF || k > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "sizes must be < 2^31");
     if (batch > 0x7FFFFFFF) return fail(FP8DSA_ERR_UNSUPPORTED, "batch must be < 2^31");
-    if ((out == nullptr && out8 == nullptr) || scale_a == nullptr || scale_b == nullptr)
+    const bool empty_out = m == 0 || n == 0 || batch == 0;  // an output without elements may be NULL
+    if ((out == nullptr && out8 == nullptr && !empty_out) || scale_a == nullptr || scale_b == nullptr)
         return fail(FP8DSA_ERR_INVALID_ARG, "an output, scale_a and scale_b are required");
     if (bias == nullptr && bias_scale != nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "bias_scale without bias");
     if (ldo < n) return fail(FP8DSA_ERR_INVALID_ARG, "ldo must be >= n");
@@ -1492,7 +1493,8 @@ extern "C" int fp8_gemm(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt_a, fp8
                         const float* scale_b, const void* bias, const float* bias_scale, void* out,
                         cudaStream_t stream) {
     clear_error();
-    if (out == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out, scale_a and scale_b are required");
+    if (out == nullptr && m > 0 && n > 0 && batch > 0)
+        return fail(FP8DSA_ERR_INVALID_ARG, "out, scale_a and scale_b are required");
     return gemm_entry(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o, scale_a,
                       scale_b, bias, bias_scale, out, FP8_E4M3, nullptr, nullptr, nullptr, nullptr, stream);
 }
@@ -1504,7 +1506,7 @@ extern "C" int fp8_gemm_fp8out(const uint8_t* a, const uint8_t* b, fp8_fmt_t fmt
                                const float* bias_scale, void* out, fp8_fmt_t out8_fmt, const float* out8_step,
                                uint8_t* out8, float* out8_amax, float* out8_step_used, cudaStream_t stream) {
     clear_error();
-    if (out8 == nullptr) return fail(FP8DSA_ERR_INVALID_ARG, "out8 is required");
+    if (out8 == nullptr && m > 0 && n > 0 && batch > 0) return fail(FP8DSA_ERR_INVALID_ARG, "out8 is required");
     return gemm_entry(a, b, fmt_a, fmt_b, layout, m, n, k, lda, ldb, ldo, batch, stride_a, stride_b, stride_o, scale_a,
                       scale_b, bias, bias_scale, out, out8_fmt, out8_step, out8, out8_amax, out8_step_used, stream);
 }

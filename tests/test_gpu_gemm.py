@@ -138,8 +138,12 @@ def test_empty_m_n_are_noops():
     out = torch.full((16,), 7, dtype=torch.int16, device=DEV)
     one = torch.ones(1, device=DEV)
     F.fp8_gemm(None, None, 0, 0, 0, 0, 16, 16, 16, 16, 16, 1, 0, 0, 0, one, one, None, None, out)
+    # an output without elements may be NULL (m = 0, n = 0 or batch = 0)
+    F.fp8_gemm(None, None, 0, 0, 0, 0, 16, 16, 16, 16, 16, 1, 0, 0, 0, one, one, None, None, None)
+    F.fp8_gemm(None, None, 0, 0, 0, 16, 0, 16, 16, 16, 16, 1, 0, 0, 0, one, one, None, None, None)
     torch.cuda.synchronize()
     assert int(out[0]) == 7
+    assert F.fp8_get_device_status() == 0
 
 
 def test_accumulation_precision_k_sweep():
