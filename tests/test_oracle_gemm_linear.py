@@ -449,3 +449,39 @@ def test_backward_prequant_equals_exact_brute_force():
             for j in range(k):
                 exact = sum(gs[p][i] * xs[p][j] for p in range(m)) * sc_w
                 assert abs(Fraction(out["dw"][i, j]) - exact) <= Fraction(2) ** -45 * Fraction(float(out["dw_abs"][i, j])) * sc_w
+
+
+def _bf16_bits(rng, shape, sd):
+    """bf16 bit patterns of N(0, sd) samples (truncated fp32)."""
+    v = (rng.standard_normal(shape) * sd).astype(np.float32)
+    return (v.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_empty_batch_follows_the_definition():
+    """No rows: amax of nothing is 0 (the ring records 0 and, from a window of zeros, publishes the
+    1e-12 floor of the formula), grad_w and grad_b are sums over no rows (0); no output columns:
+    grad_x is a sum over no columns (0); no inner dimension: y is the bias."""
+    rng = np.random.default_rng(5)
+    k, n = 64, 48
+    x = np.zeros((0, k), dtype=np.uint16)
+    g = np.zeros((0, n), dtype=np.uint16)
+    w = _bf16_bits(rng, (n, k), 0.02)
+    b = _bf16_bits(rng, (n,), 0.1)
+    rx, rw, rg = S.Ring(4, "e4m3"), S.Ring(4, "e4m3"), S.Ring(4, "e5m2")
+    rx.seed(np.zeros((0, k), np.float32))
+    rw.seed(C.bf16_bits_to_f64(w).astype(np.float32))
+    rg.seed(np.zeros((0, n), np.float32))
+    assert rx.scale == np.float32(1e-12) and rg.scale == np.float32(1e-12)
+    f = L.forward(x, w, b, "e4m3", rx, rw)
+    assert f["y"].shape == (0, n) and f["amax_x"] == 0.0
+    assert rx.state[0] == 0.0 and rx.state[4] == np.float32(1e-12)  # hist[idx] = 0; the floor
+    r = L.backward(g, x, w, "e5m2", f["sx"], f["sw"], rg)
+    assert r["dx"].shape == (0, k) and r["dw"].shape == (n, k)
+    assert not r["dw"].any() and not r["grad_b"].any() and r["amax_g"] == 0.0
+    # no output columns: grad_x = g . w over nothing
+    x2 = _bf16_bits(rng, (32, k), 1.0)
+    r2 = L.backward(np.zeros((32, 0), np.uint16), x2, np.zeros((0, k), np.uint16), "e5m2", 1.0, 1.0)
+    assert r2["dx"].shape == (32, k) and not r2["dx"].any() and r2["dw"].shape == (0, k)
+    # no inner dimension: y[i][j] = bias[j]
+    f3 = L.forward(np.zeros((32, 0), np.uint16), np.zeros((n, 0), np.uint16), b, "e4m3")
+    assert np.array_equal(f3["y"], np.broadcast_to(C.bf16_bits_to_f64(b), (32, n)))
