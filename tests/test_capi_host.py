@@ -280,30 +280,34 @@ def test_misc_argument_checks():
 
 
 def test_empty_tensors_may_be_null():
-    """A tensor without elements may come as NULL (an empty framework tensor has no storage):
-    such calls pass every argument check and only then need the device (CUDA_ERROR here, with
-    no GPU), while a NULL tensor that has elements is still INVALID_ARG."""
-    CUDA = -3
+    """A tensor without elements may come as NULL (an empty framework tensor has no storage).
+    Each call below stops at a later argument check that fails before any CUDA call (a
+    misaligned workspace, or ldo < n), which proves the NULL passed the pointer checks; a NULL
+    tensor that has elements is still INVALID_ARG with the pointer message.  No call reaches the
+    device, so this is safe with or without a GPU."""
     lib = F.lib()
     f = lib.linear_forward_fp8
-    ws = F.linear_forward_fp8_workspace_size(0, 64, 64)
-    # m = 0: x and y empty
-    assert f(None, 256, 0, None, None, None, 0, 64, 64, 0, None, None, 1.0, None, None, 1024, ws, None, None) == CUDA
+    ws = F.linear_forward_fp8_workspace_size(64, 64, 64)
+    # m = 0: x and y empty; the misaligned workspace is what fails
+    assert f(None, 256, 0, None, None, None, 0, 64, 64, 0, None, None, 1.0, None, None, 1040, ws, None, None) == UNSUPPORTED
     # m > 0: x is required
-    assert f(None, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 1024,
-             F.linear_forward_fp8_workspace_size(64, 64, 64), 2048, None) == INVALID
+    assert f(None, 256, 0, None, None, None, 64, 64, 64, 0, None, None, 1.0, None, None, 1040, ws, 2048, None) == INVALID
     b = lib.linear_backward_fp8
-    wsb = F.linear_backward_fp8_workspace_size(0, 64, 64)
+    wsb = F.linear_backward_fp8_workspace_size(64, 64, 64)
     # m = 0: g, x and grad_x empty; w, grad_w and grad_b still have elements
-    assert b(None, None, 256, 0, 64, 64, 1, 1, 1, 1, None, None, None, 1.0, None, 1024, wsb, None, 4096, 4096,
-             None) == CUDA
+    assert b(None, None, 256, 0, 64, 64, 1, 1, 1, 1, None, None, None, 1.0, None, 1040, wsb, None, 4096, 4096,
+             None) == UNSUPPORTED
     # n = 0: g, w, grad_w and grad_b empty
-    wsb0 = F.linear_backward_fp8_workspace_size(64, 64, 0)
-    assert b(None, 256, None, 64, 64, 0, 1, 1, 1, 1, None, None, None, 1.0, None, 1024, wsb0, 4096, None, None,
-             None) == CUDA
-    # a GEMM output without elements
+    assert b(None, 256, None, 64, 64, 0, 1, 1, 1, 1, None, None, None, 1.0, None, 1040, wsb, 4096, None, None,
+             None) == UNSUPPORTED
+    # m > 0 and n > 0: g is required
+    assert b(None, 256, 256, 64, 64, 64, 1, 1, 1, 1, None, None, None, 1.0, None, 1040, wsb, 4096, 4096, 4096,
+             None) == INVALID
+    # a GEMM output without elements: the NULL out passes, ldo < n fails
     one = 512
-    assert lib.fp8_gemm(None, None, 0, 0, 0, 0, 16, 16, 16, 16, 16, 1, 0, 0, 0, one, one, None, None, None,
-                        None) == CUDA
+    assert lib.fp8_gemm(None, None, 0, 0, 0, 0, 16, 16, 16, 16, 8, 1, 0, 0, 0, one, one, None, None, None,
+                        None) == INVALID
+    assert "ldo" in F.last_error()
     assert lib.fp8_gemm(None, None, 0, 0, 0, 16, 16, 16, 16, 16, 16, 1, 0, 0, 0, one, one, None, None, None,
                         None) == INVALID
+    assert "out" in F.last_error()
